@@ -1,0 +1,348 @@
+/*
+ * awq_oracle.c -- plain, slow CPU oracle for the AWQ INT4 hot path.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only tests/, __graft_entry__.smoke() and the
+ * cpu_baseline / reference legs of bench.py may load this code.  It shares no
+ * source, header, table or helper with the CUDA library, and the CUDA library
+ * never calls it.
+ *
+ * What it computes (sources, by page and section):
+ *   [P1] "From-Scratch AWQ INT4 Quantization on Qwen3-8B", sections
+ *        "AWQ scaling", "Group-wise symmetric INT4",
+ *        "AutoAWQ / HF-AWQ GEMM on-disk format" and exporter step 4.
+ *   [P3] "AWQ architecture, in depth: ...", sections "The scale search as
+ *        code" and "Quantization, storage and packing".
+ *   [P4] "Weight-Only Quantization: GPTQ and AWQ", section 4 "Tiny example"
+ *        and sections 6-9 "Under the hood: the packed format".
+ *
+ * Precision (readings are listed in the design doc):
+ *   - every decision that produces an integer (a code, the group scale, the
+ *     chosen grid index) is taken in fp32 with IEEE round-to-nearest-even,
+ *     the group scale then rounded to fp16 (round-to-nearest-even);
+ *   - the activation mean is the exact real mean, rounded once to fp64 and
+ *     then to fp32;
+ *   - the scale table is computed in fp64 and rounded once to fp32;
+ *   - error sums are the exact weighted squared error of those fp32
+ *     decisions, evaluated in fp64.
+ * Build with -O2 -ffp-contract=off and without -ffast-math.
+ *
+ * Parity pins: every function here is pinned by tests/test_oracle_pins.py
+ * (worked example, closed forms, special cases, brute force); none is
+ * "parity unpinned" except the claim that the packed words load in the
+ * third-party AutoAWQ runtime, which is not present here.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORC_SCALE_FP32 1   /* flag: keep the group scale unrounded (fp32) */
+
+/* ---------------------------------------------------------------- fp16 -- */
+
+static float h2f(uint16_t h)
+{
+    _Float16 v;
+    memcpy(&v, &h, sizeof v);
+    return (float)v;
+}
+
+static uint16_t f2h(float f)
+{
+    _Float16 v = (_Float16)f;          /* IEEE round-to-nearest-even */
+    uint16_t h;
+    memcpy(&h, &v, sizeof h);
+    return h;
+}
+
+/* ------------------------------------------------------ activation stats --
+ * x[j] = mean over tokens of |X[t, j]|        ([P1] "AWQ scaling";
+ * [P3] "The scale search as code": x.abs().float().mean(dim=0)).
+ *
+ * Every |fp16| value is an integer multiple of 2^-24 below 2^16, so the sum
+ * is accumulated exactly as an integer count of 2^-24 units.  A column that
+ * holds an infinity gets +inf; one that holds a NaN gets NaN.
+ */
+void orc_act_stats(const uint16_t *X, int64_t T, int64_t d_in, int64_t ld,
+                   float *x)
+{
+    for (int64_t j = 0; j < d_in; ++j) {
+        int64_t units = 0;          /* sum of |X[t,j]| in units of 2^-24 */
+        int saw_inf = 0, saw_nan = 0;
+        for (int64_t t = 0; t < T; ++t) {
+            float v = fabsf(h2f(X[t * ld + j]));
+            if (isnan(v)) { saw_nan = 1; continue; }
+            if (isinf(v)) { saw_inf = 1; continue; }
+            units += (int64_t)ldexp((double)v, 24);   /* exact integer */
+        }
+        if (saw_nan)
+            x[j] = NAN;
+        else if (saw_inf)
+            x[j] = INFINITY;
+        else
+            x[j] = (float)(ldexp((double)units, -24) / (double)T);
+    }
+}
+
+/* ----------------------------------------------------------- scale table --
+ * For grid index i (alpha = i / n_grid, [P3] "The scale search as code"):
+ *   s_i[j] = max(x[j], 1e-4) ^ alpha
+ *   s_i    = s_i / sqrt(max_j s_i[j] * min_j s_i[j])
+ * The clamp sits on x before the power (the stated method); the power and the
+ * normalisation are done in fp64 and rounded once to fp32.
+ */
+void orc_scale_table(const float *x, int64_t d_in, int n_grid, float *S)
+{
+    double *sd = (double *)malloc((size_t)d_in * sizeof(double));
+    for (int i = 0; i < n_grid; ++i) {
+        double alpha = (double)i / (double)n_grid;
+        double mx = -INFINITY, mn = INFINITY;
+        for (int64_t j = 0; j < d_in; ++j) {
+            float xc = fmaxf(x[j], 1e-4f);
+            sd[j] = pow((double)xc, alpha);
+            if (sd[j] > mx) mx = sd[j];
+            if (sd[j] < mn) mn = sd[j];
+        }
+        double norm = sqrt(mx * mn);
+        for (int64_t j = 0; j < d_in; ++j)
+            S[(int64_t)i * d_in + j] = (float)(sd[j] / norm);
+    }
+    free(sd);
+}
+
+/* ----------------------------------------------- group fake-quantisation --
+ * One group of n consecutive input channels of one output row
+ * ([P1] "Group-wise symmetric INT4"):
+ *   ws[j]   = w[j] * s[j]                         (fp32)
+ *   q_scale = max_j |ws[j]| / 7                   (fp32, then fp16 RNE
+ *                                                  unless ORC_SCALE_FP32)
+ *   q[j]    = clamp(rint(ws[j] / q_scale), -7, 7) (rint = half to even)
+ * An all-zero group has q_scale = 0 and all codes 0.  A q_scale that
+ * overflows fp16 is held at the largest finite fp16 value, 65504.
+ * Returns 0, or 1 when the group holds a non-finite value (codes then 0 and
+ * q_scale NaN).
+ */
+int orc_fake_quant_group(const float *w, const float *s, int64_t n, int flags,
+                         int8_t *q, float *q_scale)
+{
+    float m = 0.0f;
+    int nonfinite = 0;
+    for (int64_t j = 0; j < n; ++j) {
+        float ws = w[j] * s[j];
+        if (!isfinite(ws)) nonfinite = 1;
+        float a = fabsf(ws);
+        if (a > m) m = a;
+    }
+    if (nonfinite) {
+        for (int64_t j = 0; j < n; ++j) q[j] = 0;
+        *q_scale = NAN;
+        return 1;
+    }
+    float qs = m / 7.0f;
+    if (!(flags & ORC_SCALE_FP32)) {
+        qs = h2f(f2h(qs));
+        if (isinf(qs)) qs = 65504.0f;
+    }
+    for (int64_t j = 0; j < n; ++j) {
+        if (qs == 0.0f) { q[j] = 0; continue; }
+        float ws = w[j] * s[j];
+        float r = rintf(ws / qs);
+        if (r > 7.0f) r = 7.0f;
+        if (r < -7.0f) r = -7.0f;
+        q[j] = (int8_t)r;
+    }
+    *q_scale = qs;
+    return 0;
+}
+
+/* ------------------------------------------------- weight-space scoring --
+ * Activation-weighted reconstruction error of one candidate scale vector s
+ * over one weight matrix W[d_out, d_in] (fp16, row-major)
+ * ([P1] "AWQ scaling"):
+ *     sum_{r,j} ( (W[r,j] - q[r,j] * q_scale[r,g(j)] / s[j]) * x[j] )^2
+ * evaluated in fp64 from the fp32 decisions.  Returns NaN when any group is
+ * non-finite.
+ */
+double orc_weighted_error(const uint16_t *W, int64_t d_out, int64_t d_in,
+                          const float *x, const float *s, int64_t g, int flags)
+{
+    /* one partial per row, summed afterwards in row order, so the result
+     * does not depend on how many threads ran the rows */
+    double *row_err = (double *)malloc((size_t)d_out * sizeof(double));
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < d_out; ++r) {
+        float w[g];
+        int8_t q[g];
+        double acc = 0.0;
+        for (int64_t k = 0; k < d_in / g; ++k) {
+            const uint16_t *row = W + r * d_in + k * g;
+            for (int64_t j = 0; j < g; ++j) w[j] = h2f(row[j]);
+            float qs;
+            if (orc_fake_quant_group(w, s + k * g, g, flags, q, &qs)) {
+                acc = NAN;
+                continue;
+            }
+            for (int64_t j = 0; j < g; ++j) {
+                double what = (double)q[j] * (double)qs / (double)s[k * g + j];
+                double e = ((double)w[j] - what) * (double)x[k * g + j];
+                acc += e * e;
+            }
+        }
+        row_err[r] = acc;
+    }
+    double total = 0.0;
+    for (int64_t r = 0; r < d_out; ++r) total += row_err[r];
+    free(row_err);
+    return total;
+}
+
+/* ---------------------------------------------------------- scale search --
+ * [P3] "The scale search as code" + [P1] "AWQ scaling": for every grid
+ * index i the error of every weight segment that shares the input x is
+ * summed; the first index with the smallest error wins (strict '<', so the
+ * smallest alpha wins a tie).  s_best receives that row of the scale table.
+ * best = -1 (and s_best NaN) when any error is not finite.
+ */
+void orc_scale_search(int n_seg, const uint16_t *const *W, const int64_t *d_out,
+                      int64_t d_in, const float *x, int64_t g, int n_grid,
+                      int flags, double *err, int32_t *best, float *s_best)
+{
+    float *S = (float *)malloc((size_t)n_grid * (size_t)d_in * sizeof(float));
+    orc_scale_table(x, d_in, n_grid, S);
+    for (int i = 0; i < n_grid; ++i) {
+        double e = 0.0;
+        for (int k = 0; k < n_seg; ++k)
+            e += orc_weighted_error(W[k], d_out[k], d_in, x,
+                                    S + (int64_t)i * d_in, g, flags);
+        err[i] = e;
+    }
+    int b = 0;
+    int finite = 1;
+    for (int i = 0; i < n_grid; ++i) {
+        if (!isfinite(err[i])) finite = 0;
+        if (err[i] < err[b]) b = i;
+    }
+    if (!finite) {
+        *best = -1;
+        for (int64_t j = 0; j < d_in; ++j) s_best[j] = NAN;
+    } else {
+        *best = b;
+        memcpy(s_best, S + (int64_t)b * d_in, (size_t)d_in * sizeof(float));
+    }
+    free(S);
+}
+
+/* ----------------------------------------------------- quantise and pack --
+ * AutoAWQ GEMM layout ([P1] "AutoAWQ / HF-AWQ GEMM on-disk format" and
+ * exporter step 4; [P3] "Quantization, storage and packing"):
+ *   u[r,j]          = q[r,j] + zero_point      (unsigned code)
+ *   qweight[j, c]   = int32 whose nibble p (bits 4p..4p+3) holds
+ *                     u[8c + order[p], j],  order = {0,2,4,6,1,3,5,7}
+ *   scales[k, r]    = fp16 group scale of row r, group k
+ *   qzeros[k, c]    = zero_point in all eight nibbles
+ * s == NULL means s = 1 (plain round-to-nearest).  A non-finite group stores
+ * code zero_point and scale NaN.
+ */
+static const int kOrder[8] = {0, 2, 4, 6, 1, 3, 5, 7};
+
+void orc_quantize_pack(const uint16_t *W, int64_t d_out, int64_t d_in,
+                       const float *s, int64_t g, int zero_point,
+                       int32_t *qweight, uint16_t *scales, int32_t *qzeros)
+{
+    int64_t G = d_in / g, C = d_out / 8;
+    uint8_t *u = (uint8_t *)malloc((size_t)d_out * (size_t)d_in);
+    float *w = (float *)malloc((size_t)g * sizeof(float));
+    float *ones = (float *)malloc((size_t)g * sizeof(float));
+    int8_t *q = (int8_t *)malloc((size_t)g);
+    for (int64_t j = 0; j < g; ++j) ones[j] = 1.0f;
+
+    for (int64_t r = 0; r < d_out; ++r) {
+        for (int64_t k = 0; k < G; ++k) {
+            for (int64_t j = 0; j < g; ++j) w[j] = h2f(W[r * d_in + k * g + j]);
+            float qs;
+            orc_fake_quant_group(w, s ? s + k * g : ones, g, 0, q, &qs);
+            scales[k * d_out + r] = isnan(qs) ? (uint16_t)0x7E00 : f2h(qs);
+            for (int64_t j = 0; j < g; ++j)
+                u[r * d_in + k * g + j] = (uint8_t)(q[j] + zero_point);
+        }
+    }
+    for (int64_t j = 0; j < d_in; ++j) {
+        for (int64_t c = 0; c < C; ++c) {
+            uint32_t word = 0;
+            for (int p = 0; p < 8; ++p)
+                word |= (uint32_t)(u[(8 * c + kOrder[p]) * d_in + j] & 0xF)
+                        << (4 * p);
+            qweight[j * C + c] = (int32_t)word;
+        }
+    }
+    uint32_t zword = 0;
+    for (int p = 0; p < 8; ++p) zword |= (uint32_t)(zero_point & 0xF) << (4 * p);
+    for (int64_t k = 0; k < G; ++k)
+        for (int64_t c = 0; c < C; ++c) qzeros[k * C + c] = (int32_t)zword;
+    free(u);
+    free(w);
+    free(ones);
+    free(q);
+}
+
+/* Inverse of the packing above: codes u[r, j] (unsigned, 0..15). */
+void orc_unpack(const int32_t *qweight, int64_t d_out, int64_t d_in,
+                uint8_t *u)
+{
+    int64_t C = d_out / 8;
+    for (int64_t j = 0; j < d_in; ++j)
+        for (int64_t c = 0; c < C; ++c) {
+            uint32_t word = (uint32_t)qweight[j * C + c];
+            for (int p = 0; p < 8; ++p)
+                u[(8 * c + kOrder[p]) * d_in + j] = (uint8_t)((word >> (4 * p)) & 0xF);
+        }
+}
+
+/* ------------------------------------------------ output-space scoring --
+ * Optional scoring mode ([P3] "The scale search as code": the group output
+ * compared with the full-precision output; [P4] section 2: the output error
+ * is X (W - W_hat)):
+ *     err[i] = || X (W - W_hat_i)^T ||_F^2
+ * with W_hat_i = Q(W * s_i) / s_i from the same group fake-quantisation, in
+ * fp64.  X is fp16 [T, d_in] row-major, W fp16 [d_out, d_in].
+ */
+void orc_output_error(const uint16_t *X, int64_t T, const uint16_t *W,
+                      int64_t d_out, int64_t d_in, const float *x, int64_t g,
+                      int n_grid, int flags, double *err)
+{
+    float *S = (float *)malloc((size_t)n_grid * (size_t)d_in * sizeof(float));
+    double *dW = (double *)malloc((size_t)d_out * (size_t)d_in * sizeof(double));
+    double *Xd = (double *)malloc((size_t)T * (size_t)d_in * sizeof(double));
+    float *w = (float *)malloc((size_t)g * sizeof(float));
+    int8_t *q = (int8_t *)malloc((size_t)g);
+    orc_scale_table(x, d_in, n_grid, S);
+    for (int64_t t = 0; t < T * d_in; ++t) Xd[t] = (double)h2f(X[t]);
+
+    for (int i = 0; i < n_grid; ++i) {
+        const float *s = S + (int64_t)i * d_in;
+        int bad = 0;
+        for (int64_t r = 0; r < d_out; ++r)
+            for (int64_t k = 0; k < d_in / g; ++k) {
+                for (int64_t j = 0; j < g; ++j) w[j] = h2f(W[r * d_in + k * g + j]);
+                float qs;
+                if (orc_fake_quant_group(w, s + k * g, g, flags, q, &qs)) bad = 1;
+                for (int64_t j = 0; j < g; ++j)
+                    dW[r * d_in + k * g + j] =
+                        (double)w[j] - (double)q[j] * (double)qs / (double)s[k * g + j];
+            }
+        double total = 0.0;
+        for (int64_t t = 0; t < T; ++t)
+            for (int64_t r = 0; r < d_out; ++r) {
+                double y = 0.0;
+                for (int64_t j = 0; j < d_in; ++j)
+                    y += Xd[t * d_in + j] * dW[r * d_in + j];
+                total += y * y;
+            }
+        err[i] = bad ? NAN : total;
+    }
+    free(S);
+    free(dW);
+    free(Xd);
+    free(w);
+    free(q);
+}

@@ -1,0 +1,345 @@
+"""Pins of the CPU oracle against what the pages and the mathematics fix.
+
+Each test checks the oracle against something other than itself: a worked
+example printed on a page, a closed form, a special case that reduces to a
+textbook routine, an invariant, or brute force on tiny inputs.  No expected
+value here comes from the CUDA path.
+"""
+import itertools
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+
+
+def _floats(s):
+    return [float(v) for v in s.split()]
+
+
+def _nearest_level(v):
+    """Nearest integer in [-7, 7] to the fp32 quotient v, ties to even --
+    found by enumerating the 15 levels (not by calling a rounding routine)."""
+    v = float(v)
+    return min(range(-7, 8), key=lambda q: (abs(v - q), q % 2))
+
+
+# ---------------------------------------------------------------- worked --
+# "Weight-Only Quantization: GPTQ and AWQ", section 4 "Tiny example".
+
+def test_worked_example_fp32_scale(golden):
+    g = golden("worked_example.txt")
+    w = np.array(_floats(g["w"]), np.float32)
+    x = np.array(_floats(g["x"]), np.float64)
+    sc = np.array(_floats(g["awq_scale"]), np.float32)
+    wd = w.astype(np.float64)
+
+    assert round(float(wd @ x), 3) == float(g["exact_dot"])
+
+    qn, qs_n, bad = oracle.fake_quant_group(w, np.ones(4, np.float32), oracle.SCALE_FP32)
+    assert not bad
+    assert list(qn) == [4, -3, 7, 1]
+    naive = qn.astype(np.float64) * qs_n
+    assert np.allclose(np.round(naive, 3), _floats(g["naive_deq"]), atol=0)
+    assert round(float(naive @ x), 3) == float(g["naive_dot"])
+
+    qa, qs_a, bad = oracle.fake_quant_group(w, sc, oracle.SCALE_FP32)
+    assert list(qa) == [7, -1, 3, 0]
+    awq = qa.astype(np.float64) * qs_a / sc.astype(np.float64)
+    assert np.allclose(np.round(awq, 3), _floats(g["awq_deq"]), atol=0)
+    assert round(float(awq @ x), 3) == float(g["awq_dot"])
+
+    exact = float(wd @ x)
+    assert round(abs(exact - float(naive @ x)), 2) == float(g["naive_error"])
+    assert round(abs(exact - float(awq @ x)), 3) == float(g["awq_error"])
+
+
+def test_worked_example_codes_fp16_scale(golden):
+    """The INT4 codes of the example do not depend on rounding q_scale to fp16."""
+    g = golden("worked_example.txt")
+    w = np.array(_floats(g["w"]), np.float32)
+    sc = np.array(_floats(g["awq_scale"]), np.float32)
+    qn, qs_n, _ = oracle.fake_quant_group(w, np.ones(4, np.float32), 0)
+    qa, qs_a, _ = oracle.fake_quant_group(w, sc, 0)
+    assert list(qn) == [4, -3, 7, 1] and list(qa) == [7, -1, 3, 0]
+    # the fp16 group scale is the fp16 value nearest to max|ws| / 7
+    assert qs_n == float(np.float16(np.float32(0.8) / np.float32(7)))
+    assert qs_a == float(np.float16(np.float32(2.0) / np.float32(7)))
+
+
+def test_weighted_error_of_worked_example():
+    """Weight-space score of the example = sum ((w - w_hat) x)^2, by hand."""
+    w = np.array([[0.5, -0.3, 0.8, 0.1]], np.float16)
+    x = np.array([10, 0.1, 0.1, 0.1], np.float32)
+    s = np.array([4, 1, 1, 1], np.float32)
+    e = oracle.weighted_error(w, x, s, 4, oracle.SCALE_FP32)
+    wf = w.astype(np.float32)[0]
+    qs = float(np.float32(abs(wf[0] * 4)) / np.float32(7))
+    codes = [7, -1, 3, 0]
+    hand = sum(((float(wf[j]) - codes[j] * qs / float(s[j])) * float(x[j])) ** 2
+               for j in range(4))
+    assert e == pytest.approx(hand, rel=1e-12)
+
+
+# ------------------------------------------------------------- rounding --
+
+@pytest.mark.parametrize("w1,code", [(0.3125, 2), (0.4375, 4), (-0.3125, -2),
+                                     (-0.4375, -4), (0.0625, 0), (0.1875, 2)])
+def test_rint_ties_to_even(w1, code):
+    """Exact half-way quotients round to the even level (round / rint)."""
+    w = np.array([0.875, w1], np.float32)     # q_scale = 0.875 / 7 = 0.125 exactly
+    q, qs, _ = oracle.fake_quant_group(w, np.ones(2, np.float32), 0)
+    assert qs == 0.125
+    assert q[1] == code
+
+
+def test_codes_are_nearest_level_bruteforce():
+    rng = np.random.default_rng(11)
+    for trial in range(200):
+        n = 32
+        w = (rng.standard_normal(n) * 0.02).astype(np.float16).astype(np.float32)
+        s = np.exp(rng.standard_normal(n)).astype(np.float32)
+        q, qs, _ = oracle.fake_quant_group(w, s, 0)
+        ws = (w * s).astype(np.float32)
+        m = float(np.max(np.abs(ws)))
+        assert qs == float(np.float16(np.float32(m) / np.float32(7)))
+        for j in range(n):
+            quot = np.float32(ws[j]) / np.float32(qs)
+            assert q[j] == _nearest_level(quot)
+
+
+def test_dequant_error_within_half_step():
+    """|w s - q q_scale| <= q_scale / 2 for every weight that is not clamped
+    ("up to s/2 per weight", section 2 of the GPTQ/AWQ tutorial page)."""
+    rng = np.random.default_rng(12)
+    for _ in range(100):
+        w = (rng.standard_normal(128) * 0.02).astype(np.float16).astype(np.float32)
+        s = np.exp(rng.standard_normal(128) * 2).astype(np.float32)
+        q, qs, _ = oracle.fake_quant_group(w, s, 0)
+        ws = (w * s).astype(np.float64)
+        err = np.abs(ws - q.astype(np.float64) * qs)
+        unclamped = np.abs(q) < 7
+        assert np.all(err[unclamped] <= qs / 2 * (1 + 1e-6))
+        # a clamped code only occurs at the group maximum
+        assert np.all(np.abs(ws[~unclamped]) >= 6.5 * qs)
+
+
+def test_zero_group_and_fp16_overflow():
+    q, qs, bad = oracle.fake_quant_group(np.zeros(8, np.float32), np.ones(8, np.float32), 0)
+    assert qs == 0.0 and not bad and not q.any()
+    big = np.array([1e6, -3e5, 1.0, 0.0], np.float32)
+    q, qs, _ = oracle.fake_quant_group(big, np.ones(4, np.float32), 0)
+    assert qs == 65504.0              # held at the largest finite fp16
+    assert q[0] == 7 and q[1] == -5   # 1e6/65504 = 15.3 -> clamped to 7
+    q, qs, bad = oracle.fake_quant_group(np.array([1, np.nan], np.float32),
+                                         np.ones(2, np.float32), 0)
+    assert bad and math.isnan(qs)
+
+
+# ---------------------------------------------------------- scale table --
+
+def test_scale_table_closed_form_two_levels():
+    """x taking two values a (first half) and b: s_i = (a/b)^(+-alpha/2)."""
+    a, b = np.float32(7.5), np.float32(0.03)
+    x = np.array([a] * 8 + [b] * 8, np.float32)
+    S = oracle.scale_table(x, 20)
+    for i in range(20):
+        al = i / 20
+        hi = (float(a) / float(b)) ** (al / 2)
+        assert S[i, 0] == np.float32(hi)
+        assert S[i, 15] == np.float32(1.0 / hi)
+
+
+def test_scale_table_alpha0_is_one_and_normalised():
+    rng = np.random.default_rng(3)
+    x = np.exp(rng.standard_normal(512) * 2).astype(np.float32)
+    x[5] = 0.0          # clamped to 1e-4 before the power
+    x[6] = 1e-4
+    S = oracle.scale_table(x, 20)
+    assert np.all(S[0] == 1.0)
+    assert np.all(S[:, 5] == S[:, 6])
+    for i in range(20):
+        assert float(S[i].max()) * float(S[i].min()) == pytest.approx(1.0, rel=1e-6)
+        # s is monotone in x for alpha > 0
+        if i:
+            order = np.argsort(np.maximum(x, np.float32(1e-4)), kind="stable")
+            assert np.all(np.diff(S[i][order]) >= 0)
+
+
+# ----------------------------------------------------------------- stats --
+
+def test_act_stats_closed_form():
+    T, d = 3, 4
+    X = np.array([[1, -2, 0.5, 0], [-1, 2, 0.25, 0], [1, -2, -0.25, 1]], np.float16)
+    x = oracle.act_stats(X)
+    assert list(x) == [1.0, 2.0, np.float32(1.0 / 3.0), np.float32(1.0 / 3.0)]
+    # the mean is exact: independent of token order, bit for bit
+    rng = np.random.default_rng(5)
+    Y = (rng.standard_normal((257, 64)) * np.exp(rng.standard_normal(64) * 3)).astype(np.float16)
+    ref = oracle.act_stats(Y)
+    for _ in range(3):
+        assert np.array_equal(oracle.act_stats(Y[rng.permutation(257)]), ref)
+    exact = [float(np.float32(sum(abs(float(v)) for v in Y[:, j]) / 257)) for j in range(64)]
+    # python sums in fp64 here; equal except where fp64 rounding of the sum matters
+    assert np.allclose(ref, exact, rtol=1e-7, atol=0)
+
+
+def test_act_stats_nonfinite():
+    X = np.ones((4, 3), np.float16)
+    X[1, 0] = np.inf
+    X[2, 1] = np.nan
+    x = oracle.act_stats(X)
+    assert x[0] == np.inf and math.isnan(x[1]) and x[2] == 1.0
+
+
+# ---------------------------------------------------------------- search --
+
+def test_alpha0_error_is_rtn_bruteforce():
+    """Grid index 0 gives s = 1, i.e. plain round-to-nearest; its error equals
+    a brute-force nearest-level quantisation scored by sum ((w - w_hat) x)^2.
+    The searched error is never above it ("AWQ scaling" section)."""
+    rng = np.random.default_rng(21)
+    d_out, d_in, g = 8, 64, 32
+    W = (rng.standard_normal((d_out, d_in)) * 0.02).astype(np.float16)
+    x = np.exp(rng.standard_normal(d_in)).astype(np.float32)
+    err, best, s_best = oracle.scale_search([W], x, g, 20)
+    Wf = W.astype(np.float32)
+    total = 0.0
+    for r in range(d_out):
+        for k in range(d_in // g):
+            grp = Wf[r, k * g:(k + 1) * g]
+            qs = float(np.float16(np.float32(np.max(np.abs(grp))) / np.float32(7)))
+            for j in range(g):
+                q = _nearest_level(np.float32(grp[j]) / np.float32(qs))
+                total += ((float(grp[j]) - q * qs) * float(x[k * g + j])) ** 2
+    assert err[0] == pytest.approx(total, rel=1e-12)
+    assert err[best] <= err[0]
+    assert err[best] == err.min() and best == int(np.argmin(err))
+
+
+def test_uniform_x_gives_ties_and_first_index():
+    """x constant => every s_i = 1 => all errors tie => index 0 wins."""
+    rng = np.random.default_rng(22)
+    W = (rng.standard_normal((16, 128)) * 0.02).astype(np.float16)
+    x = np.full(128, 3.0, np.float32)
+    err, best, s_best = oracle.scale_search([W], x, 128, 20)
+    assert np.all(err == err[0]) and best == 0 and np.all(s_best == 1.0)
+
+
+def test_shared_input_segments_add():
+    """A search over segments sharing x scores the sum of their errors
+    (the grid search concatenates the linears of a group on dim 0)."""
+    rng = np.random.default_rng(23)
+    W1 = (rng.standard_normal((16, 64)) * 0.02).astype(np.float16)
+    W2 = (rng.standard_normal((8, 64)) * 0.02).astype(np.float16)
+    x = np.exp(rng.standard_normal(64) * 2).astype(np.float32)
+    e12, b12, _ = oracle.scale_search([W1, W2], x, 32, 20)
+    ecat, bcat, _ = oracle.scale_search([np.concatenate([W1, W2])], x, 32, 20)
+    e1, _, _ = oracle.scale_search([W1], x, 32, 20)
+    e2, _, _ = oracle.scale_search([W2], x, 32, 20)
+    assert np.allclose(e12, e1 + e2, rtol=1e-12)
+    assert np.allclose(e12, ecat, rtol=1e-12) and b12 == bcat
+
+
+def test_salient_channel_search_beats_rtn():
+    """With one loud input channel the search picks alpha > 0 and lowers the
+    weighted error well below RTN (the effect the worked example shows)."""
+    rng = np.random.default_rng(24)
+    W = (rng.standard_normal((64, 128)) * 0.02).astype(np.float16)
+    x = np.full(128, 0.1, np.float32)
+    x[:2] = 10.0
+    err, best, _ = oracle.scale_search([W], x, 128, 20)
+    assert best > 0 and err[best] < 0.8 * err[0]
+
+
+# ------------------------------------------------------------------ pack --
+
+def _rows_with_codes(codes_per_row, width=32):
+    """fp16 rows whose group max sets q_scale = 0.125 and whose column 1 holds
+    the given signed code."""
+    W = np.zeros((len(codes_per_row), width), np.float16)
+    for r, q in enumerate(codes_per_row):
+        W[r, :] = np.float16(q * 0.125)
+        W[r, 0] = np.float16(-0.875)
+    return W
+
+
+def test_pack_order_golden(golden):
+    g = golden("pack_order.txt")
+    assert [int(v) for v in g["order"].split()] == [0, 2, 4, 6, 1, 3, 5, 7]
+    W = _rows_with_codes([r - 7 for r in range(8)])
+    qw, sc, qz = oracle.quantize_pack(W, None, 32, 8)
+    assert qw.shape == (32, 1) and sc.shape == (1, 8) and qz.shape == (1, 1)
+    assert np.uint32(qw[1, 0]) == int(g["word_rows_r_plus_1"], 16)
+    assert np.uint32(qw[0, 0]) == int(g["word_all_minus7"], 16)
+    assert np.uint32(qz[0, 0]) == int(g["qzeros_zp8"], 16)
+    assert np.all(sc == np.float16(0.125))
+    qw7, _, _ = oracle.quantize_pack(W, None, 32, 7)
+    assert np.uint32(qw7[1, 0]) == int(g["word_rows_r_zp7"], 16)
+
+
+@pytest.mark.parametrize("zp", [8, 7])
+def test_pack_roundtrip_and_zero_requant_error(zp):
+    """unpack(pack) returns the codes, and the runtime dequant (u - zero) * scale
+    equals the signed group dequant q * q_scale exactly (exporter step 4)."""
+    rng = np.random.default_rng(31)
+    d_out, d_in, g = 48, 256, 64
+    W = (rng.standard_normal((d_out, d_in)) * 0.02).astype(np.float16)
+    s = np.exp(rng.standard_normal(d_in)).astype(np.float32)
+    qw, sc, qz = oracle.quantize_pack(W, s, g, zp)
+    u = oracle.unpack(qw, d_out)
+    Wf = W.astype(np.float32)
+    for r in range(d_out):
+        for k in range(d_in // g):
+            q, qs, _ = oracle.fake_quant_group(Wf[r, k * g:(k + 1) * g], s[k * g:(k + 1) * g], 0)
+            assert np.array_equal(u[r, k * g:(k + 1) * g].astype(np.int32), q.astype(np.int32) + zp)
+            assert sc[k, r] == np.float16(qs)
+            deq_rt = (u[r, k * g:(k + 1) * g].astype(np.float64) - zp) * float(sc[k, r])
+            assert np.array_equal(deq_rt, q.astype(np.float64) * qs)
+    assert u.min() >= zp - 7 and u.max() <= zp + 7
+
+
+def test_bits_per_weight_and_stack_size():
+    """4 + 16/128 + 4/128 ~ 4.16 bits per weight at g128 (storage sections of
+    the architecture and tutorial pages); the Qwen3-8B linear stack is
+    13.9 GB in fp16 and its INT4 codes are 4.0x smaller (results section)."""
+    d_out, d_in, g = 64, 256, 128
+    W = np.zeros((d_out, d_in), np.float16)
+    qw, sc, qz = oracle.quantize_pack(W, None, g, 8)
+    bits = 8 * (qw.nbytes + sc.nbytes + qz.nbytes) / (d_out * d_in)
+    assert bits == 4 + 16 / 128 + 4 / 128 and round(bits, 2) == 4.16
+    from post_int4_weight_b200.workloads import WORKLOADS
+    n = WORKLOADS["qwen3_8b_stack36"].params
+    assert round(2 * n / 1e9, 1) == 13.9
+    assert round(n / 2 / 1e9, 1) == 3.5 and (2 * n) / (n / 2) == 4.0
+
+
+# ----------------------------------------------------------- output mode --
+
+def test_output_mode_diagonal_x_equals_weight_space():
+    """X = diag(c) => ||X dW^T||^2 = sum_{r,j} dW[r,j]^2 c_j^2, the weight-space
+    score with x = c."""
+    rng = np.random.default_rng(41)
+    d_out, d_in, g = 16, 64, 32
+    W = (rng.standard_normal((d_out, d_in)) * 0.02).astype(np.float16)
+    c = np.exp(rng.standard_normal(d_in)).astype(np.float16)
+    X = np.diag(c.astype(np.float32)).astype(np.float16)
+    x = c.astype(np.float32)
+    eo = oracle.output_error(X, W, x, g, 20)
+    ew, _, _ = oracle.scale_search([W], x, g, 20)
+    assert np.allclose(eo, ew, rtol=1e-12)
+
+
+def test_output_mode_token_additivity_and_scaling():
+    rng = np.random.default_rng(42)
+    d_out, d_in, g, T = 8, 64, 32, 12
+    W = (rng.standard_normal((d_out, d_in)) * 0.02).astype(np.float16)
+    X = rng.standard_normal((T, d_in)).astype(np.float16)
+    x = np.exp(rng.standard_normal(d_in)).astype(np.float32)
+    e = oracle.output_error(X, W, x, g, 20)
+    e1 = oracle.output_error(X[:5], W, x, g, 20)
+    e2 = oracle.output_error(X[5:], W, x, g, 20)
+    assert np.allclose(e, e1 + e2, rtol=1e-12)
+    e4 = oracle.output_error((2 * X.astype(np.float32)).astype(np.float16), W, x, g, 20)
+    assert np.allclose(e4, 4 * e, rtol=1e-12)
