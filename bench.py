@@ -1,0 +1,385 @@
+#!/usr/bin/env python
+"""Benchmark of the AWQ INT4 hot path (activation stats + fused alpha-grid
+scale search + quantise-and-pack) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload q_proj_4096x4096]
+
+One step = one pass of the whole hot path over one linear: awq_act_stats on
+X [4096 tokens, 4096], awq_scale_search over the 20-point alpha grid,
+awq_quantize_pack of W [4096, 4096] at the chosen scale (Qwen3-8B
+q_proj-shaped layer, group 128).  Inputs are seeded synthetic (see
+post_int4_weight_b200/workloads.py) and resident in HBM when the timed region
+starts; the inputs (67 MB) fit in the 126 MB L2, so a 256 MB buffer is written
+between timed steps (outside the per-step CUDA events) to flush it.
+
+With N > 1 (torchrun) every rank quantises its own independent linear (weak
+scaling, no data-path collective); the time is the max over ranks.
+
+Prints one JSON line (rank 0).  --impl reference times the CPU oracle on the
+host cores instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "AWQ search+pack Gparam/s per layer"
+UNIT = "Gparam/s"
+FMA_OPS_PER_PAIR = 6          # FMA-pipe lane ops per (weight, alpha) pair
+FP32_LANES_PER_SM = 128
+
+
+def _args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="q_proj_4096x4096")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    return ap.parse_args()
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return json.load(f), "measured"
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "sm_max_mhz": 1965.0}, "fallback"
+
+
+# ----------------------------------------------------------------- clocks --
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML every 20 ms."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, torch_device):
+        self.samples = []
+        self.reasons = 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._h = None
+        try:
+            import pynvml as nv
+            self.nv = nv
+            nv.nvmlInit()
+            props = __import__("torch").cuda.get_device_properties(torch_device)
+            h = None
+            uuid = getattr(props, "uuid", None)
+            if uuid is not None:
+                try:
+                    h = nv.nvmlDeviceGetHandleByUUID(("GPU-" + str(uuid)).encode())
+                except Exception:
+                    h = None
+            if h is None:
+                h = nv.nvmlDeviceGetHandleByIndex(torch_device.index or 0)
+            self._h = h
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+        except Exception:
+            self._h = None
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                self.reasons |= int(nv.nvmlDeviceGetCurrentClocksEventReasons(self._h))
+            except Exception:
+                pass
+            time.sleep(0.02)
+
+    def __enter__(self):
+        if self._h is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self._h is not None:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        names = [n for b, n in self.REASONS.items() if self.reasons & b and b != 0x1]
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------- our arm --
+
+def run_ours(a):
+    import torch
+    import torch.distributed as dist
+    from post_int4_weight_b200 import awq
+    from post_int4_weight_b200 import workloads as wl
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+
+    work = wl.WORKLOADS[a.workload]
+    assert len(work.groups) == 1 and work.layers == 1, "bench runs one-group workloads"
+    grp = work.groups[0]
+    g = work.group_sizes[0]
+    n_grid = work.n_grid
+    # each rank quantises its own independent layer (weak scaling)
+    base = 100 * (work.seed + 1000 * rank)
+    Ws_h = [wl.weight(d, grp.d_in, base + m + 1) for m, (_, d) in enumerate(grp.members)]
+    X_h = wl.activations(work.tokens, grp.d_in, base)
+    params = sum(W.numel() for W in Ws_h)
+
+    Ws = [W.to(dev) for W in Ws_h]
+    X = X_h.to(dev)
+    T, d_in = X.shape
+    d_out_total = sum(W.shape[0] for W in Ws)
+    ws_stats = awq.workspace(awq.OP_ACT_STATS, dev, T, 8, d_in)
+    ws_search = awq.workspace(awq.OP_SCALE_SEARCH, dev, 1, d_out_total, d_in, g, n_grid)
+    x = torch.empty(d_in, dtype=torch.float32, device=dev)
+    err = torch.empty(n_grid, dtype=torch.float64, device=dev)
+    best = torch.empty(1, dtype=torch.int32, device=dev)
+    s_best = torch.empty(d_in, dtype=torch.float32, device=dev)
+    packs = [(torch.empty(d_in, W.shape[0] // 8, dtype=torch.int32, device=dev),
+              torch.empty(d_in // g, W.shape[0], dtype=torch.float16, device=dev),
+              torch.empty(d_in // g, W.shape[0] // 8, dtype=torch.int32, device=dev))
+             for W in Ws]
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    kernels_per_step = 3 + 3 + len(Ws)   # stats (3) + search (3) + pack (1 per linear)
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        awq.act_stats(X, out=x, ws=ws_stats)
+        if ev:
+            ev[1].record(stream)
+        awq.scale_search(Ws, x, g, n_grid, out=(err, best, s_best), ws=ws_search)
+        if ev:
+            ev[2].record(stream)
+        for W, pk in zip(Ws, packs):
+            awq.quantize_pack(W, s_best, g, 8, out=pk)
+        if ev:
+            ev[3].record(stream)
+
+    for _ in range(max(a.warmup, 3)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(dev)
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(a.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev) as clk:
+        for k in range(a.steps):
+            flush.zero_()
+            step(evs[k])
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    t_stats = [e[0].elapsed_time(e[1]) for e in evs]
+    t_search = [e[1].elapsed_time(e[2]) for e in evs]
+    t_pack = [e[2].elapsed_time(e[3]) for e in evs]
+    t_step = [e[0].elapsed_time(e[3]) for e in evs]
+    ms = sum(t_step) / len(t_step)
+    ms_search = sum(t_search) / len(t_search)
+    ms_stats = sum(t_stats) / len(t_stats)
+    ms_pack = sum(t_pack) / len(t_pack)
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+
+    # --- end to end through the public API with host buffers
+    e2e = None
+    if rank == 0 or world > 1:
+        Xp = X_h.pin_memory()
+        Wp = [W.pin_memory() for W in Ws_h]
+        out_h = [tuple(torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in pk)
+                 for pk in packs]
+        err_h = torch.empty(n_grid, dtype=torch.float64).pin_memory()
+        best_h = torch.empty(1, dtype=torch.int32).pin_memory()
+        s_h = torch.empty(d_in, dtype=torch.float32).pin_memory()
+        h2d = Xp.numel() * 2 + sum(W.numel() * 2 for W in Wp)
+        d2h = sum(t.numel() * t.element_size() for pk in packs for t in pk) + \
+            err.numel() * 8 + 4 + s_best.numel() * 4
+
+        def e2e_step():
+            X.copy_(Xp, non_blocking=True)
+            for W, w in zip(Ws, Wp):
+                W.copy_(w, non_blocking=True)
+            step()
+            for pk, oh in zip(packs, out_h):
+                for t, th in zip(pk, oh):
+                    th.copy_(t, non_blocking=True)
+            err_h.copy_(err, non_blocking=True)
+            best_h.copy_(best, non_blocking=True)
+            s_h.copy_(s_best, non_blocking=True)
+
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        n_e2e = max(5, min(50, a.steps // 20))
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms_e2e = e0.elapsed_time(e1) / n_e2e
+        if world > 1:
+            t = torch.tensor([ms_e2e], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms_e2e = float(t.item())
+        e2e = {"value": world * params / (ms_e2e * 1e-3) / 1e9, "unit": UNIT,
+               "ms_per_step": ms_e2e, "h2d_bytes_per_step": int(h2d),
+               "d2h_bytes_per_step": int(d2h), "steps": n_e2e}
+
+    if rank != 0:
+        if world > 1:
+            dist.destroy_process_group()
+        return
+
+    peaks, peak_src = _peaks()
+    clocks = clk.summary()
+    n_sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    clk_mhz = clocks["sm_mhz"] or peaks.get("sm_max_mhz", 1965.0)
+    peak_ops = n_sms * FP32_LANES_PER_SM * clk_mhz * 1e6          # lane-ops / s
+    ops = params * n_grid * FMA_OPS_PER_PAIR
+    achieved = ops / (ms_search * 1e-3)
+    bytes_stats = X.numel() * 2
+    bytes_pack = params * 2 + sum(t.numel() * t.element_size() for pk in packs for t in pk)
+    hbm = peaks["hbm_gbs"]
+    roof = {"bound": "alu", "kernel": "awq_scale_search (scale table + fused search + finalize)",
+            "achieved": achieved / 1e12, "peak": peak_ops / 1e12, "unit": "Tlane-op/s",
+            "frac": achieved / peak_ops, "traffic": None,
+            "ops_per_weight_alpha": FMA_OPS_PER_PAIR,
+            "peak_basis": f"{n_sms} SMs x {FP32_LANES_PER_SM} FP32 lanes x {clk_mhz:.0f} MHz "
+                          f"(median SM clock sampled in the timed region)"}
+    out = {
+        "metric": METRIC, "value": world * params / (ms * 1e-3) / 1e9, "unit": UNIT,
+        "n_gpus": world, "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32", "data": "synthetic",
+        "config": {"workload": a.workload, "d_out": d_out_total, "d_in": d_in,
+                   "tokens": T, "group_size": g, "n_grid": n_grid,
+                   "params_per_gpu": params, "l2": "flushed (256 MB write) between timed steps",
+                   "parallelism": f"independent layer per rank x{world}"},
+        "roofline": roof,
+        "kernels": {
+            "act_stats": {"ms": ms_stats, "GB/s": bytes_stats / (ms_stats * 1e-3) / 1e9,
+                          "hbm_frac": bytes_stats / (ms_stats * 1e-3) / 1e9 / hbm},
+            "scale_search": {"ms": ms_search, "Tlane-op/s": achieved / 1e12,
+                             "W_GB/s": params * 2 / (ms_search * 1e-3) / 1e9},
+            "quantize_pack": {"ms": ms_pack, "GB/s": bytes_pack / (ms_pack * 1e-3) / 1e9,
+                              "hbm_frac": bytes_pack / (ms_pack * 1e-3) / 1e9 / hbm},
+            "hbm_peak_GBs": hbm, "peak_source": peak_src},
+        "clocks": clocks,
+        "e2e": e2e,
+        "gpu_launches": kernels_per_step * a.steps,
+    }
+    if world == 1 and not a.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(Ws_h, X_h, g, n_grid, a.cpu_seconds)
+    print(json.dumps(out), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+# ----------------------------------------------------------- CPU oracle --
+
+def _oracle_pass(Ws, X, g, n_grid):
+    import oracle
+    x = oracle.act_stats(X)
+    err, best, s = oracle.scale_search(Ws, x, g, n_grid)
+    for W in Ws:
+        oracle.quantize_pack(W, s, g, 8)
+
+
+def cpu_baseline(Ws_h, X_h, g, n_grid, seconds):
+    """Full passes of the CPU oracle over the same workload until `seconds`."""
+    import oracle
+    Ws = [W.numpy() for W in Ws_h]
+    X = X_h.numpy()
+    params = sum(W.size for W in Ws)
+    n = 0
+    t0 = time.perf_counter()
+    while True:
+        _oracle_pass(Ws, X, g, n_grid)
+        n += 1
+        if time.perf_counter() - t0 >= seconds:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": n * params / dt / 1e9, "unit": UNIT, "cores": oracle.threads(),
+            "kind": "oracle",
+            "sample": f"{n} full pass(es) of the same workload (stats + 20-point search + pack)"}
+
+
+def run_reference(a):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    import numpy as np
+    import oracle
+    from post_int4_weight_b200 import workloads as wl
+    work = wl.WORKLOADS[a.workload]
+    grp = work.groups[0]
+    g = work.group_sizes[0]
+    # a bounded sample of the workload per step: 64 weight rows of every
+    # member and the same share of the tokens
+    rows = 64
+    base = 100 * work.seed
+    Ws = [wl.weight(d, grp.d_in, base + m + 1)[:rows].numpy()
+          for m, (_, d) in enumerate(grp.members)]
+    tok = max(1, work.tokens * rows // sum(d for _, d in grp.members))
+    X = wl.activations(work.tokens, grp.d_in, base)[:tok].numpy()
+    params = sum(W.size for W in Ws)
+    for _ in range(max(a.warmup, 3)):
+        _oracle_pass(Ws, X, g, work.n_grid)
+    t0 = time.perf_counter()
+    for _ in range(a.steps):
+        _oracle_pass(Ws, X, g, work.n_grid)
+    dt = time.perf_counter() - t0
+    v = a.steps * params / dt / 1e9
+    sample = (f"{rows} rows x {grp.d_in} of each linear and {tok} tokens per step "
+              f"(stats + 20-point search + pack)")
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": world,
+        "steps": a.steps, "warmup": a.warmup, "ms_per_step": dt / a.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic", "config": {"workload": a.workload, "group_size": g,
+                                        "n_grid": work.n_grid},
+        "cpu_baseline": {"value": v, "unit": UNIT, "cores": oracle.threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+if __name__ == "__main__":
+    args = _args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)

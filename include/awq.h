@@ -1,0 +1,208 @@
+/*
+ * awq.h -- C ABI of the B200 (sm_100a) AWQ INT4 weight-quantisation library
+ * (libawq_b200.so).
+ *
+ * The method (activation-aware weight quantisation, AWQ) as the pages define
+ * it:
+ *   "From-Scratch AWQ INT4 Quantization on Qwen3-8B" -- sections
+ *       "AWQ scaling", "Group-wise symmetric INT4",
+ *       "AutoAWQ / HF-AWQ GEMM on-disk format" (and the exporter's step 4);
+ *   "AWQ architecture, in depth: the calibration pipeline, scale search,
+ *       packed format and serving kernels" -- sections "The scale search as
+ *       code" and "Quantization, storage and packing";
+ *   "Weight-Only Quantization: GPTQ and AWQ" -- section 5 (AWQ) and
+ *       sections 6-9 (the packed format).
+ *
+ * Conventions shared by every entry point:
+ *   - Every tensor argument is a DEVICE pointer owned by the caller; the
+ *     library never allocates, frees or retains memory.  Scratch memory comes
+ *     from the caller's workspace (size from awq_workspace_size); its
+ *     contents need not be initialised and are clobbered.
+ *   - Matrices are row-major and dense: W is fp16 [d_out, d_in] (row stride
+ *     d_in), X is fp16 [T, ld] with the first d_in columns used.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Every
+ *     call only enqueues kernels on it and returns; nothing synchronises.
+ *     Outputs are valid once the stream has reached that point.
+ *   - Arguments are validated on the host before anything is enqueued; on a
+ *     validation error nothing is enqueued and the outputs are untouched.
+ *     A launch failure returns AWQ_ERR_CUDA.  The library never aborts.
+ *   - A device pointer must be 16-byte aligned (AWQ_ERR_ALIGNMENT otherwise).
+ *   - Errors found on the device (non-finite inputs, a bounded wait that
+ *     gave up) are reported in the outputs, as each entry point states.
+ *   - Results are deterministic: the same inputs give the same bits.
+ *   - The calls may run concurrently on different streams provided their
+ *     workspaces do not overlap.
+ */
+#ifndef AWQ_B200_AWQ_H
+#define AWQ_B200_AWQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum awq_status {
+    AWQ_OK = 0,
+    AWQ_ERR_INVALID_ARG = 1,   /* a size, count or pointer is out of range   */
+    AWQ_ERR_UNSUPPORTED = 2,   /* valid but not implemented (e.g. group size) */
+    AWQ_ERR_ALIGNMENT = 3,     /* a pointer or leading dimension misaligned   */
+    AWQ_ERR_WORKSPACE = 4,     /* workspace NULL or smaller than required      */
+    AWQ_ERR_CUDA = 5,          /* a CUDA runtime call or launch failed         */
+    AWQ_ERR_NONFINITE = 6      /* reserved: non-finite data (see outputs)      */
+} awq_status;
+
+/* Flags of awq_scale_search / awq_output_error. */
+#define AWQ_SCALE_FP16 0  /* group scale rounded to fp16 (the stored format) */
+#define AWQ_SCALE_FP32 1  /* group scale kept in fp32 (the worked example)  */
+
+/* Operation ids of awq_workspace_size. */
+#define AWQ_OP_ACT_STATS    0
+#define AWQ_OP_SCALE_SEARCH 1
+#define AWQ_OP_OUTPUT_ERROR 2
+
+/* Human-readable name of a status code (static storage; never NULL). */
+const char *awq_status_string(int status);
+
+/* Version of this ABI (major * 100 + minor). */
+int awq_abi_version(void);
+
+/*
+ * Bytes of workspace that `op` needs for the given sizes.  For
+ * AWQ_OP_ACT_STATS only d_in matters; for AWQ_OP_SCALE_SEARCH d_in, the
+ * group size and n_grid; for AWQ_OP_OUTPUT_ERROR all of them (T is the token
+ * count, d_out_total the rows of W).  Writes *bytes; returns
+ * AWQ_ERR_INVALID_ARG for an unknown op or out-of-range size.
+ */
+awq_status awq_workspace_size(int op, int64_t T, int64_t d_out_total,
+                              int64_t d_in, int group_size, int n_grid,
+                              size_t *bytes);
+
+/*
+ * Per-input-channel activation magnitude, the AWQ salience statistic
+ * ("From-Scratch AWQ ...", section "AWQ scaling": x = |X|.mean(0);
+ * "AWQ architecture ...", section "The scale search as code").
+ *
+ *   x_mean[j] = (1/T) * sum_{t<T} |X[t, j]|,   j < d_in
+ *
+ * The sum is exact (every |fp16| is an integer multiple of 2^-24), then
+ * divided by T in fp64 and rounded to fp32.  A column holding a NaN gives
+ * NaN, one holding an infinity (and no NaN) gives +inf.
+ *
+ *   X        fp16 [T, ld] device, 16-byte aligned; ld % 8 == 0, ld >= d_in
+ *   T        tokens, 1 <= T <= 2^31
+ *   d_in     channels, 1 <= d_in, d_in % 8 == 0
+ *   x_mean   fp32 [d_in] device output
+ *   ws       workspace of awq_workspace_size(AWQ_OP_ACT_STATS, ...) bytes
+ */
+awq_status awq_act_stats(const void *X, int64_t T, int64_t d_in, int64_t ld,
+                         float *x_mean, void *ws, size_t ws_bytes,
+                         void *stream);
+
+/*
+ * AWQ per-channel scale search over an alpha grid, fused over all grid
+ * points ("From-Scratch AWQ ...", sections "AWQ scaling" and "Group-wise
+ * symmetric INT4"; "AWQ architecture ...", section "The scale search as
+ * code").  For i < n_grid, alpha_i = i / n_grid:
+ *
+ *   s_i[j]   = max(x_mean[j], 1e-4)^alpha_i, then divided by
+ *              sqrt(max_j s_i[j] * min_j s_i[j])     (fp64, rounded to fp32)
+ *   per row r and group k of group_size channels, in fp32:
+ *     ws       = W[r, j] * s_i[j]
+ *     q_scale  = fp16_rne(max |ws| / 7)  (AWQ_SCALE_FP16; 0 for an all-zero
+ *                group; held at 65504 if it overflows fp16)
+ *     q        = clamp(rint(ws / q_scale), -7, 7)
+ *   err[i]   = sum over every segment, row and channel of
+ *              ((W[r, j] - q * q_scale / s_i[j]) * x_mean[j])^2
+ *   best_idx = first i with the smallest err[i];  s_best = s_{best_idx}.
+ *
+ * The n_seg weight segments share the input (e.g. q/k/v, or gate/up): one
+ * scale vector is searched for all of them and their errors are summed.
+ *
+ *   n_seg       1..AWQ_MAX_SEGMENTS
+ *   W           HOST array of n_seg DEVICE pointers, fp16 [d_out[k], d_in]
+ *   d_out       HOST array of n_seg row counts, each >= 1
+ *   d_in        channels, multiple of group_size
+ *   x_mean      fp32 [d_in] device (from awq_act_stats)
+ *   group_size  32, 64 or 128
+ *   n_grid      1..32 grid points (20 in the method)
+ *   flags       AWQ_SCALE_FP16 or AWQ_SCALE_FP32
+ *   err         fp64 [n_grid] device output
+ *   best_idx    int32 [1] device output; -1 if any err is not finite (NaN or
+ *               infinite input), -2 if a device-side wait gave up
+ *   s_best      fp32 [d_in] device output (NaN when best_idx < 0)
+ *   ws          workspace of awq_workspace_size(AWQ_OP_SCALE_SEARCH, ...)
+ * err is evaluated in fp32 per row and accumulated in fp64 in a fixed order;
+ * it matches the exact score of the same decisions to about 1e-6 relative.
+ */
+#define AWQ_MAX_SEGMENTS 8
+awq_status awq_scale_search(int n_seg, const void *const *W,
+                            const int64_t *d_out, int64_t d_in,
+                            const float *x_mean, int group_size, int n_grid,
+                            int flags, double *err, int32_t *best_idx,
+                            float *s_best, void *ws, size_t ws_bytes,
+                            void *stream);
+
+/*
+ * Group-wise symmetric INT4 quantisation of W * s and packing into the
+ * AutoAWQ GEMM layout ("From-Scratch AWQ ...", sections "Group-wise
+ * symmetric INT4", "AutoAWQ / HF-AWQ GEMM on-disk format" and exporter
+ * step 4; "AWQ architecture ...", section "Quantization, storage and
+ * packing").  Codes are decided exactly as in awq_scale_search (fp16 group
+ * scale) with the IEEE fp32 quotient ws / q_scale:
+ *
+ *   u[r, j]        = q[r, j] + zero_point                (0..15)
+ *   qweight[j, c]  = nibble p (bits 4p..4p+3) holds u[8c + order[p], j],
+ *                    order = {0, 2, 4, 6, 1, 3, 5, 7}
+ *   scales[k, r]   = fp16 q_scale of row r, group k
+ *   qzeros[k, c]   = zero_point in all eight nibbles
+ *
+ *   W           fp16 [d_out, d_in] device
+ *   d_out       multiple of 8;  d_in multiple of group_size
+ *   s           fp32 [d_in] device scale (s_best), or NULL for s = 1 (RTN)
+ *   group_size  32, 64 or 128
+ *   zero_point  7 or 8 (8: codes 1..15; 7: codes 0..14)
+ *   qweight     int32 [d_in, d_out / 8] device output
+ *   scales      fp16 [d_in / group_size, d_out] device output
+ *   qzeros      int32 [d_in / group_size, d_out / 8] device output
+ * A group holding a non-finite value stores scale NaN (0x7E00) and code
+ * zero_point for all its weights.
+ */
+awq_status awq_quantize_pack(const void *W, int64_t d_out, int64_t d_in,
+                             const float *s, int group_size, int zero_point,
+                             int32_t *qweight, void *scales, int32_t *qzeros,
+                             void *stream);
+
+/*
+ * Optional output-space scoring of every grid point ("AWQ architecture
+ * ...", section "The scale search as code": the group's output after
+ * fake quantisation compared with the full-precision output; "Weight-Only
+ * Quantization: GPTQ and AWQ", section 2: the output error is X (W - W_hat)):
+ *
+ *   err[i] = || X (W - W_hat_i)^T ||_F^2,   W_hat_i = Q(W * s_i) / s_i
+ *
+ * with s_i and Q exactly as in awq_scale_search.  W - W_hat_i is rounded to
+ * fp16 and multiplied by X on the tensor cores (fp16 in, fp32 accumulate);
+ * the squares are summed in fp32 per tile and in fp64 across tiles.
+ *
+ *   X           fp16 [T, d_in] device;  T >= 1
+ *   W           fp16 [d_out, d_in] device; d_out % 8 == 0
+ *   x_mean      fp32 [d_in] device (defines s_i)
+ *   group_size  32, 64 or 128;  d_in multiple of group_size and of 64
+ *   n_grid      1..32;  flags as in awq_scale_search
+ *   err         fp64 [n_grid] device output
+ *   best_idx    int32 [1] device output (first minimum; -1 if non-finite)
+ *   ws          workspace of awq_workspace_size(AWQ_OP_OUTPUT_ERROR, ...)
+ */
+awq_status awq_output_error(const void *X, int64_t T, const void *W,
+                            int64_t d_out, int64_t d_in, const float *x_mean,
+                            int group_size, int n_grid, int flags,
+                            double *err, int32_t *best_idx, void *ws,
+                            size_t ws_bytes, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* AWQ_B200_AWQ_H */

@@ -1,0 +1,123 @@
+// common.cuh -- device helpers shared by the sm_100a kernels of libawq_b200.
+//
+// Nothing here is shared with the CPU oracle; the two are written apart.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace awq {
+
+// 1.5 * 2^23: adding it to |y| < 2^22 rounds y to an integer (ties to even)
+// in the last place, because the sum's unit in the last place is 1.
+constexpr float kRoundMagic = 12582912.0f;
+constexpr uint32_t kRoundMagicBits = 0x4B400000u;
+constexpr float kHalfMax = 65504.0f;             // largest finite fp16
+constexpr float kHalfMinNormal = 6.103515625e-05f;  // 2^-14
+constexpr float kFloatMinNormal = 1.17549435e-38f;  // 2^-126
+
+// Host-visible error bits written into a workspace word by the kernels.
+constexpr int kDevErrWaitTimeout = 1;
+
+// Bound on any spin-wait: 2 seconds of %globaltimer.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// ---------------------------------------------------------------- mbarrier
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;"
+                 :: "r"(smem_addr(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_fence_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("{\n\t.reg .b64 st;\n\t"
+                 "mbarrier.arrive.shared::cta.b64 st, [%0];\n\t}"
+                 :: "r"(smem_addr(bar)) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("{\n\t.reg .b64 st;\n\t"
+                 "mbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}"
+                 :: "r"(smem_addr(bar)), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok) : "r"(smem_addr(bar)), "r"(parity) : "memory");
+    return ok != 0;
+}
+
+// Wait for the phase with the given parity to complete; gives up after
+// kWaitLimitNs and returns false (the caller reports the error and unwinds).
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (global_ns() - t0 > kWaitLimitNs) return false;
+    }
+    return true;
+}
+
+// ---------------------------------------------------------------- TMA
+
+// 2-D tiled bulk tensor load global -> shared, completion counted on `bar`.
+// x is the innermost (contiguous) coordinate in elements.
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map,
+                                            int32_t x, int32_t y, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];"
+        :: "r"(smem_addr(dst)), "l"(reinterpret_cast<uint64_t>(map)),
+           "r"(x), "r"(y), "r"(smem_addr(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
+    asm volatile("prefetch.tensormap [%0];"
+                 :: "l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// ---------------------------------------------------------------- numerics
+
+// Group scale from the group's largest |w * s| (round-to-nearest-even
+// throughout): fp32 quotient by 7, then fp16 unless fp32 scales are asked
+// for.  An fp16 overflow is held at 65504; a non-finite maximum gives NaN.
+// *exact_range is set when every |ws| / scale is known to be below 7.5, so
+// that the code needs no clamp.
+__device__ __forceinline__ float group_scale(float m, bool fp32_scale, bool* exact_range) {
+    const float qsf = __fdiv_rn(m, 7.0f);
+    float qs;
+    bool in_range;
+    if (fp32_scale) {
+        qs = qsf;
+        in_range = qs >= kFloatMinNormal;
+    } else {
+        qs = __half2float(__float2half_rn(qsf));
+        in_range = (qs >= kHalfMinNormal) && (qs <= kHalfMax);
+        if (qs > kHalfMax) qs = kHalfMax;
+    }
+    if (!(m <= 3.402823466e38f)) qs = __int_as_float(0x7fc00000);
+    *exact_range = in_range;
+    return qs;
+}
+
+}  // namespace awq

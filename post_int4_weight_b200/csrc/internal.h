@@ -1,0 +1,75 @@
+// internal.h -- host-side launchers behind the C ABI of include/awq.h.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "awq.h"
+
+namespace awq {
+
+constexpr size_t kWsAlign = 256;
+
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+inline bool aligned16(const void* p) {
+    return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
+}
+
+struct DeviceInfo {
+    int device = 0;
+    int num_sms = 0;
+    size_t max_smem_optin = 0;    // per block, opt-in
+    size_t max_smem_per_sm = 0;
+};
+cudaError_t query_device(DeviceInfo* info);
+
+// ---- activation statistics
+size_t act_stats_workspace(int64_t d_in);
+cudaError_t launch_act_stats(const void* X, int64_t T, int64_t d_in, int64_t ld,
+                             float* x_mean, void* ws, cudaStream_t stream);
+
+// ---- scale search
+size_t scale_search_workspace(int64_t d_in, int group_size, int n_grid);
+awq_status launch_scale_search(int n_seg, const void* const* W, const int64_t* d_out,
+                               int64_t d_in, const float* x_mean, int group_size,
+                               int n_grid, int flags, double* err, int32_t* best_idx,
+                               float* s_best, void* ws, cudaStream_t stream);
+
+// ---- quantise + pack
+cudaError_t launch_quantize_pack(const void* W, int64_t d_out, int64_t d_in,
+                                 const float* s, int group_size, int zero_point,
+                                 int32_t* qweight, void* scales, int32_t* qzeros,
+                                 cudaStream_t stream);
+
+// ---- output-space scoring
+size_t output_error_workspace(int64_t T, int64_t d_out, int64_t d_in, int group_size,
+                              int n_grid);
+awq_status launch_output_error(const void* X, int64_t T, const void* W, int64_t d_out,
+                               int64_t d_in, const float* x_mean, int group_size,
+                               int n_grid, int flags, double* err, int32_t* best_idx,
+                               void* ws, cudaStream_t stream);
+
+// ---- shared pieces of the search and the output-error mode
+// Writes S[i][j] and tau[i][j] = x_mean[j] / S[i][j] (fp32, [n_grid][d_in]),
+// and clears the device error word (if non-NULL).
+cudaError_t launch_scale_table(const float* x_mean, int64_t d_in, int n_grid,
+                               float* S, float* tau, int* dev_err, cudaStream_t stream);
+// Sums partial[c][i] over c in order, picks the first minimum, copies its row
+// of S into s_best (if non-NULL).
+cudaError_t launch_finalize(const double* partial, int n_parts, int n_grid,
+                            const float* S, int64_t d_in, const int* dev_err,
+                            double* err, int32_t* best_idx, float* s_best,
+                            cudaStream_t stream);
+
+// cuTensorMapEncodeTiled, fetched from the driver once.
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_tiled_fn();
+
+}  // namespace awq

@@ -1,0 +1,100 @@
+"""The C-ABI library loads on a host without a GPU, exports every symbol that
+include/awq.h declares, and rejects bad arguments on the host before any
+CUDA call (no compute call is made here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from post_int4_weight_b200 import awq
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "awq.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(awq_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_four_calls():
+    names = declared_functions()
+    for n in ("awq_act_stats", "awq_scale_search", "awq_quantize_pack",
+              "awq_output_error", "awq_workspace_size", "awq_status_string"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = awq.lib()
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+        assert ctypes.cast(getattr(lib, name), ctypes.c_void_p).value
+
+
+def test_status_strings_and_version():
+    assert awq.string(0) == "AWQ_OK"
+    for s in range(1, 7):
+        assert awq.string(s).startswith("AWQ_ERR_")
+    assert awq.lib().awq_abi_version() == 100
+
+
+def test_workspace_sizes():
+    n_stats = awq.workspace_size(awq.OP_ACT_STATS, 4096, 8, 4096, 128, 20)
+    assert n_stats >= 4096 * 12
+    n_search = awq.workspace_size(awq.OP_SCALE_SEARCH, 1, 8, 4096, 128, 20)
+    assert n_search >= 2 * 20 * 4096 * 4
+    with pytest.raises(awq.AwqError):
+        awq.workspace_size(7, 1, 8, 4096, 128, 20)
+    with pytest.raises(awq.AwqError):
+        awq.workspace_size(awq.OP_SCALE_SEARCH, 1, 8, 4096, 96, 20)
+    with pytest.raises(awq.AwqError):
+        awq.workspace_size(awq.OP_SCALE_SEARCH, 1, 8, 4096, 128, 33)
+
+
+def _vp(v):
+    return ctypes.c_void_p(v)
+
+
+def test_host_validation_without_a_gpu():
+    L = awq.lib()
+    fake = 0x10000           # 16-byte aligned, never dereferenced on the host
+    odd = 0x10004
+    # act_stats
+    assert L.awq_act_stats(None, 4, 8, 8, fake, fake, 1 << 20, None) == 1
+    assert L.awq_act_stats(fake, 0, 8, 8, fake, fake, 1 << 20, None) == 1
+    assert L.awq_act_stats(fake, 4, 12, 12, fake, fake, 1 << 20, None) == 3
+    assert L.awq_act_stats(odd, 4, 8, 8, fake, fake, 1 << 20, None) == 3
+    assert L.awq_act_stats(fake, 4, 8, 8, fake, None, 0, None) == 4
+    assert L.awq_act_stats(fake, 4, 8, 8, fake, fake, 8, None) == 4
+    # scale_search
+    W = (ctypes.c_void_p * 1)(fake)
+    d = (ctypes.c_int64 * 1)(64)
+    args = dict(n=1, W=W, d=d, d_in=256, x=fake, g=128, n_grid=20, flags=0)
+
+    def search(**kw):
+        a = dict(args, **kw)
+        return L.awq_scale_search(a["n"], a["W"], a["d"], a["d_in"], a["x"], a["g"],
+                                  a["n_grid"], a["flags"], fake, fake, fake, fake,
+                                  1 << 24, None)
+    assert search(n=0) == 1
+    assert search(n=9) == 1
+    assert search(g=96) == 2
+    assert search(n_grid=0) == 1 and search(n_grid=33) == 1
+    assert search(flags=2) == 1
+    assert search(d_in=200) == 1
+    assert search(W=(ctypes.c_void_p * 1)(odd)) == 3
+    assert search(d=(ctypes.c_int64 * 1)(0)) == 1
+    assert L.awq_scale_search(1, W, d, 256, fake, 128, 20, 0, fake, fake, fake, fake,
+                              16, None) == 4
+    # quantize_pack
+    assert L.awq_quantize_pack(fake, 12, 256, None, 128, 8, fake, fake, fake, None) == 1
+    assert L.awq_quantize_pack(fake, 64, 256, None, 128, 9, fake, fake, fake, None) == 1
+    assert L.awq_quantize_pack(fake, 64, 256, None, 48, 8, fake, fake, fake, None) == 2
+    assert L.awq_quantize_pack(fake, 64, 256, odd, 128, 8, fake, fake, fake, None) == 3
+    # output_error
+    assert L.awq_output_error(fake, 0, fake, 64, 256, fake, 128, 20, 0, fake, fake,
+                              fake, 1 << 30, None) == 1
+    assert L.awq_output_error(fake, 16, fake, 64, 256, fake, 128, 20, 0, fake, fake,
+                              fake, 16, None) == 4
