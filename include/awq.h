@@ -145,6 +145,34 @@ awq_status awq_scale_search(int n_seg, const void *const *W,
                             void *stream);
 
 /*
+ * awq_scale_search without a workspace, for callers that cannot allocate
+ * device memory (a plug-in whose host framework owns all device memory and
+ * offers it no allocator, a section where a cudaMalloc's possible device
+ * synchronisation is not acceptable, a C caller holding only its own input
+ * and output buffers).  The pages have no counterpart: this is a deployment
+ * convenience, not part of the method.
+ *
+ * Same arguments, results and errors as awq_scale_search, minus ws/ws_bytes.
+ * The scratch is one static device array of AWQ_NOALLOC_SCRATCH_BYTES inside
+ * the library; every GPU that uses the library keeps it until the process
+ * exits.  Calls whose workspace need (awq_workspace_size with
+ * AWQ_OP_SCALE_SEARCH) exceeds it return AWQ_ERR_WORKSPACE with nothing
+ * enqueued -- e.g. d_in = 16384 fits with n_grid <= 29, d_in = 12288 with
+ * n_grid <= 32.  The first call on a device looks the array's address up
+ * (cudaGetSymbolAddress, that device current) and caches it: make it before
+ * any stream capture on that device.  All calls on a device share the array;
+ * each call rewrites every scratch byte it reads, but calls that overlap on
+ * the GPU (unordered streams) race on it.  Allocates nothing.
+ */
+#define AWQ_NOALLOC_SCRATCH_BYTES (4u << 20)
+awq_status awq_scale_search_noalloc(int n_seg, const void *const *W,
+                                    const int64_t *d_out, int64_t d_in,
+                                    const float *x_mean, int group_size,
+                                    int n_grid, int flags, double *err,
+                                    int32_t *best_idx, float *s_best,
+                                    void *stream);
+
+/*
  * Group-wise symmetric INT4 quantisation of W * s and packing into the
  * AutoAWQ GEMM layout ("From-Scratch AWQ ...", sections "Group-wise
  * symmetric INT4", "AutoAWQ / HF-AWQ GEMM on-disk format" and exporter

@@ -202,3 +202,41 @@ def quantize_group(Ws: Sequence[torch.Tensor], X: torch.Tensor, group_size: int 
     err, best, s_best = scale_search(Ws, x, group_size, n_grid)
     packed = [quantize_pack(W, s_best, group_size, zero_point) for W in Ws]
     return err, best, s_best, packed
+
+
+_noalloc_fn = None
+
+
+def _noalloc_entry():
+    """ctypes handle of awq_scale_search_noalloc with its argument types."""
+    global _noalloc_fn
+    if _noalloc_fn is None:
+        fn = lib().awq_scale_search_noalloc
+        p = ctypes.c_void_p
+        fn.argtypes = [ctypes.c_int, p, p, ctypes.c_int64, p, ctypes.c_int, ctypes.c_int,
+                       ctypes.c_int, p, p, p, p]
+        fn.restype = ctypes.c_int
+        _noalloc_fn = fn
+    return _noalloc_fn
+
+
+def scale_search_noalloc(Ws: Sequence[torch.Tensor], x: torch.Tensor, group_size: int = 128,
+                         n_grid: int = 20, flags: int = SCALE_FP16):
+    """awq_scale_search_noalloc: the same search with the library's static
+    per-device scratch instead of a caller workspace.  Only the outputs are
+    allocated here (by torch); the library allocates nothing."""
+    fn = _noalloc_entry()
+    Ws = [_cuda(W, torch.float16, "W") for W in Ws]
+    _cuda(x, torch.float32, "x")
+    d_in = x.shape[0]
+    dev = x.device
+    err = torch.empty(n_grid, dtype=torch.float64, device=dev)
+    best = torch.empty(1, dtype=torch.int32, device=dev)
+    s_best = torch.empty(d_in, dtype=torch.float32, device=dev)
+    n = len(Ws)
+    ptrs = (ctypes.c_void_p * n)(*[W.data_ptr() for W in Ws])
+    d_out = (ctypes.c_int64 * n)(*[W.shape[0] for W in Ws])
+    _check(fn(n, ptrs, d_out, d_in, x.data_ptr(), group_size, n_grid, flags,
+              err.data_ptr(), best.data_ptr(), s_best.data_ptr(), _stream(dev)),
+           "awq_scale_search_noalloc")
+    return err, best, s_best
