@@ -47,6 +47,8 @@ def _args():
     ap.add_argument("--workload", default="q_proj_4096x4096")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-graph", action="store_true",
+                    help="launch each step eagerly instead of replaying a CUDA graph")
     return ap.parse_args()
 
 
@@ -166,50 +168,86 @@ def run_ours(a):
              for W in Ws]
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
-    kernels_per_step = 3 + 3 + len(Ws)   # stats (3) + search (3) + pack (1 per linear)
+    kernels_per_step = 1 + 3 + len(Ws)   # stats (1) + search (3) + pack (1 per linear)
 
-    def step(ev=None):
-        if ev:
-            ev[0].record(stream)
+    def call_stats():
         awq.act_stats(X, out=x, ws=ws_stats)
-        if ev:
-            ev[1].record(stream)
+
+    def call_search():
         awq.scale_search(Ws, x, g, n_grid, out=(err, best, s_best), ws=ws_search)
-        if ev:
-            ev[2].record(stream)
+
+    def call_pack():
         for W, pk in zip(Ws, packs):
             awq.quantize_pack(W, s_best, g, 8, out=pk)
-        if ev:
-            ev[3].record(stream)
 
+    def step():
+        call_stats()
+        call_search()
+        call_pack()
+
+    # eager warm-up (first calls do the one-time per-device set-up), then the
+    # step and each call are captured into CUDA graphs and replayed
     for _ in range(max(a.warmup, 3)):
         flush.zero_()
         step()
     torch.cuda.synchronize(dev)
+    graphs = None
+    if not a.no_graph:
+        graphs = {}
+        for name, fn in (("step", step), ("stats", call_stats), ("search", call_search),
+                         ("pack", call_pack)):
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr):
+                fn()
+            graphs[name] = gr
+        for _ in range(3):
+            flush.zero_()
+            graphs["step"].replay()
+        torch.cuda.synchronize(dev)
+    run = {k: (graphs[k].replay if graphs else f) for k, f in
+           (("step", step), ("stats", call_stats), ("search", call_search), ("pack", call_pack))}
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(a.steps)]
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(a.steps)]
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
     with ClockSampler(dev) as clk:
         for k in range(a.steps):
             flush.zero_()
-            step(evs[k])
+            evs[k][0].record(stream)
+            run["step"]()
+            evs[k][1].record(stream)
         torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
-    t_stats = [e[0].elapsed_time(e[1]) for e in evs]
-    t_search = [e[1].elapsed_time(e[2]) for e in evs]
-    t_pack = [e[2].elapsed_time(e[3]) for e in evs]
-    t_step = [e[0].elapsed_time(e[3]) for e in evs]
+    t_step = [e0.elapsed_time(e1) for e0, e1 in evs]
     ms = sum(t_step) / len(t_step)
-    ms_search = sum(t_search) / len(t_search)
-    ms_stats = sum(t_stats) / len(t_stats)
-    ms_pack = sum(t_pack) / len(t_pack)
     if world > 1:
         t = torch.tensor([ms], dtype=torch.float64, device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms = float(t.item())
+
+    # per-call breakdown (separately timed steps, L2 flushed before each)
+    n_br = max(10, min(200, a.steps))
+    br = {"stats": [], "search": [], "pack": []}
+    for _ in range(n_br):
+        flush.zero_()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        ev[0].record(stream)
+        run["stats"]()
+        ev[1].record(stream)
+        run["search"]()
+        ev[2].record(stream)
+        run["pack"]()
+        ev[3].record(stream)
+        torch.cuda.synchronize(dev)
+        br["stats"].append(ev[0].elapsed_time(ev[1]))
+        br["search"].append(ev[1].elapsed_time(ev[2]))
+        br["pack"].append(ev[2].elapsed_time(ev[3]))
+    ms_stats = sum(br["stats"]) / n_br
+    ms_search = sum(br["search"]) / n_br
+    ms_pack = sum(br["pack"]) / n_br
 
     # --- end to end through the public API with host buffers
     e2e = None
@@ -299,6 +337,7 @@ def run_ours(a):
         "clocks": clocks,
         "e2e": e2e,
         "gpu_launches": kernels_per_step * a.steps,
+        "launch": "CUDA graph per step" if graphs else "eager",
     }
     if world == 1 and not a.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(Ws_h, X_h, g, n_grid, a.cpu_seconds)

@@ -91,10 +91,11 @@ awq_status awq_workspace_size(int op, int64_t T, int64_t d_out_total,
  * NaN, one holding an infinity (and no NaN) gives +inf.
  *
  *   X        fp16 [T, ld] device, 16-byte aligned; ld % 8 == 0, ld >= d_in
- *   T        tokens, 1 <= T <= 2^31
- *   d_in     channels, 1 <= d_in, d_in % 8 == 0
+ *   T        tokens, 1 <= T <= 2^23
+ *   d_in     channels, 1 <= d_in <= 2^24, d_in % 8 == 0
  *   x_mean   fp32 [d_in] device output
- *   ws       workspace of awq_workspace_size(AWQ_OP_ACT_STATS, ...) bytes
+ *   ws       workspace of awq_workspace_size(AWQ_OP_ACT_STATS, ...) bytes;
+ *            that size is currently 0, and ws may then be NULL
  */
 awq_status awq_act_stats(const void *X, int64_t T, int64_t d_in, int64_t ld,
                          float *x_mean, void *ws, size_t ws_bytes,

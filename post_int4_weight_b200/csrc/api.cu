@@ -88,8 +88,9 @@ awq_status awq_act_stats(const void* X, int64_t T, int64_t d_in, int64_t ld, flo
     if (d_in < 1 || d_in > (int64_t(1) << 24) || ld < d_in) return AWQ_ERR_INVALID_ARG;
     if (d_in % 8 || ld % 8) return AWQ_ERR_ALIGNMENT;
     if (!aligned16(X) || !aligned16(x_mean)) return AWQ_ERR_ALIGNMENT;
-    if (!ws || ws_bytes < act_stats_workspace(d_in)) return AWQ_ERR_WORKSPACE;
-    if (!aligned16(ws)) return AWQ_ERR_ALIGNMENT;
+    const size_t need = act_stats_workspace(d_in);
+    if (need > 0 && (!ws || ws_bytes < need)) return AWQ_ERR_WORKSPACE;
+    if (ws && !aligned16(ws)) return AWQ_ERR_ALIGNMENT;
     if (launch_act_stats(X, T, d_in, ld, x_mean, ws, static_cast<cudaStream_t>(stream)) !=
         cudaSuccess)
         return AWQ_ERR_CUDA;

@@ -77,6 +77,26 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
     return true;
 }
 
+// ------------------------------------------------- dependent launches
+// Programmatic dependent launch: a kernel launched with the programmatic
+// stream-serialisation attribute may start while its predecessor drains; it
+// must call pdl_wait() before touching anything the predecessor writes (or
+// anything it writes that the predecessor may still read).
+__device__ __forceinline__ void pdl_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Approximate reciprocal (MUFU, <= 1 ulp); used only where an ulp cannot
+// change a result beyond the documented tolerance.
+__device__ __forceinline__ float rcp_approx(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // ---------------------------------------------------------------- TMA
 
 // 2-D tiled bulk tensor load global -> shared, completion counted on `bar`.
@@ -98,13 +118,52 @@ __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
 
 // ---------------------------------------------------------------- numerics
 
+// Round-to-nearest-even fp32 quotient m / 7 for finite m >= 0, from the
+// rounded reciprocal c = RN(1/7) and one residual correction (the residual
+// m - 7 q0 is exact in an FMA).  Equal to the IEEE quotient for every
+// non-negative finite fp32 m: a GPU test compares all 2^31 of them with
+// __fdiv_rn.  Values below 2^-100 take the IEEE division (their residual
+// could be subnormal).
+__device__ __forceinline__ float div7_rn(float m) {
+    if (m < 0x1p-100f) return __fdiv_rn(m, 7.0f);
+    const float c = 0.142857149f;            // RN(1/7) = 0x3E124925
+    const float q0 = __fmul_rn(m, c);
+    const float r = __fmaf_rn(-q0, 7.0f, m);
+    return __fmaf_rn(r, c, q0);
+}
+
+// div7_rn without the guard for tiny m: equal to it for m >= 2^-100, and for
+// smaller m a value below 2^-25, which rounds to the same fp16 value (zero).
+// Used where only the fp16 rounding of the quotient matters; an infinite m
+// gives NaN.
+__device__ __forceinline__ float div7_rn_for_fp16(float m) {
+    const float c = 0.142857149f;            // RN(1/7)
+    const float q0 = __fmul_rn(m, c);
+    const float r = __fmaf_rn(-q0, 7.0f, m);
+    return __fmaf_rn(r, c, q0);
+}
+
+// Round-to-nearest-even fp32 quotient a / b from y = RN(1/b), for b an fp16
+// value (positive, normal or subnormal) and |a / b| < 2^24: two residual
+// corrections (P. Markstein, "Computation of elementary functions on the
+// IBM RISC System/6000 processor", IBM J. Res. Dev. 34(1), 1990).  The
+// first makes the quotient faithful, the second rounds it correctly.
+// Checked against __fdiv_rn by a GPU test over every fp16 b.
+__device__ __forceinline__ float div_rn_rcp(float a, float b, float y) {
+    float q = __fmul_rn(a, y);
+    float r = __fmaf_rn(-q, b, a);
+    q = __fmaf_rn(r, y, q);
+    r = __fmaf_rn(-q, b, a);
+    return __fmaf_rn(r, y, q);
+}
+
 // Group scale from the group's largest |w * s| (round-to-nearest-even
 // throughout): fp32 quotient by 7, then fp16 unless fp32 scales are asked
 // for.  An fp16 overflow is held at 65504; a non-finite maximum gives NaN.
 // *exact_range is set when every |ws| / scale is known to be below 7.5, so
 // that the code needs no clamp.
 __device__ __forceinline__ float group_scale(float m, bool fp32_scale, bool* exact_range) {
-    const float qsf = __fdiv_rn(m, 7.0f);
+    const float qsf = div7_rn(m);
     float qs;
     bool in_range;
     if (fp32_scale) {

@@ -6,6 +6,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "awq.h"
 
 namespace awq {
@@ -53,10 +55,33 @@ awq_status launch_output_error(const void* X, int64_t T, const void* W, int64_t 
                                void* ws, cudaStream_t stream);
 
 // ---- shared pieces of the search and the output-error mode
-// Writes S[i][j] and tau[i][j] = x_mean[j] / S[i][j] (fp32, [n_grid][d_in]),
-// and clears the device error word (if non-NULL).
-cudaError_t launch_scale_table(const float* x_mean, int64_t d_in, int n_grid,
-                               float* S, float* tau, int* dev_err, cudaStream_t stream);
+// Writes S[i][j] and tau[i][j] = x_mean[j] / S[i][j] (fp32, [n_grid][d_in])
+// with two kernels (pow + per-slice min/max, then normalise); `part` holds
+// 2 * n_grid * kMaxTableSlices doubles.  Clears *dev_words (2 ints: error
+// word, CTA-done counter) if non-NULL.  The second kernel is a programmatic
+// dependent launch of the first.
+constexpr int kMaxTableSlices = 64;
+cudaError_t launch_scale_table(const float* x_mean, int64_t d_in, int n_grid, float* S,
+                               float* tau, double* part, int* dev_words, int num_sms,
+                               cudaStream_t stream);
+
+// Launch with the programmatic stream-serialisation attribute (the kernel
+// must call pdl_wait() before depending on its predecessor).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 // Sums partial[c][i] over c in order, picks the first minimum, copies its row
 // of S into s_best (if non-NULL).
 cudaError_t launch_finalize(const double* partial, int n_parts, int n_grid,

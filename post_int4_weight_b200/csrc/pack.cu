@@ -4,99 +4,191 @@
 // format" and exporter step 4; "AWQ architecture, in depth", section
 // "Quantization, storage and packing").
 //
-//   u[r, j]       = clamp(rint(fl32(w*s) / q_scale), -7, 7) + zero_point
+//   u[r, j]       = clamp(rint(RN(fl32(w*s) / q_scale)), -7, 7) + zero_point
 //   qweight[j, c] = nibble p holds u[8c + order[p], j], order {0,2,4,6,1,3,5,7}
 //   scales[k, r]  = fp16 q_scale;   qzeros[k, c] = zero_point in every nibble
 //
-// HBM-bound: each weight is read once (2 B) and 0.5 B of codes plus the group
-// scale is written.  One CTA handles a 256-row x 128-column tile (one or more
-// whole groups):
-//   phase 1  coalesced 16-byte loads of the tile into shared memory, with the
-//            16-byte chunk index XOR-swizzled by (r ^ r>>5) & 7 so that both
-//            later access patterns are free of bank conflicts;
-//   phase 2  one thread per (row, group): max |w*s| -> q_scale (fp32 quotient
-//            by 7, fp16 round-to-nearest-even), written to `scales`;
-//   phase 3  one thread per (4 columns, 32 rows): codes with the exact IEEE
-//            quotient, nibbles placed in AutoAWQ order, four consecutive
-//            output words per column written with one 16-byte store (eight
-//            threads cover 128 contiguous bytes of a qweight row).
+// HBM-bound: each weight is read once (2 B); 0.5 B of codes plus the group
+// scale (2/g B) and zero word (0.5/g B) are written.  One CTA handles a
+// 128-row x 128-column tile (one to four whole groups):
+//   phase 1  coalesced 16-byte loads of the tile into shared memory, the
+//            16-byte chunk index XOR-swizzled by (r ^ r>>4) & 7 so that the
+//            row-wise reads of phase 2 and the column-wise reads of phase 3
+//            are both free of bank conflicts;
+//   phase 2  two threads per (row, group): max |w*s| (NaN-propagating) ->
+//            q_scale, written to `scales`, and its correctly rounded
+//            reciprocal;
+//   phase 3  one thread per (2 columns, 32 rows): the IEEE quotient from the
+//            reciprocal with two residual corrections (div_rn_rcp), rounding
+//            by the 1.5*2^23 addition, nibble placement with one integer
+//            multiply-add per code, and one 16-byte store per column (four
+//            consecutive output words; four threads write 64 contiguous
+//            bytes of a qweight row).  Row blocks whose scales are all fp16
+//            normal numbers skip the clamp (|quotient| < 7.5 there).
 #include "common.cuh"
 #include "internal.h"
 
 namespace awq {
 namespace {
 
-constexpr int kPackRows = 256;
+constexpr int kPackRows = 128;
 constexpr int kPackCols = 128;
 constexpr int kPackChunks = kPackCols / 8;     // 16-byte chunks per tile row
 constexpr int kPackThreads = 256;
+constexpr int kBlocks32 = kPackRows / 32;      // 32-row blocks per tile
 
-__device__ __forceinline__ int pack_swz(int r) { return (r ^ (r >> 5)) & 7; }
+__device__ __forceinline__ int pack_swz(int r) { return (r ^ (r >> 4)) & 7; }
+
+// Per-row arrays are padded by one slot per 32 rows, so the four rows
+// 32*cq + i that a warp's lanes read together fall in different banks.
+constexpr int kRowStride = kPackRows + kPackRows / 32;
+__device__ __forceinline__ int row_slot(int kk, int r) { return kk * kRowStride + r + (r >> 5); }
 
 // nibble position of row offset r8 (0..7) inside its word: order[p] = r8
 __device__ __forceinline__ constexpr int nibble_of_row(int r8) {
     return (r8 >> 1) + 4 * (r8 & 1);
 }
 
+// NaN-propagating maximum of three values (a NaN anywhere gives NaN)
+__device__ __forceinline__ float max3_nan(float a, float b, float c) {
+    float d;
+    asm("max.NaN.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// |s| of tile column j is kept at j + 4 * (j / 64): the two threads of a
+// (row, group) pair in phase 2 read columns 64 apart, which then fall in
+// different banks.
+__device__ __forceinline__ int sabs_slot(int j) { return j + 4 * (j >> 6); }
+
+template <int G, bool kFast>
+__device__ __forceinline__ void pack_columns(const uint4* tile, const float2* qr_tile,
+                                             const int* bad_tile, int jp, int cq, int kk,
+                                             float2 s2, uint32_t word_init,
+                                             uint32_t words[2][4]) {
+    const float2 magic2 = make_float2(kRoundMagic, kRoundMagic);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        words[0][q] = word_init;
+        words[1][q] = word_init;
+    }
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+        const int r = 32 * cq + i;
+        const uint32_t v = reinterpret_cast<const uint32_t*>(
+            tile + r * kPackChunks + ((jp >> 2) ^ pack_swz(r)))[jp & 3];
+        const float2 qr = qr_tile[row_slot(kk, r)];     // (q_scale, 1/q_scale)
+        const float qs = qr.x, rq = qr.y;
+        const float2 w = __half22float2(*reinterpret_cast<const __half2*>(&v));
+        const float2 a = __fmul2_rn(w, s2);
+        const float2 nb2 = make_float2(-qs, -qs);
+        const float2 y2 = make_float2(rq, rq);
+        // RN(a / qs): two residual corrections of a * RN(1/qs)
+        float2 q = __fmul2_rn(a, y2);
+        float2 res = __ffma2_rn(q, nb2, a);
+        q = __ffma2_rn(res, y2, q);
+        res = __ffma2_rn(q, nb2, a);
+        q = __ffma2_rn(res, y2, q);
+        float2 t = __fadd2_rn(q, magic2);
+        if (!kFast) {
+            t.x = fminf(fmaxf(t.x, kRoundMagic - 7.f), kRoundMagic + 7.f);
+            t.y = fminf(fmaxf(t.y, kRoundMagic - 7.f), kRoundMagic + 7.f);
+            if (bad_tile[row_slot(kk, r)]) t = magic2;   // code = zero point
+        }
+        const uint32_t shift = 1u << (4 * nibble_of_row(i & 7));
+        words[0][i >> 3] += __float_as_uint(t.x) * shift;
+        words[1][i >> 3] += __float_as_uint(t.y) * shift;
+    }
+}
+
 template <int G>
-__global__ void __launch_bounds__(kPackThreads)
+__global__ void __launch_bounds__(kPackThreads, 5)
 pack_kernel(const uint4* __restrict__ W, int64_t d_out, int64_t d_in,
             const float* __restrict__ s, int zero_point, int32_t* __restrict__ qweight,
             __half* __restrict__ scales, int32_t* __restrict__ qzeros) {
     constexpr int KG = kPackCols / G;               // groups per tile
     extern __shared__ __align__(16) unsigned char smem[];
-    uint4* tile = reinterpret_cast<uint4*>(smem);                       // 64 KB
+    uint4* tile = reinterpret_cast<uint4*>(smem);                       // 32 KB
     float* s_tile = reinterpret_cast<float*>(smem + kPackRows * kPackCols * 2);
-    float* qs_tile = s_tile + kPackCols;                                 // [KG][rows]
-    int* bad_tile = reinterpret_cast<int*>(qs_tile + KG * kPackRows);   // [KG][rows]
+    float* sabs_tile = s_tile + kPackCols;                               // |s|, padded
+    float2* qr_tile = reinterpret_cast<float2*>(sabs_tile + kPackCols + 8);  // [KG][kRowStride]
+    int* bad_tile = reinterpret_cast<int*>(qr_tile + KG * kRowStride);  // [KG][kRowStride]
+    int* slow_blk = bad_tile + KG * kRowStride;                          // [KG][kBlocks32]
 
     const int tid = threadIdx.x;
     const int64_t col0 = (int64_t)blockIdx.x * kPackCols;
     const int64_t row0 = (int64_t)blockIdx.y * kPackRows;
     const int64_t ld4 = d_in / 8;
 
-    // ---- phase 1: tile -> shared memory
-    for (int i = tid; i < kPackRows * kPackChunks; i += kPackThreads) {
-        const int r = i / kPackChunks, c = i % kPackChunks;
-        const int64_t gr = row0 + r, gc = col0 + 8 * c;
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (gr < d_out && gc < d_in) v = __ldg(W + gr * ld4 + gc / 8);
-        tile[r * kPackChunks + (c ^ pack_swz(r))] = v;
+    // ---- phase 1: tile -> shared memory (all eight 16-byte loads in flight)
+    {
+        const uint4* base = W + row0 * ld4 + col0 / 8;
+        const int rows_here = (int)min((int64_t)kPackRows, d_out - row0);
+        const int chunks_here = (int)min((int64_t)kPackChunks, (d_in - col0) / 8);
+        uint4 v[kPackRows * kPackChunks / kPackThreads];
+#pragma unroll
+        for (int k = 0; k < kPackRows * kPackChunks / kPackThreads; ++k) {
+            const int i = tid + k * kPackThreads;
+            const int r = i / kPackChunks, c = i % kPackChunks;
+            v[k] = (r < rows_here && c < chunks_here) ? __ldg(base + (int64_t)r * ld4 + c)
+                                                       : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int k = 0; k < kPackRows * kPackChunks / kPackThreads; ++k) {
+            const int i = tid + k * kPackThreads;
+            const int r = i / kPackChunks, c = i % kPackChunks;
+            tile[r * kPackChunks + (c ^ pack_swz(r))] = v[k];
+        }
     }
     if (tid < kPackCols) {
         const int64_t gc = col0 + tid;
-        s_tile[tid] = gc < d_in ? (s ? s[gc] : 1.0f) : 1.0f;
+        const float sv = gc < d_in ? (s ? s[gc] : 1.0f) : 1.0f;
+        s_tile[tid] = sv;
+        sabs_tile[sabs_slot(tid)] = fabsf(sv);
     }
+    if (tid < KG * kBlocks32) slow_blk[tid] = 0;
     __syncthreads();
 
-    // ---- phase 2: group scale of every (row, group)
-    for (int task = tid; task < KG * kPackRows; task += kPackThreads) {
-        const int r = task % kPackRows, kk = task / kPackRows;
+    // ---- phase 2: group scale of every (row, group), two threads each.
+    // max |w s| = max |w| |s|: the sign bits are cleared before the fp16 ->
+    // fp32 conversion, so the products are non-negative and a three-input
+    // NaN-propagating maximum takes two of them per instruction.
+    for (int task = tid; task < 2 * KG * kPackRows; task += kPackThreads) {
+        const int half = task & 1;
+        const int r = (task >> 1) % kPackRows, kk = (task >> 1) / kPackRows;
         float m = 0.f;
-        bool bad = false;
 #pragma unroll
-        for (int cc = 0; cc < G / 8; ++cc) {
-            const int c = kk * (G / 8) + cc;
+        for (int cc = 0; cc < G / 16; ++cc) {
+            const int c = kk * (G / 8) + half * (G / 16) + cc;
             const uint4 v = tile[r * kPackChunks + (c ^ pack_swz(r))];
-            const uint32_t hw[4] = {v.x, v.y, v.z, v.w};
+            const uint32_t hw[4] = {v.x & 0x7fff7fffu, v.y & 0x7fff7fffu, v.z & 0x7fff7fffu,
+                                    v.w & 0x7fff7fffu};
+            const float4 sa = *reinterpret_cast<const float4*>(&sabs_tile[sabs_slot(8 * c)]);
+            const float4 sb = *reinterpret_cast<const float4*>(&sabs_tile[sabs_slot(8 * c + 4)]);
+            const float sv[8] = {sa.x, sa.y, sa.z, sa.w, sb.x, sb.y, sb.z, sb.w};
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const float2 w = __half22float2(*reinterpret_cast<const __half2*>(&hw[i]));
-                const float a = __fmul_rn(w.x, s_tile[8 * c + 2 * i]);
-                const float b = __fmul_rn(w.y, s_tile[8 * c + 2 * i + 1]);
-                bad |= !(fabsf(a) <= 3.402823466e38f) || !(fabsf(b) <= 3.402823466e38f);
-                m = fmaxf(m, fmaxf(fabsf(a), fabsf(b)));
+                const float2 a = __fmul2_rn(w, make_float2(sv[2 * i], sv[2 * i + 1]));
+                m = max3_nan(m, a.x, a.y);
             }
         }
-        bool in_range;
-        float qs = group_scale(m, false, &in_range);
-        if (bad) qs = __int_as_float(0x7fc00000);
-        qs_tile[kk * kPackRows + r] = qs;
-        bad_tile[kk * kPackRows + r] = bad;
-        const int64_t gr = row0 + r, gk = col0 / G + kk;
-        if (gr < d_out && gk * G < d_in)
-            scales[gk * d_out + gr] = bad ? __ushort_as_half((unsigned short)0x7E00)
-                                          : __float2half_rn(qs);
+        {
+            const float o = __shfl_xor_sync(0xffffffffu, m, 1);
+            m = max3_nan(m, o, o);
+        }
+        if (half == 0) {
+            const bool bad = !(m <= 3.402823466e38f);      // a NaN or an infinity
+            bool in_range;
+            const float qs = bad ? 1.0f : group_scale(m, false, &in_range);
+            qr_tile[row_slot(kk, r)] = make_float2(qs, (qs > 0.f) ? __frcp_rn(qs) : 0.f);
+            bad_tile[row_slot(kk, r)] = bad;
+            if (bad || !in_range) slow_blk[kk * kBlocks32 + r / 32] = 1;
+            const int64_t gr = row0 + r, gk = col0 / G + kk;
+            if (gr < d_out && gk * G < d_in)
+                scales[gk * d_out + gr] = bad ? __ushort_as_half((unsigned short)0x7E00)
+                                              : __float2half_rn(qs);
+        }
     }
     __syncthreads();
 
@@ -104,39 +196,21 @@ pack_kernel(const uint4* __restrict__ W, int64_t d_out, int64_t d_in,
     const int64_t C = d_out / 8;
     const int64_t c0 = row0 / 8;
     const uint32_t bias = kRoundMagicBits - (uint32_t)zero_point;
-    for (int task = tid; task < (kPackCols / 4) * (kPackRows / 32); task += kPackThreads) {
-        const int cq = task % (kPackRows / 32);   // 4 output words = 32 rows
-        const int jq = task / (kPackRows / 32);   // 4 input columns
-        const int kk = (4 * jq) / G;
-        float sreg[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) sreg[e] = s_tile[4 * jq + e];
-        uint32_t words[4][4] = {};
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            const int r = 32 * cq + i;
-            const uint2 v = reinterpret_cast<const uint2*>(
-                tile + r * kPackChunks + ((jq >> 1) ^ pack_swz(r)))[jq & 1];
-            const float qs = qs_tile[kk * kPackRows + r];
-            const bool bad = bad_tile[kk * kPackRows + r] != 0;
-            const float2 w01 = __half22float2(*reinterpret_cast<const __half2*>(&v.x));
-            const float2 w23 = __half22float2(*reinterpret_cast<const __half2*>(&v.y));
-            const float wv[4] = {w01.x, w01.y, w23.x, w23.y};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float ws = __fmul_rn(wv[e], sreg[e]);
-                const float y = (qs > 0.f) ? __fdiv_rn(ws, qs) : 0.f;
-                float t = __fadd_rn(y, kRoundMagic);
-                t = fminf(fmaxf(t, kRoundMagic - 7.f), kRoundMagic + 7.f);
-                uint32_t u = __float_as_uint(t) - bias;
-                if (bad) u = (uint32_t)zero_point;
-                words[e][i >> 3] |= (u & 0xFu) << (4 * nibble_of_row(i & 7));
-            }
-        }
+    const uint32_t word_init = 0u - bias * 0x11111111u;
+    {
+        const int cq = tid & 3;          // 4 output words = 32 rows
+        const int jp = tid >> 2;         // 2 input columns
+        const int kk = (2 * jp) / G;
+        const float2 s2 = make_float2(s_tile[2 * jp], s_tile[2 * jp + 1]);
+        uint32_t words[2][4];
+        if (slow_blk[kk * kBlocks32 + cq])
+            pack_columns<G, false>(tile, qr_tile, bad_tile, jp, cq, kk, s2, word_init, words);
+        else
+            pack_columns<G, true>(tile, qr_tile, bad_tile, jp, cq, kk, s2, word_init, words);
         const int64_t cw = c0 + 4 * cq;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const int64_t j = col0 + 4 * jq + e;
+        for (int e = 0; e < 2; ++e) {
+            const int64_t j = col0 + 2 * jp + e;
             if (j >= d_in) continue;
             int32_t* dst = qweight + j * C + cw;
             if ((C & 3) == 0 && cw + 3 < C) {
@@ -151,9 +225,7 @@ pack_kernel(const uint4* __restrict__ W, int64_t d_out, int64_t d_in,
 
     // ---- qzeros of the tile's groups and words
     uint32_t zword = (uint32_t)zero_point & 0xFu;
-    zword |= zword << 4;
-    zword |= zword << 8;
-    zword |= zword << 16;
+    zword *= 0x11111111u;
     for (int i = tid; i < KG * (kPackRows / 8); i += kPackThreads) {
         const int kk = i / (kPackRows / 8), cwl = i % (kPackRows / 8);
         const int64_t gk = col0 / G + kk, cw = c0 + cwl;
@@ -166,12 +238,19 @@ cudaError_t launch_pack_G(const void* W, int64_t d_out, int64_t d_in, const floa
                           int zero_point, int32_t* qweight, void* scales, int32_t* qzeros,
                           cudaStream_t stream) {
     constexpr int KG = kPackCols / G;
-    const size_t smem = (size_t)kPackRows * kPackCols * 2 + kPackCols * sizeof(float) +
-                        (size_t)KG * kPackRows * (sizeof(float) + sizeof(int));
-    cudaError_t e = cudaFuncSetAttribute(pack_kernel<G>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
-    if (e != cudaSuccess) return e;
+    const size_t smem = (size_t)kPackRows * kPackCols * 2 + (2 * kPackCols + 8) * sizeof(float) +
+                        (size_t)KG * kRowStride * (sizeof(float2) + sizeof(int)) +
+                        (size_t)KG * kBlocks32 * sizeof(int);
+    static int configured[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64 || !configured[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(pack_kernel<G>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem);
+        if (e != cudaSuccess) return e;
+        if (dev >= 0 && dev < 64) configured[dev] = 1;
+    }
     dim3 grid((unsigned)((d_in + kPackCols - 1) / kPackCols),
               (unsigned)((d_out + kPackRows - 1) / kPackRows));
     pack_kernel<G><<<grid, kPackThreads, smem, stream>>>(

@@ -7,18 +7,22 @@
 // W*s_i is fake-quantised group-wise to symmetric INT4 with an fp16 group
 // scale, and scored by sum(((W - Q(W s_i)/s_i) * x)^2).
 //
-// Kernels (all on the caller's stream):
-//   scale_table_kernel  one CTA per alpha: s_i in fp64 (pow, max, min, sqrt),
-//                       rounded to fp32, and tau_i = x / s_i;
-//   search_kernel       persistent, 2 CTAs per SM.  A work unit is one group
-//                       of g input channels x R rows of one weight segment.
-//                       Thread 0 streams units into a 2-stage shared-memory
-//                       ring with TMA (cp.async.bulk.tensor, mbarrier
-//                       completion); W is read from HBM exactly once and kept
-//                       in registers as fp32 while all grid points are
-//                       evaluated;
-//   finalize_kernel     sums the per-CTA partials in a fixed order (fp64),
-//                       picks the first minimum and copies s_best.
+// Kernels (all on the caller's stream; the second and third are programmatic
+// dependent launches of the one before):
+//   table_minmax_kernel  (slices x alphas) CTAs: s_i[j] = max(x,1e-4)^alpha in
+//                        fp64, per-slice min and max;
+//   table_write_kernel   same grid: sqrt(max*min) from the slice partials,
+//                        s_i rounded to fp32 and tau_i = x / s_i;
+//   search_kernel        persistent, 2 CTAs per SM.  A work unit is one group
+//                        of g input channels x R rows of one weight segment.
+//                        Thread 0 streams units into a 2-stage shared-memory
+//                        ring with TMA (cp.async.bulk.tensor, mbarrier
+//                        completion), starting before the scale table is
+//                        ready; W is read from HBM exactly once and kept in
+//                        registers as fp32 while all grid points are
+//                        evaluated.  The last CTA to finish sums the per-CTA
+//                        partials in a fixed order (fp64), picks the first
+//                        minimum and copies s_best.
 //
 // Register-level formulation of one (weight, alpha) pair, 6 FMA-pipe ops plus
 // one max, issued as packed fp32x2 instructions (sm_100):
@@ -47,7 +51,7 @@ namespace {
 constexpr int kConsumerWarps = 8;
 constexpr int kThreads = kConsumerWarps * 32;
 constexpr int kStages = 2;
-constexpr int kElemsPerLane = 32;          // weights of one row held per lane
+constexpr int kElemsPerRow = 16;           // weights of each of a lane's two rows
 constexpr int kUnitBytes = 16384;          // R * g * 2 for every group size
 constexpr int kMaxGrid = 32;
 
@@ -64,57 +68,163 @@ struct SearchParams {
     const float* S;        // [n_grid][d_in]
     const float* tau;      // [n_grid][d_in]
     double* partial;       // [gridDim.x][n_grid]
-    int* dev_err;
+    int* dev_words;        // [0] error bits, [1] CTAs done
+    double* err;           // [n_grid] output
+    int32_t* best_idx;     // [1] output
+    float* s_best;         // [d_in] output
 };
 
 __device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
 
-// Shared-memory layout of one alpha's table slice for a group of g = 32*L
-// channels: float4 index (k4*2 + h)*L + l holds channels 8*(l + L*k4) + 4*h
+// Shared-memory layout of one alpha's table slice for a group of g = 16*L
+// channels: float4 index (k2*2 + h)*L + l holds channels 8*(l + L*k2) + 4*h
 // + 0..3, so the L lanes of a row read L consecutive 16-byte words (all rows
 // of the warp read the same words: a broadcast).
 template <int L>
 __device__ __forceinline__ int table_slot(int c) {
     const int chunk = c >> 3;
-    const int l = chunk % L, k4 = chunk / L, h = (c >> 2) & 1, e = c & 3;
-    return (((k4 * 2 + h) * L + l) << 2) + e;
+    const int l = chunk % L, k2 = chunk / L, h = (c >> 2) & 1, e = c & 3;
+    return (((k2 * 2 + h) * L + l) << 2) + e;
 }
 
-template <int L>
+// Sum of the CTAs' partial errors in a fixed order (lane-strided, then a
+// fixed shuffle tree), the first minimum, and s_best.  Run by one CTA of
+// kThreads threads after every partial is visible.
+__device__ void finalize_cta(const double* partial, int n_parts, int n_grid,
+                             const float* S, int64_t d_in, int dev_err, double* err,
+                             int32_t* best_idx, float* s_best, double* e_s, int* best_s) {
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    for (int a = warp; a < n_grid; a += kThreads / 32) {
+        double s = 0.0;
+        for (int c = lane; c < n_parts; c += 32)
+            s += __ldcg(partial + (int64_t)c * n_grid + a);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+        if (lane == 0) {
+            e_s[a] = s;
+            err[a] = s;
+        }
+    }
+    __syncthreads();
+    if (tid == 0) {
+        int b = 0;
+        bool finite = true;
+        for (int i = 0; i < n_grid; ++i) {
+            if (!isfinite(e_s[i])) finite = false;
+            if (e_s[i] < e_s[b]) b = i;
+        }
+        if (!finite) b = -1;
+        if (dev_err) b = -2;
+        *best_s = b;
+        *best_idx = b;
+    }
+    __syncthreads();
+    if (s_best) {
+        const int b = *best_s;
+        for (int64_t j = tid; j < d_in; j += kThreads)
+            s_best[j] = b >= 0 ? __ldcg(S + (int64_t)b * d_in + j) : __int_as_float(0x7fc00000);
+    }
+}
+
+// Pass 1 of one row: ws = w * s (exact fp32 products, packed fp32x2) and the
+// lane's largest |ws|.
+__device__ __forceinline__ float row_products(const float2* w, const float4* s4, float2* ws) {
+    float mx[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        ws[2 * k] = __fmul2_rn(w[2 * k], f2(s4[k].x, s4[k].y));
+        ws[2 * k + 1] = __fmul2_rn(w[2 * k + 1], f2(s4[k].z, s4[k].w));
+        mx[k] = fmaxf(fmaxf(fabsf(ws[2 * k].x), fabsf(ws[2 * k].y)),
+                      fmaxf(fabsf(ws[2 * k + 1].x), fabsf(ws[2 * k + 1].y)));
+    }
+    return fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+}
+
+// q_scale of a row from its largest |ws| (the lane-local maxima combined
+// over the row's L lanes), its approximate reciprocal, and whether every
+// |ws| / q_scale of the row is known to stay below 7.5 (then the code needs
+// no clamp and the reciprocal is finite).  Non-finite ws need no flag here:
+// they make the row's error non-finite on their own.
+template <int L, bool kFp32>
+__device__ __forceinline__ void row_scale(float m, float* qs, float* rq, bool* in_range) {
+#pragma unroll
+    for (int o = 1; o < L; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (kFp32) {
+        const float q = div7_rn(m);
+        *qs = q;
+        *in_range = q >= kFloatMinNormal && q <= 3.402823466e38f;
+    } else {
+        const float qsf = div7_rn_for_fp16(m);
+        const float q = __half2float(__float2half_rn(qsf));
+        *in_range = (q >= kHalfMinNormal) & (q <= kHalfMax);
+        *qs = fminf(q, kHalfMax);
+    }
+    *rq = rcp_approx(*qs);
+}
+
+// Pass 2 of one row: codes from the reciprocal of q_scale and squared
+// weighted errors into two independent accumulators.  The packed fp32x2
+// instructions run on one of the two FMA sub-pipes only, scalar ones on
+// either: half of the work per pair is issued packed (the residual d and
+// the accumulation) and half scalar (the rounding t, q and the weighting e),
+// which keeps both sub-pipes busy for the fewest issue slots.  kClamp
+// handles a q_scale that is zero, fp16-subnormal or held at 65504 (codes
+// beyond +-7 are clamped, a zero scale gives code 0).
+template <bool kClamp, int L>
+__device__ __forceinline__ float2 row_errors(const float2* ws, const float4* Ta, int l,
+                                             float qs, float rq) {
+    if (kClamp && !(qs > 0.f)) rq = 0.f;
+    const float2 nqs2 = f2(-qs, -qs);
+    float2 acc2[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const float4 tv = Ta[k * L + l];
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            const int i = 2 * k + j;
+            float tx = __fmaf_rn(ws[i].x, rq, kRoundMagic);
+            float ty = __fmaf_rn(ws[i].y, rq, kRoundMagic);
+            if (kClamp) {
+                tx = fminf(fmaxf(tx, kRoundMagic - 7.f), kRoundMagic + 7.f);
+                ty = fminf(fmaxf(ty, kRoundMagic - 7.f), kRoundMagic + 7.f);
+            }
+            const float2 q = f2(__fadd_rn(tx, -kRoundMagic), __fadd_rn(ty, -kRoundMagic));
+            const float2 d = __ffma2_rn(q, nqs2, ws[i]);
+            const float2 e = j ? f2(__fmul_rn(d.x, tv.z), __fmul_rn(d.y, tv.w))
+                               : f2(__fmul_rn(d.x, tv.x), __fmul_rn(d.y, tv.y));
+            acc2[j] = __ffma2_rn(e, e, acc2[j]);
+        }
+    }
+    return __fadd2_rn(acc2[0], acc2[1]);
+}
+
+template <int L, bool kFp32>
 __global__ void __launch_bounds__(kThreads, 2)
 search_kernel(const __grid_constant__ SearchParams p) {
-    constexpr int G = 32 * L;                    // group size
-    constexpr int R = kConsumerWarps * 32 / L;   // rows per unit
+    constexpr int G = 16 * L;                    // group size
+    constexpr int RPW = 2 * 32 / L;              // rows per warp (two per lane)
+    constexpr int R = kConsumerWarps * RPW;      // rows per unit
     static_assert(R * G * 2 == kUnitBytes, "unit size");
 
     extern __shared__ __align__(1024) unsigned char smem[];
     unsigned char* stage_base = smem;                                   // kStages * 16 KB
-    float* tab = reinterpret_cast<float*>(smem + kStages * kUnitBytes); // n_grid * 2 * G
-    double* acc = reinterpret_cast<double*>(tab + p.n_grid * 2 * G);    // n_grid * kThreads
+    float* tab = reinterpret_cast<float*>(smem + kStages * kUnitBytes); // (n_grid+1) * 2 * G
+    double* wacc = reinterpret_cast<double*>(tab + (p.n_grid + 1) * 2 * G);  // n_grid * warps
+    float* acc = reinterpret_cast<float*>(wacc + p.n_grid * kConsumerWarps);   // n_grid * kThreads
     uint64_t* full = reinterpret_cast<uint64_t*>(acc + p.n_grid * kThreads);
     uint64_t* empty = full + kStages;
-    int* abort_flag = reinterpret_cast<int*>(empty + kStages);
+    int* flags_s = reinterpret_cast<int*>(empty + kStages);   // [0] abort, [1] last, [2] best
+    double* e_s = wacc;                                       // reused by the last CTA
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
-    const int row = warp * (32 / L) + lane / L;   // row within the unit
+    const int row = warp * RPW + lane / L;        // first row within the unit
     const int l = lane % L;                       // sub-lane within the row
+    // the lane's second row is row + 32 / L
 
     // contiguous, balanced range of units for this CTA
     const int64_t u0 = p.n_units * blockIdx.x / gridDim.x;
     const int64_t u1 = p.n_units * (blockIdx.x + 1) / gridDim.x;
-
-    for (int i = tid; i < p.n_grid * kThreads; i += kThreads) acc[i] = 0.0;
-    if (tid == 0) {
-        *abort_flag = 0;
-        for (int s = 0; s < kStages; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], kConsumerWarps);
-        }
-        mbar_fence_init();
-        for (int k = 0; k < p.n_seg; ++k) tma_prefetch_desc(&p.tmap[k]);
-    }
-    __syncthreads();
 
     // unit -> (segment, group, row block)
     auto decode = [&](int64_t u, int* seg, int* grp, int* rb) {
@@ -135,11 +245,22 @@ search_kernel(const __grid_constant__ SearchParams p) {
         ++issued[stage];
     };
 
+    // prologue, overlapping the scale-table kernels: W does not depend on them
     if (tid == 0) {
+        flags_s[0] = 0;
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kConsumerWarps);
+        }
+        mbar_fence_init();
+        for (int k = 0; k < p.n_seg; ++k) tma_prefetch_desc(&p.tmap[k]);
         for (int s = 0; s < kStages && u0 + s < u1; ++s) issue(u0 + s, s);
     }
+    for (int i = tid; i < p.n_grid * kThreads; i += kThreads) acc[i] = 0.f;
+    for (int i = tid; i < p.n_grid * kConsumerWarps; i += kThreads) wacc[i] = 0.0;
+    pdl_wait();          // the scale table (and the cleared counters) are ready
+    __syncthreads();
 
-    const bool fp32_scale = (p.flags & AWQ_SCALE_FP32) != 0;
     const float2 magic2 = f2(kRoundMagic, kRoundMagic);
     const float2 nmagic2 = f2(-kRoundMagic, -kRoundMagic);
     int cur_grp = -1;
@@ -157,11 +278,11 @@ search_kernel(const __grid_constant__ SearchParams p) {
         if (tid == 0 && it >= 1 && u + 1 < u1 && !failed) {
             const int ps = (it - 1) % kStages;
             const uint32_t pp = (uint32_t)((it - 1) / kStages) & 1u;
-            if (*(volatile int*)abort_flag == 0 && mbar_wait_bounded(&empty[ps], pp)) {
+            if (*(volatile int*)&flags_s[0] == 0 && mbar_wait_bounded(&empty[ps], pp)) {
                 issue(u + 1, ps);
             } else {
-                atomicOr(p.dev_err, kDevErrWaitTimeout);
-                *(volatile int*)abort_flag = 1;
+                atomicOr(&p.dev_words[0], kDevErrWaitTimeout);
+                *(volatile int*)&flags_s[0] = 1;
                 failed = true;
             }
         }
@@ -175,20 +296,19 @@ search_kernel(const __grid_constant__ SearchParams p) {
             for (int i = tid; i < p.n_grid * G; i += kThreads) {
                 const int a = i / G, c = i % G;
                 const int slot = table_slot<L>(c);
-                tab[a * 2 * G + slot] = Sg[(int64_t)a * p.d_in + c];
-                tab[a * 2 * G + G + slot] = Tg[(int64_t)a * p.d_in + c];
+                tab[a * 2 * G + slot] = __ldcg(Sg + (int64_t)a * p.d_in + c);
+                tab[a * 2 * G + G + slot] = __ldcg(Tg + (int64_t)a * p.d_in + c);
             }
+            for (int i = tid; i < 2 * G; i += kThreads) tab[p.n_grid * 2 * G + i] = 0.f;
             cur_grp = grp;
             __syncthreads();
         }
 
-        bool ok = !failed && *(volatile int*)abort_flag == 0;
+        bool ok = !failed && *(volatile int*)&flags_s[0] == 0;
         if (ok) ok = mbar_wait_bounded(&full[stage], parity);
-        if (!failed && !ok) {
-            if (lane == 0) {
-                atomicOr(p.dev_err, kDevErrWaitTimeout);
-                *(volatile int*)abort_flag = 1;
-            }
+        if (!failed && !ok && lane == 0) {
+            atomicOr(&p.dev_words[0], kDevErrWaitTimeout);
+            *(volatile int*)&flags_s[0] = 1;
         }
         failed = __any_sync(0xffffffffu, !ok) || failed;
         if (failed) {
@@ -196,18 +316,21 @@ search_kernel(const __grid_constant__ SearchParams p) {
             if (lane == 0) mbar_arrive(&empty[stage]);
             continue;
         }
-        // this lane's 32 weights: chunks l + L*k4 (8 channels each) of its row
-        float2 w[kElemsPerLane / 2];
+        // this lane's weights: chunks l and l + L (8 channels each) of its two rows
+        float2 w[2][kElemsPerRow / 2];
         {
-            const uint4* src = reinterpret_cast<const uint4*>(
-                stage_base + stage * kUnitBytes + row * G * 2);
 #pragma unroll
-            for (int k4 = 0; k4 < 4; ++k4) {
-                const uint4 v = src[l + L * k4];
-                const uint32_t hw[4] = {v.x, v.y, v.z, v.w};
+            for (int rr = 0; rr < 2; ++rr) {
+                const uint4* src = reinterpret_cast<const uint4*>(
+                    stage_base + stage * kUnitBytes + (row + rr * (32 / L)) * G * 2);
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    w[k4 * 4 + i] = __half22float2(*reinterpret_cast<const __half2*>(&hw[i]));
+                for (int k2 = 0; k2 < 2; ++k2) {
+                    const uint4 v = src[l + L * k2];
+                    const uint32_t hw[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        w[rr][k2 * 4 + i] =
+                            __half22float2(*reinterpret_cast<const __half2*>(&hw[i]));
                 }
             }
         }
@@ -217,70 +340,36 @@ search_kernel(const __grid_constant__ SearchParams p) {
         for (int a = 0; a < p.n_grid; ++a) {
             const float4* Sa = reinterpret_cast<const float4*>(tab + a * 2 * G);
             const float4* Ta = reinterpret_cast<const float4*>(tab + a * 2 * G + G);
-            float2 ws[kElemsPerLane / 2];
-            float m0 = 0.f, m1 = 0.f;
+            float4 s4[4];
 #pragma unroll
-            for (int k4 = 0; k4 < 4; ++k4) {
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const float4 s4 = Sa[(k4 * 2 + h) * L + l];
-                    const int i0 = k4 * 4 + h * 2;
-                    ws[i0] = __fmul2_rn(w[i0], f2(s4.x, s4.y));
-                    ws[i0 + 1] = __fmul2_rn(w[i0 + 1], f2(s4.z, s4.w));
-                    m0 = fmaxf(m0, fmaxf(fabsf(ws[i0].x), fabsf(ws[i0].y)));
-                    m1 = fmaxf(m1, fmaxf(fabsf(ws[i0 + 1].x), fabsf(ws[i0 + 1].y)));
-                }
+            for (int k = 0; k < 4; ++k) s4[k] = Sa[k * L + l];
+            float2 ws[2][kElemsPerRow / 2];
+            const float m0 = row_products(w[0], s4, ws[0]);
+            const float m1 = row_products(w[1], s4, ws[1]);
+            float qs0, rq0, qs1, rq1;
+            bool in0, in1;
+            row_scale<L, kFp32>(m0, &qs0, &rq0, &in0);
+            row_scale<L, kFp32>(m1, &qs1, &rq1, &in1);
+            float2 e;
+            if (__all_sync(0xffffffffu, in0 & in1)) {
+                e = __fadd2_rn(row_errors<false, L>(ws[0], Ta, l, qs0, rq0),
+                               row_errors<false, L>(ws[1], Ta, l, qs1, rq1));
+            } else {   // some row has an fp16-subnormal, overflowing, zero or NaN scale
+                e = __fadd2_rn(row_errors<true, L>(ws[0], Ta, l, qs0, rq0),
+                               row_errors<true, L>(ws[1], Ta, l, qs1, rq1));
             }
-            float m = fmaxf(m0, m1);
+            acc[a * kThreads + tid] += e.x + e.y;
+        }
+        // every 8 units the per-thread fp32 partials move into the warp's fp64
+        // accumulators (fixed order), bounding fp32 accumulation to 8 units
+        if (((it + 1) & 7) == 0 || u + 1 == u1) {
+            for (int a = 0; a < p.n_grid; ++a) {
+                double v = (double)acc[a * kThreads + tid];
+                acc[a * kThreads + tid] = 0.f;
 #pragma unroll
-            for (int o = 1; o < L; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-
-            bool in_range;
-            const float qs = group_scale(m, fp32_scale, &in_range);
-            const float rq = (qs > 0.f) ? __frcp_rn(qs) : 0.f;
-            const float2 rq2 = f2(rq, rq);
-            const float2 nqs2 = f2(-qs, -qs);
-            float2 acc2 = f2(0.f, 0.f);
-            if (in_range) {
-#pragma unroll
-                for (int k4 = 0; k4 < 4; ++k4) {
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const float4 t4 = Ta[(k4 * 2 + h) * L + l];
-                        const int i0 = k4 * 4 + h * 2;
-#pragma unroll
-                        for (int j = 0; j < 2; ++j) {
-                            const float2 tau = j ? f2(t4.z, t4.w) : f2(t4.x, t4.y);
-                            const float2 t = __ffma2_rn(ws[i0 + j], rq2, magic2);
-                            const float2 q = __fadd2_rn(t, nmagic2);
-                            const float2 d = __ffma2_rn(q, nqs2, ws[i0 + j]);
-                            const float2 e = __fmul2_rn(d, tau);
-                            acc2 = __ffma2_rn(e, e, acc2);
-                        }
-                    }
-                }
-            } else {   // fp16-subnormal, overflowing, zero or NaN scale: clamp codes
-#pragma unroll
-                for (int k4 = 0; k4 < 4; ++k4) {
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const float4 t4 = Ta[(k4 * 2 + h) * L + l];
-                        const int i0 = k4 * 4 + h * 2;
-#pragma unroll
-                        for (int j = 0; j < 2; ++j) {
-                            const float2 tau = j ? f2(t4.z, t4.w) : f2(t4.x, t4.y);
-                            float2 t = __ffma2_rn(ws[i0 + j], rq2, magic2);
-                            t.x = fminf(fmaxf(t.x, kRoundMagic - 7.f), kRoundMagic + 7.f);
-                            t.y = fminf(fmaxf(t.y, kRoundMagic - 7.f), kRoundMagic + 7.f);
-                            const float2 q = __fadd2_rn(t, nmagic2);
-                            const float2 d = __ffma2_rn(q, nqs2, ws[i0 + j]);
-                            const float2 e = __fmul2_rn(d, tau);
-                            acc2 = __ffma2_rn(e, e, acc2);
-                        }
-                    }
-                }
+                for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+                if (lane == 0) wacc[a * kConsumerWarps + warp] += v;
             }
-            acc[a * kThreads + tid] += (double)(acc2.x + acc2.y);
         }
     }
 
@@ -292,28 +381,51 @@ search_kernel(const __grid_constant__ SearchParams p) {
     }
     __syncthreads();
 
-    // fixed-order reduction of the per-thread partials: warp w reduces
-    // grid points a = w, w + 8, ...
-    for (int a = warp; a < p.n_grid; a += kConsumerWarps) {
-        double s = 0.0;
-        for (int i = lane; i < kThreads; i += 32) s += acc[a * kThreads + i];
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-        if (lane == 0) p.partial[(int64_t)blockIdx.x * p.n_grid + a] = s;
+    // fixed-order reduction of the per-warp partials
+    if (tid < p.n_grid) {
+        double v = 0.0;
+        for (int w8 = 0; w8 < kConsumerWarps; ++w8) v += wacc[tid * kConsumerWarps + w8];
+        p.partial[(int64_t)blockIdx.x * p.n_grid + tid] = v;
+    }
+
+    // the last CTA to arrive reduces every partial
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) {
+        const int done = atomicAdd(&p.dev_words[1], 1);
+        flags_s[1] = (done == (int)gridDim.x - 1);
+    }
+    __syncthreads();
+    if (flags_s[1]) {
+        __threadfence();
+        finalize_cta(p.partial, gridDim.x, p.n_grid, p.S, p.d_in,
+                     *(volatile int*)&p.dev_words[0], p.err, p.best_idx, p.s_best, e_s,
+                     &flags_s[2]);
     }
 }
 
+// ---- scale table: s_i[j] = max(x_j, 1e-4)^alpha_i / sqrt(max_j * min_j)
+
+__device__ __forceinline__ double table_pow(const float* x, int64_t j, double alpha) {
+    return pow((double)fmaxf(x[j], 1e-4f), alpha);
+}
+
 __global__ void __launch_bounds__(256)
-scale_table_kernel(const float* __restrict__ x, int64_t d_in, int n_grid,
-                   float* __restrict__ S, float* __restrict__ tau, int* __restrict__ dev_err) {
-    __shared__ double red_mx[32], red_mn[32];
-    const int a = blockIdx.x;
-    if (dev_err && a == 0 && threadIdx.x == 0) *dev_err = 0;
+table_minmax_kernel(const float* __restrict__ x, int64_t d_in, int n_grid, int64_t slice,
+                    double* __restrict__ part, int* __restrict__ dev_words) {
+    __shared__ double red_mx[8], red_mn[8];
+    pdl_launch_dependents();
+    const int a = blockIdx.y;
+    const int sl = blockIdx.x;
+    if (dev_words && a == 0 && sl == 0 && threadIdx.x == 0) {
+        dev_words[0] = 0;
+        dev_words[1] = 0;
+    }
     const double alpha = __ddiv_rn((double)a, (double)n_grid);
-    double mx = -__longlong_as_double(0x7ff0000000000000ll);
-    double mn = __longlong_as_double(0x7ff0000000000000ll);
-    for (int64_t j = threadIdx.x; j < d_in; j += blockDim.x) {
-        const double sd = pow((double)fmaxf(x[j], 1e-4f), alpha);
+    double mx = 0.0, mn = __longlong_as_double(0x7ff0000000000000ll);
+    const int64_t j0 = (int64_t)sl * slice, j1 = min(d_in, j0 + slice);
+    for (int64_t j = j0 + threadIdx.x; j < j1; j += blockDim.x) {
+        const double sd = table_pow(x, j, alpha);
         mx = fmax(mx, sd);
         mn = fmin(mn, sd);
     }
@@ -327,70 +439,56 @@ scale_table_kernel(const float* __restrict__ x, int64_t d_in, int n_grid,
         red_mn[threadIdx.x >> 5] = mn;
     }
     __syncthreads();
-    if (threadIdx.x < 32) {
-        const int nw = blockDim.x >> 5;
-        mx = threadIdx.x < nw ? red_mx[threadIdx.x] : red_mx[0];
-        mn = threadIdx.x < nw ? red_mn[threadIdx.x] : red_mn[0];
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-            mn = fmin(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    if (threadIdx.x == 0) {
+        for (int k = 1; k < (int)(blockDim.x >> 5); ++k) {
+            mx = fmax(mx, red_mx[k]);
+            mn = fmin(mn, red_mn[k]);
         }
-        if (threadIdx.x == 0) {
-            red_mx[0] = mx;
-            red_mn[0] = mn;
-        }
+        part[((int64_t)a * gridDim.x + sl) * 2 + 0] = fmax(mx, red_mx[0]);
+        part[((int64_t)a * gridDim.x + sl) * 2 + 1] = fmin(mn, red_mn[0]);
     }
-    __syncthreads();
-    const double norm = __dsqrt_rn(__dmul_rn(red_mx[0], red_mn[0]));
-    for (int64_t j = threadIdx.x; j < d_in; j += blockDim.x) {
-        const double sd = pow((double)fmaxf(x[j], 1e-4f), alpha);
-        const float s = __double2float_rn(__ddiv_rn(sd, norm));
+}
+
+__global__ void __launch_bounds__(256)
+table_write_kernel(const float* __restrict__ x, int64_t d_in, int n_grid, int64_t slice,
+                   const double* __restrict__ part, float* __restrict__ S,
+                   float* __restrict__ tau) {
+    pdl_launch_dependents();
+    pdl_wait();
+    const int a = blockIdx.y;
+    const int sl = blockIdx.x;
+    double mx = 0.0, mn = __longlong_as_double(0x7ff0000000000000ll);
+    for (int k = 0; k < (int)gridDim.x; ++k) {   // max and min are order-independent
+        mx = fmax(mx, __ldcg(part + ((int64_t)a * gridDim.x + k) * 2 + 0));
+        mn = fmin(mn, __ldcg(part + ((int64_t)a * gridDim.x + k) * 2 + 1));
+    }
+    const double norm = __dsqrt_rn(__dmul_rn(mx, mn));
+    const double alpha = __ddiv_rn((double)a, (double)n_grid);
+    const int64_t j0 = (int64_t)sl * slice, j1 = min(d_in, j0 + slice);
+    for (int64_t j = j0 + threadIdx.x; j < j1; j += blockDim.x) {
+        const float s = __double2float_rn(__ddiv_rn(table_pow(x, j, alpha), norm));
         S[(int64_t)a * d_in + j] = s;
         tau[(int64_t)a * d_in + j] = __fdiv_rn(x[j], s);
     }
 }
 
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(kThreads)
 finalize_kernel(const double* __restrict__ partial, int n_parts, int n_grid,
                 const float* __restrict__ S, int64_t d_in, const int* __restrict__ dev_err,
                 double* __restrict__ err, int32_t* __restrict__ best_idx,
                 float* __restrict__ s_best) {
     __shared__ double e_s[kMaxGrid];
     __shared__ int best_s;
-    const int t = threadIdx.x;
-    if (t < n_grid) {
-        double s = 0.0;
-        for (int c = 0; c < n_parts; ++c) s += partial[(int64_t)c * n_grid + t];
-        e_s[t] = s;
-        err[t] = s;
-    }
-    __syncthreads();
-    if (t == 0) {
-        int b = 0;
-        bool finite = true;
-        for (int i = 0; i < n_grid; ++i) {
-            if (!isfinite(e_s[i])) finite = false;
-            if (e_s[i] < e_s[b]) b = i;
-        }
-        if (!finite) b = -1;
-        if (dev_err && *dev_err) b = -2;
-        best_s = b;
-        *best_idx = b;
-    }
-    __syncthreads();
-    if (s_best) {
-        const int b = best_s;
-        for (int64_t j = t; j < d_in; j += blockDim.x)
-            s_best[j] = b >= 0 ? S[(int64_t)b * d_in + j] : __int_as_float(0x7fc00000);
-    }
+    pdl_wait();
+    finalize_cta(partial, n_parts, n_grid, S, d_in, dev_err ? *dev_err : 0, err, best_idx,
+                 s_best, e_s, &best_s);
 }
 
 struct SearchWs {
     float* S;
     float* tau;
     double* partial;
-    int* dev_err;
+    int* dev_words;
 };
 
 size_t max_search_ctas() { return 1024; }
@@ -402,24 +500,41 @@ SearchWs carve_search_ws(void* ws, int64_t d_in, int n_grid) {
     w.S = reinterpret_cast<float*>(p);
     w.tau = reinterpret_cast<float*>(p + tab);
     w.partial = reinterpret_cast<double*>(p + 2 * tab);
-    w.dev_err = reinterpret_cast<int*>(
+    w.dev_words = reinterpret_cast<int*>(
         p + 2 * tab + align_up(max_search_ctas() * kMaxGrid * sizeof(double), kWsAlign));
     return w;
 }
 
 size_t search_smem_bytes(int group_size, int n_grid) {
-    return (size_t)kStages * kUnitBytes + (size_t)n_grid * 2 * group_size * sizeof(float) +
-           (size_t)n_grid * kThreads * sizeof(double) + 2 * kStages * sizeof(uint64_t) + 16;
+    return (size_t)kStages * kUnitBytes + (size_t)(n_grid + 1) * 2 * group_size * sizeof(float) +
+           (size_t)n_grid * kConsumerWarps * sizeof(double) +
+           (size_t)n_grid * kThreads * sizeof(float) + 2 * kStages * sizeof(uint64_t) + 16;
 }
 
-template <int L>
+template <int L, bool kFp32>
 cudaError_t launch_search_L(const SearchParams& p, int grid, size_t smem, cudaStream_t st) {
-    cudaError_t e = cudaFuncSetAttribute(search_kernel<L>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
-    if (e != cudaSuccess) return e;
-    search_kernel<L><<<grid, kThreads, smem, st>>>(p);
-    return cudaGetLastError();
+    static int configured_smem[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64 || configured_smem[dev] < (int)smem) {
+        cudaError_t e = cudaFuncSetAttribute(search_kernel<L, kFp32>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem);
+        if (e != cudaSuccess) return e;
+        if (dev >= 0 && dev < 64) configured_smem[dev] = (int)smem;
+    }
+    return launch_pdl(search_kernel<L, kFp32>, dim3(grid), dim3(kThreads), smem, st, p);
+}
+
+template <bool kFp32>
+cudaError_t launch_search(int L, const SearchParams& p, int grid, size_t smem,
+                          cudaStream_t st) {
+    switch (L) {
+        case 2: return launch_search_L<2, kFp32>(p, grid, smem, st);
+        case 4: return launch_search_L<4, kFp32>(p, grid, smem, st);
+        case 8: return launch_search_L<8, kFp32>(p, grid, smem, st);
+        default: return cudaErrorInvalidValue;
+    }
 }
 
 }  // namespace
@@ -432,17 +547,27 @@ size_t scale_search_workspace(int64_t d_in, int group_size, int n_grid) {
 }
 
 cudaError_t launch_scale_table(const float* x_mean, int64_t d_in, int n_grid, float* S,
-                               float* tau, int* dev_err, cudaStream_t stream) {
-    scale_table_kernel<<<n_grid, 256, 0, stream>>>(x_mean, d_in, n_grid, S, tau, dev_err);
-    return cudaGetLastError();
+                               float* tau, double* part, int* dev_words, int num_sms,
+                               cudaStream_t stream) {
+    int64_t slices = (2 * (int64_t)num_sms + n_grid - 1) / n_grid;
+    slices = std::min<int64_t>(slices, (d_in + 63) / 64);
+    slices = std::max<int64_t>(1, std::min<int64_t>(slices, kMaxTableSlices));
+    const int64_t slice = (d_in + slices - 1) / slices;
+    slices = (d_in + slice - 1) / slice;
+    const dim3 grid((unsigned)slices, (unsigned)n_grid);
+    table_minmax_kernel<<<grid, 256, 0, stream>>>(x_mean, d_in, n_grid, slice, part,
+                                                  dev_words);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    return launch_pdl(table_write_kernel, grid, dim3(256), 0, stream, x_mean, d_in, n_grid,
+                      slice, (const double*)part, S, tau);
 }
 
 cudaError_t launch_finalize(const double* partial, int n_parts, int n_grid, const float* S,
                             int64_t d_in, const int* dev_err, double* err,
                             int32_t* best_idx, float* s_best, cudaStream_t stream) {
-    finalize_kernel<<<1, 256, 0, stream>>>(partial, n_parts, n_grid, S, d_in, dev_err, err,
-                                           best_idx, s_best);
-    return cudaGetLastError();
+    return launch_pdl(finalize_kernel, dim3(1), dim3(kThreads), 0, stream, partial, n_parts,
+                      n_grid, S, d_in, dev_err, err, best_idx, s_best);
 }
 
 awq_status launch_scale_search(int n_seg, const void* const* W, const int64_t* d_out,
@@ -454,8 +579,8 @@ awq_status launch_scale_search(int n_seg, const void* const* W, const int64_t* d
     EncodeTiledFn encode = encode_tiled_fn();
     if (!encode) return AWQ_ERR_CUDA;
 
-    const int L = group_size / 32;
-    const int R = kConsumerWarps * 32 / L;
+    const int L = group_size / 16;
+    const int R = kConsumerWarps * 2 * 32 / L;
     SearchWs w = carve_search_ws(ws, d_in, n_grid);
 
     SearchParams p;
@@ -468,7 +593,10 @@ awq_status launch_scale_search(int n_seg, const void* const* W, const int64_t* d
     p.S = w.S;
     p.tau = w.tau;
     p.partial = w.partial;
-    p.dev_err = w.dev_err;
+    p.dev_words = w.dev_words;
+    p.err = err;
+    p.best_idx = best_idx;
+    p.s_best = s_best;
     const int64_t G = d_in / group_size;
     int64_t units = 0;
     for (int k = 0; k < n_seg; ++k) {
@@ -490,24 +618,19 @@ awq_status launch_scale_search(int n_seg, const void* const* W, const int64_t* d
     p.n_units = units;
 
     const size_t smem = search_smem_bytes(group_size, n_grid);
-    const int per_sm = (2 * (smem + 1024) <= dev.max_smem_per_sm) ? 2 : 1;
+    int per_sm = 2;
+    while (per_sm > 1 && (size_t)per_sm * (smem + 1024) > dev.max_smem_per_sm) --per_sm;
     int64_t grid = (int64_t)dev.num_sms * per_sm;
     if (grid > units) grid = units;
     if (grid > (int64_t)max_search_ctas()) grid = (int64_t)max_search_ctas();
 
-    if (launch_scale_table(x_mean, d_in, n_grid, w.S, w.tau, w.dev_err, stream) != cudaSuccess)
+    if (launch_scale_table(x_mean, d_in, n_grid, w.S, w.tau, w.partial, w.dev_words,
+                           dev.num_sms, stream) != cudaSuccess)
         return AWQ_ERR_CUDA;
-    cudaError_t e;
-    switch (L) {
-        case 1: e = launch_search_L<1>(p, (int)grid, smem, stream); break;
-        case 2: e = launch_search_L<2>(p, (int)grid, smem, stream); break;
-        case 4: e = launch_search_L<4>(p, (int)grid, smem, stream); break;
-        default: return AWQ_ERR_UNSUPPORTED;
-    }
+    const cudaError_t e = (flags & AWQ_SCALE_FP32)
+                              ? launch_search<true>(L, p, (int)grid, smem, stream)
+                              : launch_search<false>(L, p, (int)grid, smem, stream);
     if (e != cudaSuccess) return AWQ_ERR_CUDA;
-    if (launch_finalize(w.partial, (int)grid, n_grid, w.S, d_in, w.dev_err, err, best_idx,
-                        s_best, stream) != cudaSuccess)
-        return AWQ_ERR_CUDA;
     return AWQ_OK;
 }
 

@@ -2,165 +2,187 @@
 // ("From-Scratch AWQ INT4 Quantization on Qwen3-8B", section "AWQ scaling";
 // "AWQ architecture, in depth", section "The scale search as code").
 //
-// A column reduction over X (fp16 [T, ld]).  It is bound by the HBM read of X
-// (2 bytes per element).  Each thread owns one 16-byte chunk (8 channels) of
-// a row and walks down the rows of its token slice, so a warp reads 512
-// contiguous bytes per row.  The sum is exact: |h| of an fp16 h is an integer
-// number of 2^-24 units below 2^40, accumulated in 64-bit integers, so the
-// order of the additions (and the integer atomics across CTAs) cannot change
-// the result.
+// A column reduction over X (fp16 [T, ld]), bound by the HBM read of X
+// (2 bytes per element).  One launch, no workspace:
+//   * a CTA owns 64 channels (8 chunks of 16 bytes) and one eighth of the
+//     tokens; the 8 CTAs of a thread-block cluster (1 x 8 x 1) cover all
+//     tokens of the same channels;
+//   * each thread walks its chunk down every 32nd row of its slice with eight
+//     16-byte loads in flight and adds |h| in fp64.  Every |fp16| is an
+//     integer multiple of 2^-24 below 2^16, so a sum of up to 4096 of them is
+//     an integer multiple of 2^-24 below 2^28: exact in fp64.  Every 4096
+//     rows the fp64 sums are moved, exactly, into 64-bit integer counts of
+//     2^-24;
+//   * the integer sums are added across the warp's row lanes with shuffles,
+//     then meet in shared memory, then in CTA 0 of the cluster
+//     through distributed shared memory atomics; integer addition makes the
+//     result independent of order.  CTA 0 writes x[j] = (sum * 2^-24) / T
+//     (fp64 division, rounded to fp32).
+// A NaN makes its column's fp64 sum NaN and an infinity makes it +inf; they
+// are carried as flag bits (NaN wins).
+#include <cooperative_groups.h>
+
 #include <algorithm>
 
 #include "common.cuh"
 #include "internal.h"
 
+namespace cg = cooperative_groups;
+
 namespace awq {
 namespace {
 
-constexpr int kStatsChunks = 32;   // 16-byte chunks per CTA row (256 channels)
-constexpr int kStatsRows = 8;      // rows walked in parallel per CTA
+constexpr int kCluster = 8;        // CTAs per cluster, splitting the tokens
+constexpr int kChunks = 8;         // 16-byte chunks per CTA (64 channels)
+constexpr int kRowLanes = 32;      // rows walked in parallel per CTA
+constexpr int kInFlight = 8;       // 16-byte loads in flight per thread
+constexpr int kFlushRows = 4096;   // rows per thread between exact flushes
 
-// |h| in units of 2^-24.  A non-finite h adds nothing and sets bit 2*col
-// (infinity) or 2*col+1 (NaN) of *flags, col being the channel's place in its
-// 16-byte chunk.
-__device__ __forceinline__ uint64_t abs_half_units(uint32_t h, int col, uint32_t* flags) {
-    const uint32_t e = (h >> 10) & 0x1fu;
-    const uint32_t mant = h & 0x3ffu;
-    if (e == 0x1fu) {
-        *flags |= (mant ? 2u : 1u) << (2 * col);
-        return 0;
+// |h| as an fp64 value without the (slow-pipe) fp32 -> fp64 conversion: the
+// fp16 -> fp32 conversion is exact, and an fp32 value f with at most 11
+// significant bits is the fp64 value whose high word is (bits(f) >> 3) +
+// ((1023 - 127) << 20) and whose low word is 0.  Zero maps to 2^-127 instead
+// of 0; a sum of integers multiples of 2^-24 is unaffected by such terms once
+// it is scaled by 2^24 and rounded to an integer, which is what flush()
+// does.  Non-finite inputs are caught separately by the lane's running
+// maximum of |h| bit patterns (hmax).
+__device__ __forceinline__ void add_halves(const uint4& v, double* acc, uint32_t* hmax) {
+    const uint32_t wv[4] = {v.x & 0x7fff7fffu, v.y & 0x7fff7fffu, v.z & 0x7fff7fffu,
+                            v.w & 0x7fff7fffu};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        hmax[i] = __vmaxu2(hmax[i], wv[i]);
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&wv[i]));
+        const uint32_t hx = (__float_as_uint(f.x) >> 3) + 0x38000000u;
+        const uint32_t hy = (__float_as_uint(f.y) >> 3) + 0x38000000u;
+        acc[2 * i] += __hiloint2double((int)hx, 0);
+        acc[2 * i + 1] += __hiloint2double((int)hy, 0);
     }
-    return e ? (static_cast<uint64_t>(mant | 0x400u) << (e - 1)) : mant;
 }
 
-__global__ void stats_zero_kernel(unsigned long long* sums, uint32_t* flags, int64_t d_in) {
-    for (int64_t j = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; j < d_in;
-         j += (int64_t)gridDim.x * blockDim.x) {
-        sums[j] = 0;
-        flags[j] = 0;
-    }
-}
-
-__global__ void __launch_bounds__(kStatsChunks * kStatsRows)
-stats_accumulate_kernel(const uint4* __restrict__ X, int64_t T, int64_t d_in,
-                        int64_t ld_chunks, int64_t rows_per_split,
-                        unsigned long long* __restrict__ sums,
-                        uint32_t* __restrict__ flags) {
-    __shared__ unsigned long long red[kStatsRows][kStatsChunks][8];
-    __shared__ uint32_t fred[kStatsRows][kStatsChunks];
-
-    const int cx = threadIdx.x % kStatsChunks;
-    const int ry = threadIdx.x / kStatsChunks;
-    const int64_t chunk = (int64_t)blockIdx.x * kStatsChunks + cx;
-    const bool active = chunk * 8 < d_in;
-    const int64_t r0 = (int64_t)blockIdx.y * rows_per_split;
-    const int64_t r1 = min(T, r0 + rows_per_split);
-
-    unsigned long long acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    uint32_t fl = 0;
-    if (active) {
-        const uint4* p = X + chunk;
-        int64_t r = r0 + ry;
-        // two rows in flight per iteration
-        for (; r + kStatsRows < r1; r += 2 * kStatsRows) {
-            const uint4 a = __ldg(p + r * ld_chunks);
-            const uint4 b = __ldg(p + (r + kStatsRows) * ld_chunks);
-            const uint32_t wa[4] = {a.x, a.y, a.z, a.w};
-            const uint32_t wb[4] = {b.x, b.y, b.z, b.w};
+// Moves the exact fp64 partial sums into integer counts of 2^-24 (or flag
+// bits for a column that held a non-finite value: bit 0 infinity, bit 1
+// NaN, from the largest |h| bit patterns seen), adds them over the warp's
+// row lanes (lanes with the same chunk) and into the CTA's shared
+// accumulators, and clears them.  Called by every lane of a warp together.
+__device__ __forceinline__ void flush(double* acc, const uint32_t* hmax, int cx,
+                                      unsigned long long* red, uint32_t* fred) {
+    const int lane = threadIdx.x & 31;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                acc[2 * i] += abs_half_units(wa[i] & 0xffffu, 2 * i, &fl) +
-                              abs_half_units(wb[i] & 0xffffu, 2 * i, &fl);
-                acc[2 * i + 1] += abs_half_units(wa[i] >> 16, 2 * i + 1, &fl) +
-                                  abs_half_units(wb[i] >> 16, 2 * i + 1, &fl);
-            }
-        }
-        if (r < r1) {
-            const uint4 a = __ldg(p + r * ld_chunks);
-            const uint32_t wa[4] = {a.x, a.y, a.z, a.w};
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                acc[2 * i] += abs_half_units(wa[i] & 0xffffu, 2 * i, &fl);
-                acc[2 * i + 1] += abs_half_units(wa[i] >> 16, 2 * i + 1, &fl);
-            }
-        }
-    }
-#pragma unroll
-    for (int i = 0; i < 8; ++i) red[ry][cx][i] = acc[i];
-    fred[ry][cx] = fl;
-    __syncthreads();
-    if (ry == 0 && active) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            unsigned long long s = 0;
-            for (int k = 0; k < kStatsRows; ++k) s += red[k][cx][i];
-            if (s) atomicAdd(sums + chunk * 8 + i, s);
-        }
+    for (int i = 0; i < 8; ++i) {
+        const uint32_t hm = (hmax[i >> 1] >> (16 * (i & 1))) & 0xffffu;
+        unsigned long long u = __double2ull_rn(acc[i] * 0x1p24);
         uint32_t f = 0;
-        for (int k = 0; k < kStatsRows; ++k) f |= fred[k][cx];
-        if (f) {
-            for (int i = 0; i < 8; ++i) {
-                const uint32_t fi = (f >> (2 * i)) & 3u;
-                if (fi) atomicOr(flags + chunk * 8 + i, fi);
-            }
+        if (hm > 0x7c00u) {
+            f = 2u;
+            u = 0;
+        } else if (hm == 0x7c00u) {
+            f = 1u;
+            u = 0;
         }
+#pragma unroll
+        for (int o = kChunks; o < 32; o <<= 1) {
+            u += __shfl_xor_sync(0xffffffffu, u, o);
+            f |= __shfl_xor_sync(0xffffffffu, f, o);
+        }
+        if (lane < kChunks) {
+            if (u) atomicAdd(&red[cx * 8 + i], u);
+            if (f) atomicOr(&fred[cx * 8 + i], f);
+        }
+        acc[i] = 0.0;
     }
 }
 
-// x[j] = (exact sum * 2^-24) / T in fp64, rounded to fp32; NaN if the column
-// held a NaN, +inf if it held an infinity.
-__global__ void stats_finalize_kernel(const unsigned long long* __restrict__ sums,
-                                      const uint32_t* __restrict__ flags, int64_t T,
-                                      int64_t d_in, float* __restrict__ x_mean) {
-    for (int64_t j = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; j < d_in;
-         j += (int64_t)gridDim.x * blockDim.x) {
-        const uint32_t f = flags[j];
-        float v;
-        if (f & 2u) {
-            v = __int_as_float(0x7fc00000);
-        } else if (f & 1u) {
-            v = __int_as_float(0x7f800000);
-        } else {
-            const double s = __ll2double_rn(static_cast<long long>(sums[j]));
-            v = __double2float_rn(__ddiv_rn(s * 0x1p-24, (double)T));
+__global__ void __cluster_dims__(1, kCluster, 1) __launch_bounds__(kChunks * kRowLanes, 4)
+stats_kernel(const uint4* __restrict__ X, int64_t T, int64_t d_in, int64_t ld_chunks,
+             float* __restrict__ x_mean) {
+    __shared__ unsigned long long red[kChunks * 8];
+    __shared__ uint32_t fred[kChunks * 8];
+    cg::cluster_group cluster = cg::this_cluster();
+    const int rank = (int)cluster.block_rank();
+
+    const int tid = threadIdx.x;
+    const int cx = tid % kChunks;
+    const int ry = tid / kChunks;
+    if (tid < kChunks * 8) {
+        red[tid] = 0;
+        fred[tid] = 0;
+    }
+    cluster.sync();   // every CTA's accumulators are cleared before remote adds
+
+    const int64_t chunk = (int64_t)blockIdx.x * kChunks + cx;
+    const bool active = chunk * 8 < d_in;
+    const int64_t per = (T + kCluster - 1) / kCluster;
+    const int64_t r0 = rank * per;
+    const int64_t r1 = min(T, r0 + per);
+
+    double acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    uint32_t hmax[4] = {0, 0, 0, 0};   // per word: max |h| bits of its two channels
+    const uint4* p = X + (active ? chunk : 0);
+    // The 32 lanes of a warp hold row offsets 4w .. 4w+3 (and 8 chunks each):
+    // the main loop's trip count depends only on the warp's first row, so
+    // every lane of a warp runs it (and the shuffles in flush) together.
+    const int64_t warp_row = r0 + (ry & ~3);
+    const int sub = ry & 3;
+    int64_t base = warp_row;
+    int since_flush = 0;
+    for (; base + 3 + (kInFlight - 1) * kRowLanes < r1; base += kInFlight * kRowLanes) {
+        const int64_t r = base + sub;
+        uint4 v[kInFlight];
+#pragma unroll
+        for (int k = 0; k < kInFlight; ++k)
+            v[k] = active ? __ldg(p + (r + k * kRowLanes) * ld_chunks) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int k = 0; k < kInFlight; ++k) add_halves(v[k], acc, hmax);
+        since_flush += kInFlight;
+        if (since_flush >= kFlushRows) {
+            flush(acc, hmax, cx, red, fred);
+            since_flush = 0;
         }
-        x_mean[j] = v;
+    }
+    for (int64_t r = base + sub; r < r1; r += kRowLanes)
+        if (active) add_halves(__ldg(p + r * ld_chunks), acc, hmax);
+    flush(acc, hmax, cx, red, fred);
+    __syncthreads();
+    if (rank != 0 && tid < kChunks * 8) {
+        unsigned long long* red0 = cluster.map_shared_rank(red, 0);
+        uint32_t* fred0 = cluster.map_shared_rank(fred, 0);
+        if (red[tid]) atomicAdd(&red0[tid], red[tid]);
+        if (fred[tid]) atomicOr(&fred0[tid], fred[tid]);
+    }
+    cluster.sync();
+    if (rank == 0 && tid < kChunks * 8) {
+        const int64_t j = (int64_t)blockIdx.x * kChunks * 8 + tid;
+        if (j < d_in) {
+            const uint32_t f = fred[tid];
+            float v;
+            if (f & 2u) {
+                v = __int_as_float(0x7fc00000);
+            } else if (f & 1u) {
+                v = __int_as_float(0x7f800000);
+            } else {
+                const double s = __ull2double_rn(red[tid]);
+                v = __double2float_rn(__ddiv_rn(s * 0x1p-24, (double)T));
+            }
+            x_mean[j] = v;
+        }
     }
 }
 
 }  // namespace
 
 size_t act_stats_workspace(int64_t d_in) {
-    return align_up((size_t)d_in * sizeof(unsigned long long), kWsAlign) +
-           align_up((size_t)d_in * sizeof(uint32_t), kWsAlign);
+    (void)d_in;
+    return 0;
 }
 
 cudaError_t launch_act_stats(const void* X, int64_t T, int64_t d_in, int64_t ld,
                              float* x_mean, void* ws, cudaStream_t stream) {
-    DeviceInfo dev;
-    cudaError_t e = query_device(&dev);
-    if (e != cudaSuccess) return e;
-    auto* sums = static_cast<unsigned long long*>(ws);
-    auto* flags = reinterpret_cast<uint32_t*>(
-        static_cast<char*>(ws) + align_up((size_t)d_in * sizeof(unsigned long long), kWsAlign));
-
-    const int zero_blocks = (int)std::min<int64_t>((d_in + 255) / 256, 1024);
-    stats_zero_kernel<<<zero_blocks, 256, 0, stream>>>(sums, flags, d_in);
-
-    const int64_t col_blocks = (d_in / 8 + kStatsChunks - 1) / kStatsChunks;
-    const int64_t want = 4ll * dev.num_sms;
-    int64_t splits = (want + col_blocks - 1) / col_blocks;
-    const int64_t max_splits = (T + 2 * kStatsRows - 1) / (2 * kStatsRows);
-    if (splits > max_splits) splits = max_splits;
-    if (splits < 1) splits = 1;
-    if (splits > 65535) splits = 65535;
-    const int64_t rows_per_split = (T + splits - 1) / splits;
-    splits = (T + rows_per_split - 1) / rows_per_split;
-    dim3 grid((unsigned)col_blocks, (unsigned)splits);
-    stats_accumulate_kernel<<<grid, kStatsChunks * kStatsRows, 0, stream>>>(
-        static_cast<const uint4*>(X), T, d_in, ld / 8, rows_per_split, sums, flags);
-
-    stats_finalize_kernel<<<zero_blocks, 256, 0, stream>>>(sums, flags, T, d_in, x_mean);
+    (void)ws;
+    const int64_t col_blocks = (d_in / 8 + kChunks - 1) / kChunks;
+    dim3 grid((unsigned)col_blocks, kCluster);
+    stats_kernel<<<grid, kChunks * kRowLanes, 0, stream>>>(static_cast<const uint4*>(X), T,
+                                                            d_in, ld / 8, x_mean);
     return cudaGetLastError();
 }
 

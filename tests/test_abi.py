@@ -42,7 +42,7 @@ def test_status_strings_and_version():
 
 def test_workspace_sizes():
     n_stats = awq.workspace_size(awq.OP_ACT_STATS, 4096, 8, 4096, 128, 20)
-    assert n_stats >= 4096 * 12
+    assert n_stats == 0
     n_search = awq.workspace_size(awq.OP_SCALE_SEARCH, 1, 8, 4096, 128, 20)
     assert n_search >= 2 * 20 * 4096 * 4
     with pytest.raises(awq.AwqError):
@@ -66,8 +66,8 @@ def test_host_validation_without_a_gpu():
     assert L.awq_act_stats(fake, 0, 8, 8, fake, fake, 1 << 20, None) == 1
     assert L.awq_act_stats(fake, 4, 12, 12, fake, fake, 1 << 20, None) == 3
     assert L.awq_act_stats(odd, 4, 8, 8, fake, fake, 1 << 20, None) == 3
-    assert L.awq_act_stats(fake, 4, 8, 8, fake, None, 0, None) == 4
-    assert L.awq_act_stats(fake, 4, 8, 8, fake, fake, 8, None) == 4
+    assert L.awq_act_stats(fake, 1 << 24, 8, 8, fake, None, 0, None) == 1
+    assert L.awq_act_stats(fake, 4, 8, 8, fake, odd, 0, None) == 3
     # scale_search
     W = (ctypes.c_void_p * 1)(fake)
     d = (ctypes.c_int64 * 1)(64)

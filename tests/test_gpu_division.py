@@ -1,0 +1,35 @@
+"""The exact-division helpers of the CUDA kernels equal IEEE fp32 division.
+
+The kernels decide q_scale = fp16(RN(m / 7)) and the stored codes
+rint(RN(ws / q_scale)) with cheaper FMA sequences (common.cuh: div7_rn,
+div_rn_rcp).  This test compiles a small check library from
+tests/cuda/division_check.cu and compares them bit for bit with __fdiv_rn:
+div7_rn over every non-negative finite fp32 value, div_rn_rcp over every
+positive finite fp16 divisor with numerators at and around every half-integer
+multiple of it (the rounding decisions) plus a sweep.
+"""
+import ctypes
+import os
+import subprocess
+import tempfile
+
+import pytest
+
+pytestmark = pytest.mark.gpu
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def test_division_helpers_equal_ieee_division():
+    src = os.path.join(ROOT, "tests", "cuda", "division_check.cu")
+    inc = os.path.join(ROOT, "post_int4_weight_b200", "csrc")
+    with tempfile.TemporaryDirectory() as d:
+        so = os.path.join(d, "division_check.so")
+        subprocess.run(["/usr/local/cuda/bin/nvcc", "-gencode", "arch=compute_100a,code=sm_100a",
+                        "-O3", "-std=c++17", "-Xcompiler", "-fPIC", "-shared", "-I" + inc,
+                        src, "-o", so], check=True)
+        lib = ctypes.CDLL(so)
+        out = (ctypes.c_ulonglong * 4)()
+        assert lib.run_checks(out) == 0
+    assert out[0] == 0, f"div7_rn differs from IEEE for {out[0]} values, first bits {out[1]:#x}"
+    assert out[2] == 0, f"div_rn_rcp differs for {out[2]} pairs, first fp16 divisor {out[3]:#x}"

@@ -80,6 +80,16 @@ def test_act_stats_bit_exact(T, d_in):
     assert np.array_equal(_np(x), oracle.act_stats(X.numpy()))
 
 
+def test_act_stats_long_token_slices():
+    """More than 4096 rows per thread: the exact fp64 partial sums are moved
+    into the integer accumulators mid-way (rows of 16 lanes x 8 CTAs)."""
+    X = wl.activations(600_011, 16, seed=77)
+    X[:, 3] = 65504.0                      # the largest sums the format allows
+    x = awq.act_stats(X.cuda())
+    torch.cuda.synchronize()
+    assert np.array_equal(_np(x), oracle.act_stats(X.numpy()))
+
+
 def test_act_stats_nonfinite_and_extremes():
     X = wl.activations(40, 64, seed=5)
     X[3, 1] = float("inf")
@@ -216,6 +226,33 @@ def test_pack_edge_groups():
     gen = torch.Generator().manual_seed(22)
     s = torch.exp(torch.randn(256, generator=gen)).float()
     _assert_pack_parity(W.cuda(), s.numpy(), s.cuda(), 128, 8)
+
+
+def test_pack_every_fp16_quotient_below_many_maxima():
+    """Row k's group holds its maximum m_k at column 0 and then every fp16
+    value in [-m_k, m_k] in turn (s = 1, so ws = w exactly and q_scale =
+    fp16(m_k / 7)): every rounding decision of those scales, ties included,
+    is compared bit for bit."""
+    rng = np.random.default_rng(5)
+    all_pos = np.arange(1, 0x7C00, dtype=np.uint16).view(np.float16).astype(np.float32)
+    maxima = np.concatenate([
+        np.array([65504.0, 1.0, 0.875, 7 * 2.0 ** -14, 7 * 2.0 ** -14 * 0.999, 3e-7, 1e-3],
+                 np.float32),
+        np.float16(np.exp(rng.uniform(np.log(1e-6), np.log(6e4), 41))).astype(np.float32)])
+    rows = []
+    for m in np.float16(maxima).astype(np.float32):
+        vals = all_pos[all_pos <= m]
+        vals = np.concatenate([vals, -vals])
+        for k in range(0, len(vals), 127):
+            chunk = vals[k:k + 127]
+            row = np.zeros(128, np.float32)
+            row[0] = m
+            row[1:1 + len(chunk)] = chunk
+            rows.append(row)
+    pad = (-len(rows)) % 8
+    rows += [np.zeros(128, np.float32)] * pad
+    W = torch.from_numpy(np.stack(rows).astype(np.float16))
+    _assert_pack_parity(W.cuda(), None, None, 128, 8)
 
 
 # ------------------------------------------------------- end to end --
