@@ -68,6 +68,11 @@ const char *awq_status_string(int status);
 /* Version of this ABI (major * 100 + minor). */
 int awq_abi_version(void);
 
+/* Text of the last failed CUDA runtime call seen by the library on the
+ * calling host thread (which call, the error name and its description), for
+ * an AWQ_ERR_CUDA.  Static thread-local storage; never NULL. */
+const char *awq_last_error(void);
+
 /*
  * Bytes of workspace that `op` needs for the given sizes.  For
  * AWQ_OP_ACT_STATS only d_in matters; for AWQ_OP_SCALE_SEARCH d_in, the

@@ -313,36 +313,49 @@ void orc_output_error(const uint16_t *X, int64_t T, const uint16_t *W,
     float *S = (float *)malloc((size_t)n_grid * (size_t)d_in * sizeof(float));
     double *dW = (double *)malloc((size_t)d_out * (size_t)d_in * sizeof(double));
     double *Xd = (double *)malloc((size_t)T * (size_t)d_in * sizeof(double));
-    float *w = (float *)malloc((size_t)g * sizeof(float));
-    int8_t *q = (int8_t *)malloc((size_t)g);
+    double *tok = (double *)malloc((size_t)T * sizeof(double));
+    int *bad_row = (int *)malloc((size_t)d_out * sizeof(int));
     orc_scale_table(x, d_in, n_grid, S);
     for (int64_t t = 0; t < T * d_in; ++t) Xd[t] = (double)h2f(X[t]);
 
     for (int i = 0; i < n_grid; ++i) {
         const float *s = S + (int64_t)i * d_in;
-        int bad = 0;
-        for (int64_t r = 0; r < d_out; ++r)
+        /* W - W_hat_i, exactly (fp64) from the fp32 decisions */
+#pragma omp parallel for schedule(static)
+        for (int64_t r = 0; r < d_out; ++r) {
+            float w[g];
+            int8_t q[g];
+            bad_row[r] = 0;
             for (int64_t k = 0; k < d_in / g; ++k) {
                 for (int64_t j = 0; j < g; ++j) w[j] = h2f(W[r * d_in + k * g + j]);
                 float qs;
-                if (orc_fake_quant_group(w, s + k * g, g, flags, q, &qs)) bad = 1;
+                if (orc_fake_quant_group(w, s + k * g, g, flags, q, &qs)) bad_row[r] = 1;
                 for (int64_t j = 0; j < g; ++j)
                     dW[r * d_in + k * g + j] =
                         (double)w[j] - (double)q[j] * (double)qs / (double)s[k * g + j];
             }
-        double total = 0.0;
-        for (int64_t t = 0; t < T; ++t)
+        }
+        /* ||X dW^T||^2: one partial per token, summed in token order */
+#pragma omp parallel for schedule(static)
+        for (int64_t t = 0; t < T; ++t) {
+            double acc = 0.0;
             for (int64_t r = 0; r < d_out; ++r) {
                 double y = 0.0;
                 for (int64_t j = 0; j < d_in; ++j)
                     y += Xd[t * d_in + j] * dW[r * d_in + j];
-                total += y * y;
+                acc += y * y;
             }
+            tok[t] = acc;
+        }
+        double total = 0.0;
+        int bad = 0;
+        for (int64_t t = 0; t < T; ++t) total += tok[t];
+        for (int64_t r = 0; r < d_out; ++r) bad |= bad_row[r];
         err[i] = bad ? NAN : total;
     }
     free(S);
     free(dW);
     free(Xd);
-    free(w);
-    free(q);
+    free(tok);
+    free(bad_row);
 }

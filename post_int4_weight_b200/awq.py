@@ -33,7 +33,10 @@ class AwqError(RuntimeError):
 
     def __init__(self, status: int, where: str):
         self.status = status
-        super().__init__(f"{where}: {string(status)}")
+        detail = ""
+        if status == 5:   # AWQ_ERR_CUDA
+            detail = " [" + lib().awq_last_error().decode() + "]"
+        super().__init__(f"{where}: {string(status)}{detail}")
 
 
 def lib() -> ctypes.CDLL:
@@ -50,6 +53,7 @@ def lib() -> ctypes.CDLL:
         L.awq_status_string.argtypes = [i32]
         L.awq_status_string.restype = ctypes.c_char_p
         L.awq_abi_version.restype = i32
+        L.awq_last_error.restype = ctypes.c_char_p
         L.awq_workspace_size.argtypes = [i32, i64, i64, i64, i32, i32, ctypes.POINTER(sz)]
         L.awq_workspace_size.restype = i32
         L.awq_act_stats.argtypes = [p, i64, i64, i64, p, p, sz, p]

@@ -1,10 +1,22 @@
 // api.cu -- the extern "C" entry points of include/awq.h: host-side argument
 // validation, workspace sizing, and dispatch to the launchers.
+#include <cstdio>
 #include <cstring>
 
 #include "internal.h"
 
 namespace awq {
+
+namespace {
+thread_local char g_last_error[256] = "no CUDA error recorded";
+}
+
+cudaError_t note_cuda(cudaError_t e, const char* where) {
+    if (e != cudaSuccess)
+        snprintf(g_last_error, sizeof g_last_error, "%s: %s (%s)", where, cudaGetErrorName(e),
+                 cudaGetErrorString(e));
+    return e;
+}
 
 cudaError_t query_device(DeviceInfo* info) {
     cudaError_t e = cudaGetDevice(&info->device);
@@ -57,6 +69,8 @@ const char* awq_status_string(int status) {
 }
 
 int awq_abi_version(void) { return 100; }
+
+const char* awq_last_error(void) { return g_last_error; }
 
 awq_status awq_workspace_size(int op, int64_t T, int64_t d_out_total, int64_t d_in,
                               int group_size, int n_grid, size_t* bytes) {

@@ -20,6 +20,10 @@ inline bool aligned16(const void* p) {
     return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
 }
 
+// Records a failed CUDA runtime call for awq_last_error() (per host thread)
+// and passes the error through.
+cudaError_t note_cuda(cudaError_t e, const char* where);
+
 struct DeviceInfo {
     int device = 0;
     int num_sms = 0;
@@ -55,15 +59,16 @@ awq_status launch_output_error(const void* X, int64_t T, const void* W, int64_t 
                                void* ws, cudaStream_t stream);
 
 // ---- shared pieces of the search and the output-error mode
-// Writes S[i][j] and tau[i][j] = x_mean[j] / S[i][j] (fp32, [n_grid][d_in])
-// with two kernels (pow + per-slice min/max, then normalise); `part` holds
-// 2 * n_grid * kMaxTableSlices doubles.  Clears *dev_words (2 ints: error
-// word, CTA-done counter) if non-NULL.  The second kernel is a programmatic
-// dependent launch of the first.
+// Writes S[i][j] and tau[i][j] = x_mean[j] / S[i][j] (or 1 / S[i][j] when
+// write_inverse) (fp32, [n_grid][d_in]) with two kernels (pow + per-slice
+// min/max, then normalise); `part` holds 2 * n_grid * kMaxTableSlices
+// doubles.  Clears *dev_words (2 ints: error word, CTA-done counter) if
+// non-NULL.  The second kernel is a programmatic dependent launch of the
+// first.
 constexpr int kMaxTableSlices = 64;
 cudaError_t launch_scale_table(const float* x_mean, int64_t d_in, int n_grid, float* S,
                                float* tau, double* part, int* dev_words, int num_sms,
-                               cudaStream_t stream);
+                               cudaStream_t stream, bool write_inverse = false);
 
 // Launch with the programmatic stream-serialisation attribute (the kernel
 // must call pdl_wait() before depending on its predecessor).

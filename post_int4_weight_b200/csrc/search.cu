@@ -452,7 +452,7 @@ table_minmax_kernel(const float* __restrict__ x, int64_t d_in, int n_grid, int64
 __global__ void __launch_bounds__(256)
 table_write_kernel(const float* __restrict__ x, int64_t d_in, int n_grid, int64_t slice,
                    const double* __restrict__ part, float* __restrict__ S,
-                   float* __restrict__ tau) {
+                   float* __restrict__ tau, int write_inverse) {
     pdl_launch_dependents();
     pdl_wait();
     const int a = blockIdx.y;
@@ -468,7 +468,7 @@ table_write_kernel(const float* __restrict__ x, int64_t d_in, int n_grid, int64_
     for (int64_t j = j0 + threadIdx.x; j < j1; j += blockDim.x) {
         const float s = __double2float_rn(__ddiv_rn(table_pow(x, j, alpha), norm));
         S[(int64_t)a * d_in + j] = s;
-        tau[(int64_t)a * d_in + j] = __fdiv_rn(x[j], s);
+        tau[(int64_t)a * d_in + j] = write_inverse ? __frcp_rn(s) : __fdiv_rn(x[j], s);
     }
 }
 
@@ -548,7 +548,7 @@ size_t scale_search_workspace(int64_t d_in, int group_size, int n_grid) {
 
 cudaError_t launch_scale_table(const float* x_mean, int64_t d_in, int n_grid, float* S,
                                float* tau, double* part, int* dev_words, int num_sms,
-                               cudaStream_t stream) {
+                               cudaStream_t stream, bool write_inverse) {
     int64_t slices = (2 * (int64_t)num_sms + n_grid - 1) / n_grid;
     slices = std::min<int64_t>(slices, (d_in + 63) / 64);
     slices = std::max<int64_t>(1, std::min<int64_t>(slices, kMaxTableSlices));
@@ -560,7 +560,7 @@ cudaError_t launch_scale_table(const float* x_mean, int64_t d_in, int n_grid, fl
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     return launch_pdl(table_write_kernel, grid, dim3(256), 0, stream, x_mean, d_in, n_grid,
-                      slice, (const double*)part, S, tau);
+                      slice, (const double*)part, S, tau, (int)write_inverse);
 }
 
 cudaError_t launch_finalize(const double* partial, int n_parts, int n_grid, const float* S,
