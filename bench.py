@@ -3,18 +3,33 @@
 scale search + quantise-and-pack) on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload q_proj_4096x4096]
+                    [--workload NAME] [--group-size G]
 
-One step = one pass of the whole hot path over one linear: awq_act_stats on
-X [4096 tokens, 4096], awq_scale_search over the 20-point alpha grid,
-awq_quantize_pack of W [4096, 4096] at the chosen scale (Qwen3-8B
-q_proj-shaped layer, group 128).  Inputs are seeded synthetic (see
-post_int4_weight_b200/workloads.py) and resident in HBM when the timed region
-starts; the inputs (67 MB) fit in the 126 MB L2, so a 256 MB buffer is written
-between timed steps (outside the per-step CUDA events) to flush it.
+One step = one pass of the whole hot path over the workload: for every
+search group (linears sharing one input), awq_act_stats on its X,
+awq_scale_search over the 20-point alpha grid (or awq_output_error for the
+output-space workload), and awq_quantize_pack of every member at the chosen
+scale.  Workloads (post_int4_weight_b200/workloads.py):
 
-With N > 1 (torchrun) every rank quantises its own independent linear (weak
-scaling, no data-path collective); the time is the max over ranks.
+  q_proj_4096x4096        (default) one 4096x4096 linear, 4096 tokens, g128
+  qwen3_8b_block          one decoder block, 7 linears in 4 groups, 16384
+                          tokens, g128 (or --group-size 64)
+  down_proj_output_error  4096x12288 down_proj scored in output space,
+                          8192 tokens, on the tensor cores
+  qwen3_8b_stack36        36 such blocks (6.95 B weights), 2048 tokens per
+                          layer, streamed layer by layer
+
+Inputs are seeded synthetic and resident in HBM when the timed region
+starts.  Workloads whose inputs fit in the 126 MB L2 get a 256 MB buffer
+written between timed steps (outside the per-step CUDA events); larger ones
+are not flushed.  The end-to-end number ("e2e") streams the same work from
+pinned host memory: copies in, kernels, results out, overlapped layer by
+layer on three streams.
+
+Scaling: one-layer workloads give every rank its own independent layer (weak
+scaling); the 36-layer stack is split over the ranks by layer (strong
+scaling).  No data-path collective either way; the time is the max over
+ranks.
 
 Prints one JSON line (rank 0).  --impl reference times the CPU oracle on the
 host cores instead (rank 0 only).
@@ -36,20 +51,29 @@ METRIC = "AWQ search+pack Gparam/s per layer"
 UNIT = "Gparam/s"
 FMA_OPS_PER_PAIR = 6          # FMA-pipe lane ops per (weight, alpha) pair
 FP32_LANES_PER_SM = 128
+DEFAULT_STEPS = {"single_linear_256x512": 1000, "q_proj_4096x4096": 1000,
+                 "qwen3_8b_block": 100, "down_proj_output_error": 10,
+                 "qwen3_8b_stack36": 20}
 
 
 def _args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--steps", type=int, default=None,
+                    help="timed steps (default: about a second or more of work per workload)")
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="q_proj_4096x4096")
+    ap.add_argument("--group-size", type=int, default=0,
+                    help="group size (default: the workload's first)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-graph", action="store_true",
                     help="launch each step eagerly instead of replaying a CUDA graph")
-    return ap.parse_args()
+    a = ap.parse_args()
+    if a.steps is None:
+        a.steps = DEFAULT_STEPS.get(a.workload, 20)
+    return a
 
 
 def _peaks():
@@ -126,10 +150,31 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- our arm --
 
+def _group_size(a, work):
+    g = a.group_size or work.group_sizes[0]
+    if g not in work.group_sizes:
+        raise SystemExit(f"--group-size {g}: workload {work.name} is defined for "
+                         f"{list(work.group_sizes)}")
+    return g
+
+
+def _layer_ids(work, world, rank):
+    """(layers this rank runs, input seed override per layer, scaling)."""
+    from post_int4_weight_b200 import pipeline
+    if work.layers > 1:
+        return pipeline.shard_layers(work.layers, world, rank), [], "strong"
+    return [0], [work.seed + 1000 * rank], "weak"
+
+
+def _inputs(work, layer, seed, device):
+    from post_int4_weight_b200 import workloads as wl
+    return [(Ws, X) for _, Ws, X in wl.group_inputs(work, layer, device, seed)]
+
+
 def run_ours(a):
     import torch
     import torch.distributed as dist
-    from post_int4_weight_b200 import awq
+    from post_int4_weight_b200 import pipeline
     from post_int4_weight_b200 import workloads as wl
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -142,53 +187,57 @@ def run_ours(a):
     torch.cuda.set_device(dev)
 
     work = wl.WORKLOADS[a.workload]
-    assert len(work.groups) == 1 and work.layers == 1, "bench runs one-group workloads"
-    grp = work.groups[0]
-    g = work.group_sizes[0]
+    g = _group_size(a, work)
     n_grid = work.n_grid
-    # each rank quantises its own independent layer (weak scaling)
-    base = 100 * (work.seed + 1000 * rank)
-    Ws_h = [wl.weight(d, grp.d_in, base + m + 1) for m, (_, d) in enumerate(grp.members)]
-    X_h = wl.activations(work.tokens, grp.d_in, base)
-    params = sum(W.numel() for W in Ws_h)
-
-    Ws = [W.to(dev) for W in Ws_h]
-    X = X_h.to(dev)
-    T, d_in = X.shape
-    d_out_total = sum(W.shape[0] for W in Ws)
-    ws_stats = awq.workspace(awq.OP_ACT_STATS, dev, T, 8, d_in)
-    ws_search = awq.workspace(awq.OP_SCALE_SEARCH, dev, 1, d_out_total, d_in, g, n_grid)
-    x = torch.empty(d_in, dtype=torch.float32, device=dev)
-    err = torch.empty(n_grid, dtype=torch.float64, device=dev)
-    best = torch.empty(1, dtype=torch.int32, device=dev)
-    s_best = torch.empty(d_in, dtype=torch.float32, device=dev)
-    packs = [(torch.empty(d_in, W.shape[0] // 8, dtype=torch.int32, device=dev),
-              torch.empty(d_in // g, W.shape[0], dtype=torch.float16, device=dev),
-              torch.empty(d_in // g, W.shape[0] // 8, dtype=torch.int32, device=dev))
-             for W in Ws]
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    layers, seeds, scaling = _layer_ids(work, world, rank)
+    # one-layer workloads: generated on the CPU (the same tensors the parity
+    # tests and the CPU baseline use); the stack: generated on the device
+    gen_dev = "cpu" if work.layers == 1 else dev
+    layer_inputs = []
+    for i, l in enumerate(layers):
+        seed = seeds[i] if i < len(seeds) else None
+        layer_inputs.append([(Ws, X) for Ws, X in _inputs(work, l, seed, gen_dev)])
+    jobs = []
+    for li in layer_inputs:
+        for Ws, X in li:
+            jobs.append(pipeline.GroupJob([W.to(dev) for W in Ws], X.to(dev), g, n_grid,
+                                          work.output_mode))
+    if work.layers == 1:
+        host_layer = [([W.pin_memory() for W in Ws], X.pin_memory()) for Ws, X in layer_inputs[0]]
+    else:
+        host_layer = None
+    wss = pipeline.Workspaces(jobs, dev)
+    params = sum(j.params for j in jobs)
+    in_bytes = sum(j.X.numel() * 2 + sum(W.numel() * 2 for W in j.Ws) for j in jobs)
+    flush_l2 = in_bytes < (512 << 20)
+    flush = torch.empty(256 << 20 if flush_l2 else 1, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
-    kernels_per_step = 1 + 3 + len(Ws)   # stats (1) + search (3) + pack (1 per linear)
+    launches_per_step = sum(j.launches for j in jobs)
 
     def call_stats():
-        awq.act_stats(X, out=x, ws=ws_stats)
+        for j in jobs:
+            j.stats(wss.stats)
 
     def call_search():
-        awq.scale_search(Ws, x, g, n_grid, out=(err, best, s_best), ws=ws_search)
+        for j in jobs:
+            j.search(wss.search)
 
     def call_pack():
-        for W, pk in zip(Ws, packs):
-            awq.quantize_pack(W, s_best, g, 8, out=pk)
+        for j in jobs:
+            j.pack()
 
     def step():
-        call_stats()
-        call_search()
-        call_pack()
+        for j in jobs:
+            j.run(wss)
+
+    def do_flush():
+        if flush_l2:
+            flush.zero_()
 
     # eager warm-up (first calls do the one-time per-device set-up), then the
     # step and each call are captured into CUDA graphs and replayed
     for _ in range(max(a.warmup, 3)):
-        flush.zero_()
+        do_flush()
         step()
     torch.cuda.synchronize(dev)
     graphs = None
@@ -201,7 +250,7 @@ def run_ours(a):
                 fn()
             graphs[name] = gr
         for _ in range(3):
-            flush.zero_()
+            do_flush()
             graphs["step"].replay()
         torch.cuda.synchronize(dev)
     run = {k: (graphs[k].replay if graphs else f) for k, f in
@@ -214,7 +263,7 @@ def run_ours(a):
     torch.cuda.synchronize(dev)
     with ClockSampler(dev) as clk:
         for k in range(a.steps):
-            flush.zero_()
+            do_flush()
             evs[k][0].record(stream)
             run["step"]()
             evs[k][1].record(stream)
@@ -222,17 +271,13 @@ def run_ours(a):
     if world > 1:
         dist.barrier()
     t_step = [e0.elapsed_time(e1) for e0, e1 in evs]
-    ms = sum(t_step) / len(t_step)
-    if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = pipeline.max_over_ranks(sum(t_step) / len(t_step), dev)
 
-    # per-call breakdown (separately timed steps, L2 flushed before each)
-    n_br = max(10, min(200, a.steps))
+    # per-call breakdown (separately timed passes, L2 flushed before each)
+    n_br = max(3, min(200, a.steps))
     br = {"stats": [], "search": [], "pack": []}
     for _ in range(n_br):
-        flush.zero_()
+        do_flush()
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
         ev[0].record(stream)
         run["stats"]()
@@ -248,52 +293,45 @@ def run_ours(a):
     ms_stats = sum(br["stats"]) / n_br
     ms_search = sum(br["search"]) / n_br
     ms_pack = sum(br["pack"]) / n_br
+    del graphs
 
-    # --- end to end through the public API with host buffers
-    e2e = None
-    if rank == 0 or world > 1:
-        Xp = X_h.pin_memory()
-        Wp = [W.pin_memory() for W in Ws_h]
-        out_h = [tuple(torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in pk)
-                 for pk in packs]
-        err_h = torch.empty(n_grid, dtype=torch.float64).pin_memory()
-        best_h = torch.empty(1, dtype=torch.int32).pin_memory()
-        s_h = torch.empty(d_in, dtype=torch.float32).pin_memory()
-        h2d = Xp.numel() * 2 + sum(W.numel() * 2 for W in Wp)
-        d2h = sum(t.numel() * t.element_size() for pk in packs for t in pk) + \
-            err.numel() * 8 + 4 + s_best.numel() * 4
-
-        def e2e_step():
-            X.copy_(Xp, non_blocking=True)
-            for W, w in zip(Ws, Wp):
-                W.copy_(w, non_blocking=True)
-            step()
-            for pk, oh in zip(packs, out_h):
-                for t, th in zip(pk, oh):
-                    th.copy_(t, non_blocking=True)
-            err_h.copy_(err, non_blocking=True)
-            best_h.copy_(best, non_blocking=True)
-            s_h.copy_(s_best, non_blocking=True)
-
-        for _ in range(3):
-            e2e_step()
-        torch.cuda.synchronize(dev)
+    # --- end to end: the same work streamed from pinned host memory
+    template = layer_inputs[0]
+    streamer = pipeline.LayerStreamer(template, dev, g, n_grid, work.output_mode)
+    if work.layers == 1:
         n_e2e = max(5, min(50, a.steps // 20))
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(n_e2e):
-            e2e_step()
-        e1.record(stream)
-        torch.cuda.synchronize(dev)
-        ms_e2e = e0.elapsed_time(e1) / n_e2e
-        if world > 1:
-            t = torch.tensor([ms_e2e], dtype=torch.float64, device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms_e2e = float(t.item())
-        e2e = {"value": world * params / (ms_e2e * 1e-3) / 1e9, "unit": UNIT,
-               "ms_per_step": ms_e2e, "h2d_bytes_per_step": int(h2d),
-               "d2h_bytes_per_step": int(d2h), "steps": n_e2e}
+        host_layers = [host_layer] * n_e2e
+        out_one = streamer.host_outputs()
+        host_out = [out_one] * n_e2e
+        e2e_units = n_e2e
+    else:
+        # this rank's layers, copied once to pinned host memory (not timed)
+        def pinned(t):
+            return torch.empty(t.shape, dtype=t.dtype, pin_memory=True).copy_(t)
+        host_layers = [[([pinned(W) for W in Ws], pinned(X)) for Ws, X in li]
+                       for li in layer_inputs]
+        host_out = [streamer.host_outputs() for _ in host_layers]
+        e2e_units = 1
+    del layer_inputs
+    for _ in range(2):   # warm-up passes over at most two layers
+        streamer.run(host_layers[:2], host_out[:2])
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    streamer.run(host_layers, host_out, after=e0)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms_e2e = pipeline.max_over_ranks(e0.elapsed_time(e1) / e2e_units, dev)
+    h2d_l, d2h_l = streamer.bytes_per_layer()
+    per_step_layers = len(host_layers) // e2e_units
+    e2e = {"value": _total_params(work, world, params) / (ms_e2e * 1e-3) / 1e9, "unit": UNIT,
+           "ms_per_step": ms_e2e, "h2d_bytes_per_step": int(h2d_l * per_step_layers),
+           "d2h_bytes_per_step": int(d2h_l * per_step_layers), "steps": e2e_units,
+           "pipeline": "pinned host -> 2-slot device ring; H2D, kernels and D2H on three "
+                       "streams, overlapped across layers"}
 
     if rank != 0:
         if world > 1:
@@ -304,75 +342,150 @@ def run_ours(a):
     clocks = clk.summary()
     n_sms = torch.cuda.get_device_properties(dev).multi_processor_count
     clk_mhz = clocks["sm_mhz"] or peaks.get("sm_max_mhz", 1965.0)
-    peak_ops = n_sms * FP32_LANES_PER_SM * clk_mhz * 1e6          # lane-ops / s
-    ops = params * n_grid * FMA_OPS_PER_PAIR
-    achieved = ops / (ms_search * 1e-3)
-    bytes_stats = X.numel() * 2
-    bytes_pack = params * 2 + sum(t.numel() * t.element_size() for pk in packs for t in pk)
     hbm = peaks["hbm_gbs"]
-    roof = {"bound": "alu", "kernel": "awq_scale_search (scale table + fused search + finalize)",
-            "achieved": achieved / 1e12, "peak": peak_ops / 1e12, "unit": "Tlane-op/s",
-            "frac": achieved / peak_ops, "traffic": None,
-            "ops_per_weight_alpha": FMA_OPS_PER_PAIR,
-            "peak_basis": f"{n_sms} SMs x {FP32_LANES_PER_SM} FP32 lanes x {clk_mhz:.0f} MHz "
-                          f"(median SM clock sampled in the timed region)"}
+    bytes_stats = sum(j.X.numel() * 2 for j in jobs)
+    bytes_pack = sum(W.numel() * 2 for j in jobs for W in j.Ws) + \
+        sum(t.numel() * t.element_size() for j in jobs for pk in j.packs for t in pk)
+    kernels = {
+        "act_stats": {"ms": ms_stats, "GB/s": bytes_stats / (ms_stats * 1e-3) / 1e9,
+                      "hbm_frac": bytes_stats / (ms_stats * 1e-3) / 1e9 / hbm},
+        "quantize_pack": {"ms": ms_pack, "GB/s": bytes_pack / (ms_pack * 1e-3) / 1e9,
+                          "hbm_frac": bytes_pack / (ms_pack * 1e-3) / 1e9 / hbm},
+        "hbm_peak_GBs": hbm, "peak_source": peak_src}
+    if work.output_mode:
+        flops = sum(2.0 * j.X.shape[0] * W.numel() * n_grid for j in jobs for W in j.Ws)
+        achieved = flops / (ms_search * 1e-3)
+        peak_t = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]) * 1e12
+        roof = {"bound": "tensor",
+                "kernel": "awq_output_error (scale table + per alpha: dW builder + tcgen05 "
+                          "GEMM with fused square-sum + finalize)",
+                "achieved": achieved / 1e12, "peak": peak_t / 1e12, "unit": "TFLOP/s",
+                "frac": achieved / peak_t, "traffic": None,
+                "flops_per_step": flops, "executed_flops_per_step": 2 * flops,
+                "peak_basis": "measured bf16 dense GEMM, sustained (fp16 has the same "
+                              "nominal tensor rate); algorithmic FLOPs 2*T*d_out*d_in per "
+                              "alpha, the tensor cores execute twice that (hi and lo "
+                              "fp16 parts of W - W_hat)"}
+        kernels["output_error"] = {"ms": ms_search, "TFLOP/s": achieved / 1e12,
+                                   "executed_TFLOP/s": 2 * achieved / 1e12}
+    else:
+        peak_ops = n_sms * FP32_LANES_PER_SM * clk_mhz * 1e6          # lane-ops / s
+        ops = params * n_grid * FMA_OPS_PER_PAIR
+        achieved = ops / (ms_search * 1e-3)
+        roof = {"bound": "alu",
+                "kernel": "awq_scale_search (scale table + fused search + finalize)",
+                "achieved": achieved / 1e12, "peak": peak_ops / 1e12, "unit": "Tlane-op/s",
+                "frac": achieved / peak_ops, "traffic": None,
+                "ops_per_weight_alpha": FMA_OPS_PER_PAIR,
+                "peak_basis": f"{n_sms} SMs x {FP32_LANES_PER_SM} FP32 lanes x "
+                              f"{clk_mhz:.0f} MHz (median SM clock sampled in the timed "
+                              f"region)"}
+        kernels["scale_search"] = {"ms": ms_search, "Tlane-op/s": achieved / 1e12,
+                                   "W_GB/s": params * 2 / (ms_search * 1e-3) / 1e9}
+    if work.layers == 1:
+        par = f"independent layer per rank x{world}"
+    else:
+        par = f"layers split over {world} rank(s), {len(layers)} on rank 0"
     out = {
-        "metric": METRIC, "value": world * params / (ms * 1e-3) / 1e9, "unit": UNIT,
-        "n_gpus": world, "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "f32", "data": "synthetic",
-        "config": {"workload": a.workload, "d_out": d_out_total, "d_in": d_in,
-                   "tokens": T, "group_size": g, "n_grid": n_grid,
-                   "params_per_gpu": params, "l2": "flushed (256 MB write) between timed steps",
-                   "parallelism": f"independent layer per rank x{world}"},
+        "metric": METRIC, "value": _total_params(work, world, params) / (ms * 1e-3) / 1e9,
+        "unit": UNIT, "n_gpus": world, "steps": a.steps, "warmup": a.warmup,
+        "ms_per_step": ms, "higher_is_better": True, "scaling": scaling,
+        "vs_baseline": None, "dtype": "f16" if work.output_mode else "f32",
+        "data": "synthetic",
+        "config": {"workload": a.workload, "layers": work.layers, "tokens": work.tokens,
+                   "group_size": g, "n_grid": n_grid,
+                   "params_per_step": _total_params(work, world, params),
+                   "params_rank0": params,
+                   "l2": ("flushed (256 MB write) between timed steps" if flush_l2 else
+                          f"not flushed: {in_bytes / 1e9:.2f} GB of inputs per step "
+                          f"(> 126 MB L2)"),
+                   "parallelism": par},
         "roofline": roof,
-        "kernels": {
-            "act_stats": {"ms": ms_stats, "GB/s": bytes_stats / (ms_stats * 1e-3) / 1e9,
-                          "hbm_frac": bytes_stats / (ms_stats * 1e-3) / 1e9 / hbm},
-            "scale_search": {"ms": ms_search, "Tlane-op/s": achieved / 1e12,
-                             "W_GB/s": params * 2 / (ms_search * 1e-3) / 1e9},
-            "quantize_pack": {"ms": ms_pack, "GB/s": bytes_pack / (ms_pack * 1e-3) / 1e9,
-                              "hbm_frac": bytes_pack / (ms_pack * 1e-3) / 1e9 / hbm},
-            "hbm_peak_GBs": hbm, "peak_source": peak_src},
+        "kernels": kernels,
         "clocks": clocks,
         "e2e": e2e,
-        "gpu_launches": kernels_per_step * a.steps,
-        "launch": "CUDA graph per step" if graphs else "eager",
+        "gpu_launches": launches_per_step * a.steps,
+        "launch": "CUDA graph per step" if not a.no_graph else "eager",
     }
     if world == 1 and not a.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(Ws_h, X_h, g, n_grid, a.cpu_seconds)
+        out["cpu_baseline"] = cpu_baseline(work, g, a.cpu_seconds)
     print(json.dumps(out), flush=True)
     if world > 1:
         dist.destroy_process_group()
 
 
+def _total_params(work, world, params_rank0):
+    """Weights quantised per step by all ranks together."""
+    if work.layers > 1:
+        return work.params          # the stack is split, not replicated
+    return world * params_rank0
+
+
 # ----------------------------------------------------------- CPU oracle --
 
-def _oracle_pass(Ws, X, g, n_grid):
-    import oracle
-    x = oracle.act_stats(X)
-    err, best, s = oracle.scale_search(Ws, x, g, n_grid)
-    for W in Ws:
-        oracle.quantize_pack(W, s, g, 8)
+def oracle_sample(work, g, row_cap=256, out_rows=16, out_tokens=None):
+    """A bounded sample of layer 0 of the workload for the CPU oracle.
+
+    Weight-space workloads: the first rows of every member (all of a linear
+    up to 2^24 weights, else ``row_cap`` rows in proportion to the members'
+    sizes) with the same share of the tokens, so the stats : search : pack
+    costs keep the full layer's ratio.  The output-space workload:
+    ``out_rows`` rows of the linear with ``out_tokens`` tokens (all by
+    default); its cost per weight grows with the tokens, so the sample's
+    weights are counted times tokens / T.
+    Returns ([(Ws, X)], weights counted, description)."""
+    from post_int4_weight_b200 import workloads as wl
+    groups = wl.group_inputs(work, 0)
+    out, params, parts = [], 0.0, []
+    for grp, Ws, X in groups:
+        d_out = sum(W.shape[0] for W in Ws)
+        T = X.shape[0]
+        if work.output_mode:
+            rows, tok = out_rows, min(T, out_tokens or T)
+        else:
+            rows = d_out if d_out * grp.d_in <= (1 << 24) and row_cap >= 256 else row_cap
+            tok = max(1, T * rows // d_out)
+        Ws_s = [W[:max(8, W.shape[0] * rows // d_out)].numpy() for W in Ws]
+        out.append((Ws_s, X[:tok].numpy()))
+        n = sum(W.size for W in Ws_s)
+        params += n * tok / T if work.output_mode else n
+        parts.append(f"{grp.name}: {sum(W.shape[0] for W in Ws_s)} rows x {grp.d_in}, "
+                     f"{tok} tokens")
+    if work.output_mode:
+        mode = "stats + 20-point output-space search + pack; weights counted x tokens/T"
+    else:
+        mode = "stats + 20-point search + pack"
+    return out, params, "; ".join(parts) + f" ({mode})"
 
 
-def cpu_baseline(Ws_h, X_h, g, n_grid, seconds):
-    """Full passes of the CPU oracle over the same workload until `seconds`."""
+def _oracle_pass(sample, g, n_grid, output_mode):
     import oracle
-    Ws = [W.numpy() for W in Ws_h]
-    X = X_h.numpy()
-    params = sum(W.size for W in Ws)
+    for Ws, X in sample:
+        x = oracle.act_stats(X)
+        if output_mode:
+            err = oracle.output_error(X, Ws[0], x, g, n_grid)
+            s = oracle.scale_table(x, n_grid)[int(err.argmin())]
+        else:
+            err, best, s = oracle.scale_search(Ws, x, g, n_grid)
+        for W in Ws:
+            oracle.quantize_pack(W, s, g, 8)
+
+
+def cpu_baseline(work, g, seconds):
+    """Passes of the CPU oracle over a bounded sample of the workload until
+    `seconds` have elapsed."""
+    import oracle
+    sample, params, text = oracle_sample(work, g)
     n = 0
     t0 = time.perf_counter()
     while True:
-        _oracle_pass(Ws, X, g, n_grid)
+        _oracle_pass(sample, g, work.n_grid, work.output_mode)
         n += 1
         if time.perf_counter() - t0 >= seconds:
             break
     dt = time.perf_counter() - t0
     return {"value": n * params / dt / 1e9, "unit": UNIT, "cores": oracle.threads(),
-            "kind": "oracle",
-            "sample": f"{n} full pass(es) of the same workload (stats + 20-point search + pack)"}
+            "kind": "oracle", "sample": f"{n} pass(es) over {text}"}
 
 
 def run_reference(a):
@@ -380,38 +493,28 @@ def run_reference(a):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     if rank != 0:
         return
-    import numpy as np
     import oracle
     from post_int4_weight_b200 import workloads as wl
     work = wl.WORKLOADS[a.workload]
-    grp = work.groups[0]
-    g = work.group_sizes[0]
-    # a bounded sample of the workload per step: 64 weight rows of every
-    # member and the same share of the tokens
-    rows = 64
-    base = 100 * work.seed
-    Ws = [wl.weight(d, grp.d_in, base + m + 1)[:rows].numpy()
-          for m, (_, d) in enumerate(grp.members)]
-    tok = max(1, work.tokens * rows // sum(d for _, d in grp.members))
-    X = wl.activations(work.tokens, grp.d_in, base)[:tok].numpy()
-    params = sum(W.size for W in Ws)
+    g = _group_size(a, work)
+    # a small sample per step, so that even thousands of steps end in minutes
+    sample, params, text = oracle_sample(work, g, row_cap=64, out_rows=8, out_tokens=1024)
     for _ in range(max(a.warmup, 3)):
-        _oracle_pass(Ws, X, g, work.n_grid)
+        _oracle_pass(sample, g, work.n_grid, work.output_mode)
     t0 = time.perf_counter()
     for _ in range(a.steps):
-        _oracle_pass(Ws, X, g, work.n_grid)
+        _oracle_pass(sample, g, work.n_grid, work.output_mode)
     dt = time.perf_counter() - t0
     v = a.steps * params / dt / 1e9
-    sample = (f"{rows} rows x {grp.d_in} of each linear and {tok} tokens per step "
-              f"(stats + 20-point search + pack)")
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": world,
         "steps": a.steps, "warmup": a.warmup, "ms_per_step": dt / a.steps * 1e3,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "higher_is_better": True, "scaling": "strong" if work.layers > 1 else "weak",
+        "vs_baseline": None, "dtype": "f64" if work.output_mode else "f32",
         "data": "synthetic", "config": {"workload": a.workload, "group_size": g,
                                         "n_grid": work.n_grid},
         "cpu_baseline": {"value": v, "unit": UNIT, "cores": oracle.threads(),
-                         "kind": "oracle", "sample": sample},
+                         "kind": "oracle", "sample": f"per step, one pass over {text}"},
         "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }), flush=True)
 

@@ -216,24 +216,39 @@ awq_status awq_quantize_pack(const void *W, int64_t d_out, int64_t d_in,
  *
  *   err[i] = || X (W - W_hat_i)^T ||_F^2,   W_hat_i = Q(W * s_i) / s_i
  *
- * with s_i and Q exactly as in awq_scale_search.  W - W_hat_i is rounded to
- * fp16 and multiplied by X on the tensor cores (fp16 in, fp32 accumulate);
- * the squares are summed in fp32 per tile and in fp64 across tiles.
+ * with s_i and Q exactly as in awq_scale_search.  The contraction runs on
+ * the tensor cores with fp16 operands and fp32 accumulation.  W - W_hat_i
+ * is formed exactly in fp32, scaled per row by a power of two, and split
+ * into two fp16 parts hi + lo (lo = the rounding error of hi), so that the
+ * product sees the difference to about 22 bits; X is fp16 already, so
+ * X (hi + lo)^T accumulates both parts into one fp32 accumulator.  The
+ * running accumulator is folded into a second fp32 sum every 2048 terms of
+ * the (hi, lo)-doubled reduction, the squares are summed in fp32 per 128 x 256 output tile and
+ * in fp64 across tiles.  The result is tested against the fp64
+ * definition at 1e-5 relative.
  *
- *   X           fp16 [T, d_in] device;  T >= 1
+ *   X           fp16 [T, d_in] device;  1 <= T <= 2^24
  *   W           fp16 [d_out, d_in] device; d_out % 8 == 0
  *   x_mean      fp32 [d_in] device (defines s_i)
  *   group_size  32, 64 or 128;  d_in multiple of group_size and of 64
  *   n_grid      1..32;  flags as in awq_scale_search
- *   err         fp64 [n_grid] device output
- *   best_idx    int32 [1] device output (first minimum; -1 if non-finite)
- *   ws          workspace of awq_workspace_size(AWQ_OP_OUTPUT_ERROR, ...)
+ *   err         fp64 [n_grid] device output (NaN for every i if W holds a
+ *               non-finite value)
+ *   best_idx    int32 [1] device output (first minimum; -1 if non-finite,
+ *               -2 if a bounded wait inside a kernel gave up)
+ *   s_best      fp32 [d_in] device output s_{best_idx} (NaN if best_idx < 0),
+ *               or NULL when the caller does not want it
+ *   ws          workspace of awq_workspace_size(AWQ_OP_OUTPUT_ERROR, ...),
+ *               256-byte aligned
+ * Errors: AWQ_ERR_INVALID_ARG / AWQ_ERR_UNSUPPORTED / AWQ_ERR_ALIGNMENT /
+ * AWQ_ERR_WORKSPACE before any launch, AWQ_ERR_CUDA when a launch fails
+ * (awq_last_error() then holds the CUDA error text).
  */
 awq_status awq_output_error(const void *X, int64_t T, const void *W,
                             int64_t d_out, int64_t d_in, const float *x_mean,
                             int group_size, int n_grid, int flags,
-                            double *err, int32_t *best_idx, void *ws,
-                            size_t ws_bytes, void *stream);
+                            double *err, int32_t *best_idx, float *s_best,
+                            void *ws, size_t ws_bytes, void *stream);
 
 #ifdef __cplusplus
 }

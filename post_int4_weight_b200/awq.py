@@ -62,7 +62,7 @@ def lib() -> ctypes.CDLL:
         L.awq_scale_search.restype = i32
         L.awq_quantize_pack.argtypes = [p, i64, i64, p, i32, i32, p, p, p, p]
         L.awq_quantize_pack.restype = i32
-        L.awq_output_error.argtypes = [p, i64, p, i64, i64, p, i32, i32, i32, p, p, p, sz, p]
+        L.awq_output_error.argtypes = [p, i64, p, i64, i64, p, i32, i32, i32, p, p, p, p, sz, p]
         L.awq_output_error.restype = i32
         _lib = L
     return _lib
@@ -176,24 +176,29 @@ def quantize_pack(W: torch.Tensor, s: Optional[torch.Tensor] = None, group_size:
 
 
 def output_error(X: torch.Tensor, W: torch.Tensor, x: torch.Tensor, group_size: int = 128,
-                 n_grid: int = 20, flags: int = SCALE_FP16, ws: Optional[torch.Tensor] = None):
+                 n_grid: int = 20, flags: int = SCALE_FP16,
+                 out: Optional[Tuple[torch.Tensor, torch.Tensor, torch.Tensor]] = None,
+                 ws: Optional[torch.Tensor] = None):
     """Output-space score ||X (W - W_hat_i)^T||^2 per grid point:
-    (err fp64[n_grid], best_idx int32[1])."""
+    (err fp64[n_grid], best_idx int32[1], s_best fp32[d_in])."""
     _cuda(X, torch.float16, "X")
     _cuda(W, torch.float16, "W")
     _cuda(x, torch.float32, "x")
     T, d_in = X.shape
     d_out = W.shape[0]
     dev = X.device
-    err = torch.empty(n_grid, dtype=torch.float64, device=dev)
-    best = torch.empty(1, dtype=torch.int32, device=dev)
+    if out is None:
+        out = (torch.empty(n_grid, dtype=torch.float64, device=dev),
+               torch.empty(1, dtype=torch.int32, device=dev),
+               torch.empty(d_in, dtype=torch.float32, device=dev))
+    err, best, s_best = out
     if ws is None:
         ws = workspace(OP_OUTPUT_ERROR, dev, T, d_out, d_in, group_size, n_grid)
     _check(lib().awq_output_error(X.data_ptr(), T, W.data_ptr(), d_out, d_in, x.data_ptr(),
                                   group_size, n_grid, flags, err.data_ptr(), best.data_ptr(),
-                                  ws.data_ptr(), ws.numel(), _stream(dev)),
+                                  s_best.data_ptr(), ws.data_ptr(), ws.numel(), _stream(dev)),
            "awq_output_error")
-    return err, best
+    return err, best, s_best
 
 
 def quantize_group(Ws: Sequence[torch.Tensor], X: torch.Tensor, group_size: int = 128,

@@ -156,8 +156,8 @@ awq_status awq_quantize_pack(const void* W, int64_t d_out, int64_t d_in, const f
 
 awq_status awq_output_error(const void* X, int64_t T, const void* W, int64_t d_out,
                             int64_t d_in, const float* x_mean, int group_size, int n_grid,
-                            int flags, double* err, int32_t* best_idx, void* ws,
-                            size_t ws_bytes, void* stream) {
+                            int flags, double* err, int32_t* best_idx, float* s_best,
+                            void* ws, size_t ws_bytes, void* stream) {
     if (!X || !W || !x_mean || !err || !best_idx) return AWQ_ERR_INVALID_ARG;
     if (!valid_group(group_size)) return AWQ_ERR_UNSUPPORTED;
     if (n_grid < 1 || n_grid > 32) return AWQ_ERR_INVALID_ARG;
@@ -167,13 +167,13 @@ awq_status awq_output_error(const void* X, int64_t T, const void* W, int64_t d_o
     if (d_in < group_size || d_in % group_size || d_in % 64 || d_in > (int64_t(1) << 20))
         return AWQ_ERR_INVALID_ARG;
     if (!aligned16(X) || !aligned16(W) || !aligned16(x_mean) || !aligned16(err) ||
-        !aligned16(best_idx))
+        !aligned16(best_idx) || (s_best && !aligned16(s_best)))
         return AWQ_ERR_ALIGNMENT;
     if (!ws || ws_bytes < output_error_workspace(T, d_out, d_in, group_size, n_grid))
         return AWQ_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(ws) & (kWsAlign - 1)) != 0) return AWQ_ERR_ALIGNMENT;
     return launch_output_error(X, T, W, d_out, d_in, x_mean, group_size, n_grid, flags, err,
-                               best_idx, ws, static_cast<cudaStream_t>(stream));
+                               best_idx, s_best, ws, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

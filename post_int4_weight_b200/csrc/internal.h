@@ -56,7 +56,7 @@ size_t output_error_workspace(int64_t T, int64_t d_out, int64_t d_in, int group_
 awq_status launch_output_error(const void* X, int64_t T, const void* W, int64_t d_out,
                                int64_t d_in, const float* x_mean, int group_size,
                                int n_grid, int flags, double* err, int32_t* best_idx,
-                               void* ws, cudaStream_t stream);
+                               float* s_best, void* ws, cudaStream_t stream);
 
 // ---- shared pieces of the search and the output-error mode
 // Writes S[i][j] and tau[i][j] = x_mean[j] / S[i][j] (or 1 / S[i][j] when

@@ -501,8 +501,8 @@ size_t output_error_workspace(int64_t T, int64_t d_out, int64_t d_in, int group_
 
 awq_status launch_output_error(const void* X, int64_t T, const void* W, int64_t d_out,
                                int64_t d_in, const float* x_mean, int group_size, int n_grid,
-                               int flags, double* err, int32_t* best_idx, void* ws,
-                               cudaStream_t stream) {
+                               int flags, double* err, int32_t* best_idx, float* s_best,
+                               void* ws, cudaStream_t stream) {
     DeviceInfo dev;
     if (query_device(&dev) != cudaSuccess) return AWQ_ERR_CUDA;
     EncodeTiledFn encode = encode_tiled_fn();
@@ -574,7 +574,7 @@ awq_status launch_output_error(const void* X, int64_t T, const void* W, int64_t 
         if (note_cuda(cudaGetLastError(), "oe_gemm launch") != cudaSuccess) return AWQ_ERR_CUDA;
     }
     if (note_cuda(launch_finalize(w.partial, grid, n_grid, w.S, d_in, w.dev_words, err,
-                                  best_idx, nullptr, stream),
+                                  best_idx, s_best, stream),
                   "finalize launch") != cudaSuccess)
         return AWQ_ERR_CUDA;
     return AWQ_OK;

@@ -1,0 +1,230 @@
+"""Orchestration of the AWQ hot path over search groups, layers and stacks.
+
+Host plumbing only: output buffers, shared workspaces, CUDA streams, events
+and the split of a stack's layers over ranks.  Every step of the method runs
+in the library's kernels through the calls of :mod:`awq`.
+
+The unit of work is a *search group*: the linears that read one input X
+(q/k/v, gate/up, or a linear alone).  Its path is awq_act_stats on X, the
+scale search (weight-space, or output-space with ``output_mode``) over all
+members at once, then awq_quantize_pack of every member at the chosen scale
+("From-Scratch AWQ INT4 Quantization on Qwen3-8B", pipeline and AWQ scaling
+sections; "AWQ architecture, in depth", section "The scale search as code").
+"""
+from __future__ import annotations
+
+from typing import List, Sequence, Tuple
+
+import torch
+
+from . import awq
+
+# kernels each call launches (the library's own count, used for reporting)
+LAUNCHES_STATS = 1
+LAUNCHES_SEARCH = 3            # scale table (2) + fused search with finalize
+
+
+def launches_output_error(n_grid: int) -> int:
+    """Scale table (2) + one dW builder and one GEMM per grid point + finalize."""
+    return 2 + 2 * n_grid + 1
+
+
+def shard_layers(n_layers: int, world: int, rank: int) -> List[int]:
+    """Layers of a stack that one rank quantises: layer l goes to rank l % world.
+
+    Layers are independent units of the path (each has its own inputs and
+    outputs), so the split needs no exchange between ranks."""
+    if world < 1 or not 0 <= rank < world:
+        raise ValueError(f"rank {rank} outside world of {world}")
+    return list(range(rank, n_layers, world))
+
+
+def max_over_ranks(value: float, device=None) -> float:
+    """Maximum of a per-rank number over all ranks of the default process
+    group (the rank's own value when there is no group)."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    if device is None:
+        device = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+class GroupJob:
+    """One search group on the device with its output buffers.
+
+    Ws: fp16 [d_out_k, d_in] device tensors sharing the input X fp16 [T, d_in].
+    After :meth:`run`: ``x`` (activation magnitude), ``err`` (per grid point),
+    ``best``, ``s_best`` and ``packs`` [(qweight, scales, qzeros) per member].
+    """
+
+    def __init__(self, Ws: Sequence[torch.Tensor], X: torch.Tensor, group_size: int = 128,
+                 n_grid: int = 20, output_mode: bool = False, zero_point: int = 8):
+        if output_mode and len(Ws) != 1:
+            raise ValueError("the output-space score takes one linear per call")
+        self.Ws = list(Ws)
+        self.X = X
+        self.g = group_size
+        self.n_grid = n_grid
+        self.output_mode = output_mode
+        self.zero_point = zero_point
+        dev = X.device
+        T, d_in = X.shape
+        self.x = torch.empty(d_in, dtype=torch.float32, device=dev)
+        self.err = torch.empty(n_grid, dtype=torch.float64, device=dev)
+        self.best = torch.empty(1, dtype=torch.int32, device=dev)
+        self.s_best = torch.empty(d_in, dtype=torch.float32, device=dev)
+        G = d_in // group_size
+        self.packs = [(torch.empty(d_in, W.shape[0] // 8, dtype=torch.int32, device=dev),
+                       torch.empty(G, W.shape[0], dtype=torch.float16, device=dev),
+                       torch.empty(G, W.shape[0] // 8, dtype=torch.int32, device=dev))
+                      for W in self.Ws]
+
+    @property
+    def params(self) -> int:
+        return sum(W.numel() for W in self.Ws)
+
+    @property
+    def launches(self) -> int:
+        search = launches_output_error(self.n_grid) if self.output_mode else LAUNCHES_SEARCH
+        return LAUNCHES_STATS + search + len(self.Ws)
+
+    def workspace_bytes(self) -> Tuple[int, int]:
+        """(act_stats, search) workspace bytes of this job."""
+        T, d_in = self.X.shape
+        d_out = sum(W.shape[0] for W in self.Ws)
+        st = awq.workspace_size(awq.OP_ACT_STATS, T, 8, d_in, self.g, self.n_grid)
+        op = awq.OP_OUTPUT_ERROR if self.output_mode else awq.OP_SCALE_SEARCH
+        se = awq.workspace_size(op, T, d_out, d_in, self.g, self.n_grid)
+        return st, se
+
+    def stats(self, ws: torch.Tensor):
+        awq.act_stats(self.X, out=self.x, ws=ws)
+
+    def search(self, ws: torch.Tensor):
+        out = (self.err, self.best, self.s_best)
+        if self.output_mode:
+            awq.output_error(self.X, self.Ws[0], self.x, self.g, self.n_grid, out=out, ws=ws)
+        else:
+            awq.scale_search(self.Ws, self.x, self.g, self.n_grid, out=out, ws=ws)
+
+    def pack(self):
+        for W, pk in zip(self.Ws, self.packs):
+            awq.quantize_pack(W, self.s_best, self.g, self.zero_point, out=pk)
+
+    def run(self, ws: "Workspaces"):
+        self.stats(ws.stats)
+        self.search(ws.search)
+        self.pack()
+
+
+class Workspaces:
+    """One workspace per call kind, sized for the largest of ``jobs``.  Jobs
+    that run one after another on one stream may share it; jobs that run
+    concurrently need their own."""
+
+    def __init__(self, jobs: Sequence[GroupJob], device):
+        st = max([j.workspace_bytes()[0] for j in jobs] + [1])
+        se = max([j.workspace_bytes()[1] for j in jobs] + [1])
+        self.stats = torch.empty(st, dtype=torch.uint8, device=device)
+        self.search = torch.empty(se, dtype=torch.uint8, device=device)
+
+
+def _pinned_like(t: torch.Tensor) -> torch.Tensor:
+    return torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+
+
+class LayerStreamer:
+    """Quantises layers held in pinned host memory, end to end.
+
+    A ring of ``depth`` device slots (each slot: the inputs and outputs of one
+    layer) is driven by three streams: host-to-device copies of layer l+1 run
+    on one, the kernels of layer l on another, and the device-to-host copies
+    of layer l-1's results on a third, ordered by events per slot.  A layer is
+    given as [(Ws, X) per search group] of pinned CPU tensors; all layers have
+    the shapes of ``template`` (the same list with device or CPU tensors).
+    """
+
+    def __init__(self, template, device, group_size: int = 128, n_grid: int = 20,
+                 output_mode: bool = False, zero_point: int = 8, depth: int = 2):
+        self.device = torch.device(device)
+        self.depth = depth
+        self.slots = []
+        for _ in range(depth):
+            jobs = []
+            for Ws, X in template:
+                dWs = [torch.empty(W.shape, dtype=torch.float16, device=self.device) for W in Ws]
+                dX = torch.empty(X.shape, dtype=torch.float16, device=self.device)
+                jobs.append(GroupJob(dWs, dX, group_size, n_grid, output_mode, zero_point))
+            self.slots.append(jobs)
+        self.ws = Workspaces(self.slots[0], self.device)
+        self.h2d = torch.cuda.Stream(self.device)
+        self.compute = torch.cuda.Stream(self.device)
+        self.d2h = torch.cuda.Stream(self.device)
+        self.loaded = [torch.cuda.Event() for _ in range(depth)]
+        self.computed = [torch.cuda.Event() for _ in range(depth)]
+        self.drained = [torch.cuda.Event() for _ in range(depth)]
+        cur = torch.cuda.current_stream(self.device)
+        for evs in (self.loaded, self.computed, self.drained):
+            for e in evs:
+                e.record(cur)
+
+    @property
+    def launches_per_layer(self) -> int:
+        return sum(j.launches for j in self.slots[0])
+
+    def host_outputs(self):
+        """Pinned host buffers for one layer's results:
+        [(err, best, s_best, [(qweight, scales, qzeros) per member]) per group]."""
+        return [(_pinned_like(j.err), _pinned_like(j.best), _pinned_like(j.s_best),
+                 [tuple(_pinned_like(t) for t in pk) for pk in j.packs])
+                for j in self.slots[0]]
+
+    def bytes_per_layer(self) -> Tuple[int, int]:
+        """(host-to-device, device-to-host) bytes copied per layer."""
+        jobs = self.slots[0]
+        h2d = sum(j.X.numel() * 2 + sum(W.numel() * 2 for W in j.Ws) for j in jobs)
+        d2h = sum(j.err.numel() * 8 + 4 + j.s_best.numel() * 4 +
+                  sum(t.numel() * t.element_size() for pk in j.packs for t in pk)
+                  for j in jobs)
+        return h2d, d2h
+
+    def run(self, host_layers, host_out, after=None):
+        """Enqueue every layer of ``host_layers``; results land in the matching
+        entries of ``host_out``.  ``after``: an event the copies must wait
+        for.  Returns with the work enqueued; the current stream waits for all
+        of it."""
+        if after is not None:
+            for s in (self.h2d, self.compute, self.d2h):
+                s.wait_event(after)
+        for l, layer in enumerate(host_layers):
+            k = l % self.depth
+            jobs = self.slots[k]
+            self.h2d.wait_event(self.computed[k])     # the slot's inputs are free
+            with torch.cuda.stream(self.h2d):
+                for job, (Ws, X) in zip(jobs, layer):
+                    job.X.copy_(X, non_blocking=True)
+                    for dW, W in zip(job.Ws, Ws):
+                        dW.copy_(W, non_blocking=True)
+            self.loaded[k].record(self.h2d)
+            self.compute.wait_event(self.loaded[k])
+            self.compute.wait_event(self.drained[k])  # the slot's outputs are free
+            with torch.cuda.stream(self.compute):
+                for job in jobs:
+                    job.run(self.ws)
+            self.computed[k].record(self.compute)
+            self.d2h.wait_event(self.computed[k])
+            with torch.cuda.stream(self.d2h):
+                for job, (err, best, s_best, packs) in zip(jobs, host_out[l]):
+                    err.copy_(job.err, non_blocking=True)
+                    best.copy_(job.best, non_blocking=True)
+                    s_best.copy_(job.s_best, non_blocking=True)
+                    for pk_h, pk in zip(packs, job.packs):
+                        for th, t in zip(pk_h, pk):
+                            th.copy_(t, non_blocking=True)
+            self.drained[k].record(self.d2h)
+        cur = torch.cuda.current_stream(self.device)
+        for s in (self.h2d, self.compute, self.d2h):
+            cur.wait_stream(s)

@@ -118,13 +118,14 @@ def layer_seed(workload: Workload, layer: int) -> int:
     return 1000 * (workload.seed + 1) + layer
 
 
-def group_inputs(workload: Workload, layer: int = 0, device="cpu"):
+def group_inputs(workload: Workload, layer: int = 0, device="cpu", seed=None):
     """Weights and activations of every search group of one layer.
 
-    Returns a list of (SearchGroup, [W per member], X).  Member m of group k
-    uses seed ``base + 16*k + m + 1`` and the group's X uses ``base + 16*k``.
+    Returns a list of (SearchGroup, [W per member], X).  With base = 100 *
+    (``seed`` if given, else the layer's seed), member m of group k uses seed
+    ``base + 16*k + m + 1`` and the group's X uses ``base + 16*k``.
     """
-    base = 100 * layer_seed(workload, layer)
+    base = 100 * (layer_seed(workload, layer) if seed is None else int(seed))
     out = []
     for k, grp in enumerate(workload.groups):
         Ws = [weight(d, grp.d_in, base + 16 * k + m + 1, device)

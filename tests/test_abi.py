@@ -95,6 +95,26 @@ def test_host_validation_without_a_gpu():
     assert L.awq_quantize_pack(fake, 64, 256, odd, 128, 8, fake, fake, fake, None) == 3
     # output_error
     assert L.awq_output_error(fake, 0, fake, 64, 256, fake, 128, 20, 0, fake, fake,
-                              fake, 1 << 30, None) == 1
+                              None, fake, 1 << 30, None) == 1
     assert L.awq_output_error(fake, 16, fake, 64, 256, fake, 128, 20, 0, fake, fake,
-                              fake, 16, None) == 4
+                              None, fake, 16, None) == 4
+    assert L.awq_output_error(fake, 16, fake, 64, 256, fake, 128, 20, 0, fake, fake,
+                              odd, fake, 1 << 30, None) == 3
+
+
+def test_pipeline_workspace_sizes_from_host_query():
+    """GroupJob sizes its workspaces through awq_workspace_size (a host-only
+    call): the weight-space and output-space searches of the same group."""
+    import torch
+    from post_int4_weight_b200 import pipeline
+    Ws = [torch.zeros(256, 512, dtype=torch.float16), torch.zeros(128, 512, dtype=torch.float16)]
+    X = torch.zeros(64, 512, dtype=torch.float16)
+    j = pipeline.GroupJob(Ws, X, 128, 20)
+    st, se = j.workspace_bytes()
+    assert st >= 0 and se > 0
+    jo = pipeline.GroupJob(Ws[:1], X, 128, 20, output_mode=True)
+    st_o, se_o = jo.workspace_bytes()
+    assert se_o >= 2 * 256 * 512 * 2            # the hi/lo dW buffer at least
+    assert j.launches == 1 + 3 + 2 and jo.launches == 1 + 43 + 1
+    ws = pipeline.Workspaces([j, jo], "cpu")
+    assert ws.search.numel() == max(se, se_o)

@@ -1,10 +1,11 @@
 """Output-space scoring (tcgen05 GEMM path) against the CPU oracle.
 
 err[i] = ||X (W - W_hat_i)^T||^2.  The oracle evaluates it in fp64 from the
-exact W - W_hat_i; the GPU rounds W - W_hat_i to fp16 (row-scaled) and
-accumulates X dW^T in fp32 on the tensor cores, so the bar is the error-sum
-tolerance, 1e-5 relative, and the chosen index must agree (or tie within
-1e-6).
+exact W - W_hat_i; the GPU splits the row-scaled W - W_hat_i into two fp16
+parts and accumulates X dW^T in fp32 on the tensor cores, so the bar is the
+error-sum tolerance, 1e-5 relative, and the chosen index must agree (or tie
+within 1e-6).  The returned s_best is the scale-table row of the chosen
+index, bit-exact.
 """
 import numpy as np
 import pytest
@@ -25,10 +26,17 @@ def _cuda():
 
 
 def _run(X, W, x_np, g, n_grid=20, flags=0):
-    err, best = awq.output_error(X.cuda(), W.cuda(), torch.from_numpy(x_np).cuda(), g,
-                                 n_grid, flags)
+    err, best, s_best = awq.output_error(X.cuda(), W.cuda(), torch.from_numpy(x_np).cuda(),
+                                         g, n_grid, flags)
     torch.cuda.synchronize()
-    return err.cpu().numpy(), int(best.cpu()[0])
+    b = int(best.cpu()[0])
+    s_best = s_best.cpu().numpy()
+    if b >= 0:
+        S = oracle.scale_table(x_np, n_grid)
+        np.testing.assert_array_equal(s_best.view(np.uint32), S[b].view(np.uint32))
+    else:
+        assert np.isnan(s_best).all()
+    return err.cpu().numpy(), b
 
 
 def _check(err_g, best_g, err_o):

@@ -1,0 +1,100 @@
+"""Layer orchestration on the GPU against the CPU oracle.
+
+* LayerStreamer: layers streamed from pinned host memory through a 2-slot
+  device ring on three streams give, layer by layer, exactly the oracle's
+  results (a slot reused too early would mix two layers' data).
+* One full layer of the 36-layer Qwen3-8B-shaped stack (2048 tokens per
+  layer, 7 linears in 4 search groups) through GroupJob, every group
+  compared with the oracle: bit-exact means, scales, codes, words, index;
+  error sums within 1e-5 relative.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from post_int4_weight_b200 import pipeline
+from post_int4_weight_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+ERR_RTOL = 1e-5
+TIE_RTOL = 1e-6
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    assert torch.cuda.is_available(), "the gpu tests need a CUDA device"
+
+
+def _oracle_group(Ws, X, g, n_grid, output_mode):
+    x = oracle.act_stats(X)
+    if output_mode:
+        err = oracle.output_error(X, Ws[0], x, g, n_grid)
+        best = int(np.argmin(err))
+        s = oracle.scale_table(x, n_grid)[best]
+    else:
+        err, best, s = oracle.scale_search(Ws, x, g, n_grid)
+    packs = [oracle.quantize_pack(W, s, g, 8) for W in Ws]
+    return x, err, best, s, packs
+
+
+def _compare(got, Ws, X, g, n_grid, output_mode):
+    """got = (x or None, err, best, s_best, packs) as numpy."""
+    x_o, err_o, best_o, s_o, packs_o = _oracle_group(Ws, X, g, n_grid, output_mode)
+    x, err, best, s, packs = got
+    if x is not None:
+        assert np.array_equal(x, x_o)
+    np.testing.assert_allclose(err, err_o, rtol=ERR_RTOL, atol=0)
+    if best != best_o:
+        assert abs(err_o[best] - err_o[best_o]) <= TIE_RTOL * err_o[best_o]
+        return
+    assert np.array_equal(s, s_o)
+    for (qw, sc, qz), (qw_o, sc_o, qz_o) in zip(packs, packs_o):
+        assert np.array_equal(qw, qw_o)
+        assert np.array_equal(sc.view(np.uint16), sc_o.view(np.uint16))
+        assert np.array_equal(qz, qz_o)
+
+
+def _small_layer(seed):
+    """Two search groups: (256 + 128) x 512 with 64 tokens, 128 x 1024 with
+    96 tokens."""
+    return [([wl.weight(256, 512, seed + 1), wl.weight(128, 512, seed + 2)],
+             wl.activations(64, 512, seed)),
+            ([wl.weight(128, 1024, seed + 4)], wl.activations(96, 1024, seed + 3))]
+
+
+@pytest.mark.parametrize("output_mode", [False, True])
+def test_layer_streamer_matches_oracle_per_layer(output_mode):
+    g, n_grid, n_layers = 128, 20, 5
+    layers = [_small_layer(1000 + 10 * l) for l in range(n_layers)]
+    if output_mode:
+        layers = [[(Ws[:1], X) for Ws, X in lay] for lay in layers]
+    host = [[([W.pin_memory() for W in Ws], X.pin_memory()) for Ws, X in lay]
+            for lay in layers]
+    st = pipeline.LayerStreamer(layers[0], "cuda", g, n_grid, output_mode)
+    out = [st.host_outputs() for _ in range(n_layers)]
+    st.run(host, out)
+    torch.cuda.synchronize()
+    for lay, res in zip(layers, out):
+        for (Ws, X), (err, best, s, packs) in zip(lay, res):
+            got = (None, err.numpy(), int(best[0]), s.numpy(),
+                   [tuple(t.numpy() for t in pk) for pk in packs])
+            _compare(got, [W.numpy() for W in Ws], X.numpy(), g, n_grid, output_mode)
+
+
+def test_stack36_layer_full_parity():
+    work = wl.WORKLOADS["qwen3_8b_stack36"]
+    layer = work.layers - 1
+    groups = wl.group_inputs(work, layer)
+    dev = torch.device("cuda")
+    jobs = [pipeline.GroupJob([W.to(dev) for W in Ws], X.to(dev), 128, work.n_grid)
+            for _, Ws, X in groups]
+    wss = pipeline.Workspaces(jobs, dev)
+    for j in jobs:
+        j.run(wss)
+    torch.cuda.synchronize()
+    for (grp, Ws, X), j in zip(groups, jobs):
+        got = (j.x.cpu().numpy(), j.err.cpu().numpy(), int(j.best.cpu()[0]),
+               j.s_best.cpu().numpy(), [tuple(t.cpu().numpy() for t in pk) for pk in j.packs])
+        _compare(got, [W.numpy() for W in Ws], X.numpy(), 128, work.n_grid, False)
