@@ -59,16 +59,17 @@ awq_status launch_output_error(const void* X, int64_t T, const void* W, int64_t 
                                float* s_best, void* ws, cudaStream_t stream);
 
 // ---- shared pieces of the search and the output-error mode
-// Writes S[i][j] and tau[i][j] = x_mean[j] / S[i][j] (or 1 / S[i][j] when
-// write_inverse) (fp32, [n_grid][d_in]) with two kernels (pow + per-slice
-// min/max, then normalise); `part` holds 2 * n_grid * kMaxTableSlices
-// doubles.  Clears *dev_words (2 ints: error word, CTA-done counter) if
-// non-NULL.  The second kernel is a programmatic dependent launch of the
-// first.
+// Writes S[i][j] (fp32, [n_grid][d_in]) and a companion table T[i][j] of the
+// same shape: (x_mean[j] / S[i][j])^2 for the weight-space search
+// (kTableTauSq) or 1 / S[i][j] for the output-space mode (kTableInverse).
+// One kernel; clears dev_words[0..1] (error word, CTA-done counter) if
+// non-NULL.  Launched as an ordinary launch, so it follows every earlier
+// kernel of the stream completely.
+enum TableKind { kTableTauSq = 0, kTableInverse = 1 };
 constexpr int kMaxTableSlices = 64;
 cudaError_t launch_scale_table(const float* x_mean, int64_t d_in, int n_grid, float* S,
-                               float* tau, double* part, int* dev_words, int num_sms,
-                               cudaStream_t stream, bool write_inverse = false);
+                               float* T, int* dev_words, int num_sms, cudaStream_t stream,
+                               TableKind kind);
 
 // Launch with the programmatic stream-serialisation attribute (the kernel
 // must call pdl_wait() before depending on its predecessor).

@@ -554,8 +554,8 @@ awq_status launch_output_error(const void* X, int64_t T, const void* W, int64_t 
         configured[dev.device] = 1;
     }
 
-    if (note_cuda(launch_scale_table(x_mean, d_in, n_grid, w.S, w.inv_s, w.partial,
-                                     w.dev_words, dev.num_sms, stream, /*write_inverse=*/true),
+    if (note_cuda(launch_scale_table(x_mean, d_in, n_grid, w.S, w.inv_s, w.dev_words,
+                                     dev.num_sms, stream, kTableInverse),
                   "scale table launch") != cudaSuccess)
         return AWQ_ERR_CUDA;
     for (int a = 0; a < n_grid; ++a) {

@@ -7,38 +7,43 @@
 // W*s_i is fake-quantised group-wise to symmetric INT4 with an fp16 group
 // scale, and scored by sum(((W - Q(W s_i)/s_i) * x)^2).
 //
-// Kernels (all on the caller's stream; the second and third are programmatic
-// dependent launches of the one before):
-//   table_minmax_kernel  (slices x alphas) CTAs: s_i[j] = max(x,1e-4)^alpha in
-//                        fp64, per-slice min and max;
-//   table_write_kernel   same grid: sqrt(max*min) from the slice partials,
-//                        s_i rounded to fp32 and tau_i = x / s_i;
-//   search_kernel        persistent, 2 CTAs per SM.  A work unit is one group
-//                        of g input channels x R rows of one weight segment.
-//                        Thread 0 streams units into a 2-stage shared-memory
-//                        ring with TMA (cp.async.bulk.tensor, mbarrier
-//                        completion), starting before the scale table is
-//                        ready; W is read from HBM exactly once and kept in
-//                        registers as fp32 while all grid points are
-//                        evaluated.  The last CTA to finish sums the per-CTA
-//                        partials in a fixed order (fp64), picks the first
-//                        minimum and copies s_best.
+// Kernels (all on the caller's stream):
+//   table_kernel   (slices x alphas) CTAs.  pow is monotonic in x, so
+//                  max_j s_i[j] and min_j s_i[j] come from the largest and
+//                  smallest max(x_j, 1e-4), which every CTA finds by itself;
+//                  then s_i[j] = pow(max(x_j,1e-4), alpha_i) / sqrt(max*min)
+//                  (fp64, rounded once to fp32) and tau2_i[j] = (x_j/s_i[j])^2
+//                  for the CTA's slice of channels.
+//   search_kernel  persistent, one CTA of 16 warps per SM (a programmatic
+//                  dependent launch of the table kernel).  A work unit is one
+//                  group of g input channels x R rows of one weight segment.
+//                  Thread 0 streams units into a 2-stage shared-memory ring
+//                  with TMA (cp.async.bulk.tensor, mbarrier completion),
+//                  starting before the scale table is ready; W is read from
+//                  HBM exactly once and kept in registers as fp32 while all
+//                  grid points are evaluated.  The last CTA to finish sums
+//                  the per-CTA partials in a fixed order (fp64), picks the
+//                  first minimum and copies s_best.
+// One CTA per SM (rather than two of 8 warps) keeps the SM's warps on one
+// range of units: two co-resident CTAs drift apart under the scheduler's
+// age priority and the later one ends alone on its SM.
 //
-// Register-level formulation of one (weight, alpha) pair, 6 FMA-pipe ops plus
-// one max, issued as packed fp32x2 instructions (sm_100):
+// Register-level formulation of one (weight, alpha) pair: 5 FMA-pipe ops and
+// one max, mostly packed fp32x2 instructions (sm_100).  Each lane holds the
+// same 16 channels of two rows r0, r1:
 //   ws = w * s                         (exact fp32 product, as the method)
 //   m  = max(m, |ws|)                  (then shuffled across the L lanes)
 //   t  = ws * (1/q_scale) + 1.5*2^23   (rounds to the nearest code, ties even)
 //   q  = t - 1.5*2^23
 //   d  = ws - q * q_scale              (= (w - w_hat) * s)
-//   e  = d * tau,  tau = x / s         (= (w - w_hat) * x)
-//   acc += e * e
-// q_scale itself is computed exactly as the method states (IEEE fp32 quotient
-// by 7, fp16 round-to-nearest-even).  The code decision uses the reciprocal of
-// q_scale instead of the IEEE quotient; the two differ only when ws/q_scale
-// lies within an ulp of a half-integer, where either code's error is the same
-// to ~1e-7 of a step.  The exact quotient is used where codes are stored
-// (pack.cu).
+//   acc += tau2 * (d_r0^2 + d_r1^2),   tau2 = (x / s)^2
+// so that ((w - w_hat) * x)^2 = d^2 * tau2 is summed without forming each
+// product d * tau.  q_scale itself is computed exactly as the method states
+// (IEEE fp32 quotient by 7, fp16 round-to-nearest-even).  The code decision
+// uses the reciprocal of q_scale instead of the IEEE quotient; the two differ
+// only when ws/q_scale lies within an ulp of a half-integer, where either
+// code's error is the same to ~1e-7 of a step.  The exact quotient is used
+// where codes are stored (pack.cu).
 #include <algorithm>
 #include <cstring>
 
@@ -48,12 +53,14 @@
 namespace awq {
 namespace {
 
-constexpr int kConsumerWarps = 8;
+constexpr int kConsumerWarps = 16;
 constexpr int kThreads = kConsumerWarps * 32;
 constexpr int kStages = 2;
 constexpr int kElemsPerRow = 16;           // weights of each of a lane's two rows
-constexpr int kUnitBytes = 16384;          // R * g * 2 for every group size
+constexpr int kUnitBytes = 32768;          // R * g * 2 for every group size
+constexpr int kMaxBoxRows = 256;           // TMA box limit: R is loaded in boxes of <= 256 rows
 constexpr int kMaxGrid = 32;
+constexpr int kMaxParts = 1024;            // per-CTA partials (grid size bound)
 
 struct SearchParams {
     CUtensorMap tmap[AWQ_MAX_SEGMENTS];    // fp16 [d_out_k, d_in], box [g, R]
@@ -66,7 +73,7 @@ struct SearchParams {
     int64_t n_units;
     int64_t d_in;
     const float* S;        // [n_grid][d_in]
-    const float* tau;      // [n_grid][d_in]
+    const float* tau2;     // [n_grid][d_in], (x / s)^2
     double* partial;       // [gridDim.x][n_grid]
     int* dev_words;        // [0] error bits, [1] CTAs done
     double* err;           // [n_grid] output
@@ -87,22 +94,48 @@ __device__ __forceinline__ int table_slot(int c) {
     return (((k2 * 2 + h) * L + l) << 2) + e;
 }
 
-// Sum of the CTAs' partial errors in a fixed order (lane-strided, then a
-// fixed shuffle tree), the first minimum, and s_best.  Run by one CTA of
-// kThreads threads after every partial is visible.
+// Sum of the CTAs' partial errors in a fixed order (for every alpha, lane k
+// adds the partials k, k + 32, k + 64, ... in that order, then a fixed
+// shuffle tree), the first minimum, and s_best.  Run by one CTA of kThreads
+// threads after every partial is visible.  All loads of a batch are issued
+// before any add, so the pass costs a few L2 round trips.
 __device__ void finalize_cta(const double* partial, int n_parts, int n_grid,
                              const float* S, int64_t d_in, int dev_err, double* err,
                              int32_t* best_idx, float* s_best, double* e_s, int* best_s) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    for (int a = warp; a < n_grid; a += kThreads / 32) {
-        double s = 0.0;
-        for (int c = lane; c < n_parts; c += 32)
-            s += __ldcg(partial + (int64_t)c * n_grid + a);
+    constexpr int kWarps = kThreads / 32;
+    constexpr int kA = (kMaxGrid + kWarps - 1) / kWarps;   // alphas per warp
+    constexpr int kBatch = 8;                              // partials per lane per batch
+    double sums[kA];
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-        if (lane == 0) {
-            e_s[a] = s;
-            err[a] = s;
+    for (int i = 0; i < kA; ++i) sums[i] = 0.0;
+    for (int c0 = 0; c0 * 32 < n_parts; c0 += kBatch) {
+        double v[kA][kBatch];
+#pragma unroll
+        for (int i = 0; i < kA; ++i) {
+            const int a = warp + i * kWarps;
+#pragma unroll
+            for (int k = 0; k < kBatch; ++k) {
+                const int c = lane + 32 * (c0 + k);
+                v[i][k] = (a < n_grid && c < n_parts)
+                              ? __ldcg(partial + (int64_t)c * n_grid + a) : 0.0;
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < kA; ++i)
+#pragma unroll
+            for (int k = 0; k < kBatch; ++k)
+                if (lane + 32 * (c0 + k) < n_parts) sums[i] += v[i][k];
+    }
+#pragma unroll
+    for (int i = 0; i < kA; ++i) {
+        const int a = warp + i * kWarps;
+        double t = sums[i];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+        if (lane == 0 && a < n_grid) {
+            e_s[a] = t;
+            err[a] = t;
         }
     }
     __syncthreads();
@@ -120,9 +153,25 @@ __device__ void finalize_cta(const double* partial, int n_parts, int n_grid,
     }
     __syncthreads();
     if (s_best) {
+        // S rows and s_best are 16-byte aligned (d_in % 32 == 0)
         const int b = *best_s;
-        for (int64_t j = tid; j < d_in; j += kThreads)
-            s_best[j] = b >= 0 ? __ldcg(S + (int64_t)b * d_in + j) : __int_as_float(0x7fc00000);
+        const float4* src = reinterpret_cast<const float4*>(S + (int64_t)(b >= 0 ? b : 0) * d_in);
+        float4* dst = reinterpret_cast<float4*>(s_best);
+        const int64_t n4 = d_in / 4;
+        const float nan = __int_as_float(0x7fc00000);
+        for (int64_t j0 = tid; j0 < n4; j0 += 4 * kThreads) {
+            float4 v[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int64_t j = j0 + (int64_t)k * kThreads;
+                v[k] = (j < n4 && b >= 0) ? __ldcg(src + j) : make_float4(nan, nan, nan, nan);
+            }
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int64_t j = j0 + (int64_t)k * kThreads;
+                if (j < n4) dst[j] = v[k];
+            }
+        }
     }
 }
 
@@ -162,44 +211,49 @@ __device__ __forceinline__ void row_scale(float m, float* qs, float* rq, bool* i
     *rq = rcp_approx(*qs);
 }
 
-// Pass 2 of one row: codes from the reciprocal of q_scale and squared
-// weighted errors into two independent accumulators.  The packed fp32x2
-// instructions run on one of the two FMA sub-pipes only, scalar ones on
-// either: half of the work per pair is issued packed (the residual d and
-// the accumulation) and half scalar (the rounding t, q and the weighting e),
-// which keeps both sub-pipes busy for the fewest issue slots.  kClamp
-// handles a q_scale that is zero, fp16-subnormal or held at 65504 (codes
-// beyond +-7 are clamped, a zero scale gives code 0).
+// Pass 2 of a lane's two rows for one alpha: codes (no clamp when the whole
+// warp's rows are known to stay in range), residuals d = ws - q * q_scale,
+// and sum over the lane's channels of tau2 * (d_r0^2 + d_r1^2).  With kClamp
+// a row whose q_scale is zero or NaN uses a zero reciprocal (all codes 0,
+// d = ws) and its NaN/inf propagates into the sum by itself.
 template <bool kClamp, int L>
-__device__ __forceinline__ float2 row_errors(const float2* ws, const float4* Ta, int l,
-                                             float qs, float rq) {
-    if (kClamp && !(qs > 0.f)) rq = 0.f;
-    const float2 nqs2 = f2(-qs, -qs);
+__device__ __forceinline__ float2 rows_errors(const float2* ws0, const float2* ws1,
+                                              const float4* T2, int l, float qs0, float rq0,
+                                              float qs1, float rq1) {
+    if (kClamp && !(qs0 > 0.f)) rq0 = 0.f;
+    if (kClamp && !(qs1 > 0.f)) rq1 = 0.f;
+    const float2 nqs0 = f2(-qs0, -qs0), nqs1 = f2(-qs1, -qs1);
     float2 acc2[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-        const float4 tv = Ta[k * L + l];
+        const float4 tv = T2[k * L + l];
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
             const int i = 2 * k + j;
-            float tx = __fmaf_rn(ws[i].x, rq, kRoundMagic);
-            float ty = __fmaf_rn(ws[i].y, rq, kRoundMagic);
+            float t0x = __fmaf_rn(ws0[i].x, rq0, kRoundMagic);
+            float t0y = __fmaf_rn(ws0[i].y, rq0, kRoundMagic);
+            float t1x = __fmaf_rn(ws1[i].x, rq1, kRoundMagic);
+            float t1y = __fmaf_rn(ws1[i].y, rq1, kRoundMagic);
             if (kClamp) {
-                tx = fminf(fmaxf(tx, kRoundMagic - 7.f), kRoundMagic + 7.f);
-                ty = fminf(fmaxf(ty, kRoundMagic - 7.f), kRoundMagic + 7.f);
+                t0x = fminf(fmaxf(t0x, kRoundMagic - 7.f), kRoundMagic + 7.f);
+                t0y = fminf(fmaxf(t0y, kRoundMagic - 7.f), kRoundMagic + 7.f);
+                t1x = fminf(fmaxf(t1x, kRoundMagic - 7.f), kRoundMagic + 7.f);
+                t1y = fminf(fmaxf(t1y, kRoundMagic - 7.f), kRoundMagic + 7.f);
             }
-            const float2 q = f2(__fadd_rn(tx, -kRoundMagic), __fadd_rn(ty, -kRoundMagic));
-            const float2 d = __ffma2_rn(q, nqs2, ws[i]);
-            const float2 e = j ? f2(__fmul_rn(d.x, tv.z), __fmul_rn(d.y, tv.w))
-                               : f2(__fmul_rn(d.x, tv.x), __fmul_rn(d.y, tv.y));
-            acc2[j] = __ffma2_rn(e, e, acc2[j]);
+            const float2 q0 = f2(__fadd_rn(t0x, -kRoundMagic), __fadd_rn(t0y, -kRoundMagic));
+            const float2 q1 = f2(__fadd_rn(t1x, -kRoundMagic), __fadd_rn(t1y, -kRoundMagic));
+            const float2 d0 = __ffma2_rn(q0, nqs0, ws0[i]);
+            const float2 d1 = __ffma2_rn(q1, nqs1, ws1[i]);
+            float2 sq = __fmul2_rn(d0, d0);
+            sq = __ffma2_rn(d1, d1, sq);
+            acc2[j] = __ffma2_rn(j ? f2(tv.z, tv.w) : f2(tv.x, tv.y), sq, acc2[j]);
         }
     }
     return __fadd2_rn(acc2[0], acc2[1]);
 }
 
 template <int L, bool kFp32>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, 1)
 search_kernel(const __grid_constant__ SearchParams p) {
     constexpr int G = 16 * L;                    // group size
     constexpr int RPW = 2 * 32 / L;              // rows per warp (two per lane)
@@ -240,8 +294,11 @@ search_kernel(const __grid_constant__ SearchParams p) {
         int seg, grp, rb;
         decode(u, &seg, &grp, &rb);
         mbar_arrive_expect_tx(&full[stage], kUnitBytes);
-        tma_load_2d(stage_base + stage * kUnitBytes, &p.tmap[seg], grp * G, rb * R,
-                    &full[stage]);
+        // R rows in boxes of at most kMaxBoxRows (R = 512 for g = 32)
+#pragma unroll
+        for (int b = 0; b * kMaxBoxRows < R; ++b)
+            tma_load_2d(stage_base + stage * kUnitBytes + b * kMaxBoxRows * G * 2, &p.tmap[seg],
+                        grp * G, rb * R + b * kMaxBoxRows, &full[stage]);
         ++issued[stage];
     };
 
@@ -292,7 +349,7 @@ search_kernel(const __grid_constant__ SearchParams p) {
         if (grp != cur_grp) {   // uniform: every thread walks the same units
             __syncthreads();
             const float* Sg = p.S + (int64_t)grp * G;
-            const float* Tg = p.tau + (int64_t)grp * G;
+            const float* Tg = p.tau2 + (int64_t)grp * G;
             for (int i = tid; i < p.n_grid * G; i += kThreads) {
                 const int a = i / G, c = i % G;
                 const int slot = table_slot<L>(c);
@@ -352,11 +409,9 @@ search_kernel(const __grid_constant__ SearchParams p) {
             row_scale<L, kFp32>(m1, &qs1, &rq1, &in1);
             float2 e;
             if (__all_sync(0xffffffffu, in0 & in1)) {
-                e = __fadd2_rn(row_errors<false, L>(ws[0], Ta, l, qs0, rq0),
-                               row_errors<false, L>(ws[1], Ta, l, qs1, rq1));
+                e = rows_errors<false, L>(ws[0], ws[1], Ta, l, qs0, rq0, qs1, rq1);
             } else {   // some row has an fp16-subnormal, overflowing, zero or NaN scale
-                e = __fadd2_rn(row_errors<true, L>(ws[0], Ta, l, qs0, rq0),
-                               row_errors<true, L>(ws[1], Ta, l, qs1, rq1));
+                e = rows_errors<true, L>(ws[0], ws[1], Ta, l, qs0, rq0, qs1, rq1);
             }
             acc[a * kThreads + tid] += e.x + e.y;
         }
@@ -406,14 +461,21 @@ search_kernel(const __grid_constant__ SearchParams p) {
 
 // ---- scale table: s_i[j] = max(x_j, 1e-4)^alpha_i / sqrt(max_j * min_j)
 
-__device__ __forceinline__ double table_pow(const float* x, int64_t j, double alpha) {
-    return pow((double)fmaxf(x[j], 1e-4f), alpha);
+__device__ __forceinline__ double table_pow(float xj, double alpha) {
+    return pow((double)fmaxf(xj, 1e-4f), alpha);
 }
 
+// Every CTA reduces max_j and min_j of max(x_j, 1e-4) over all channels (x
+// is at most a few tens of KB and stays in L2): pow(., alpha) is monotonic
+// for alpha >= 0 and its fp64 error is far below the spacing of pow at
+// distinct fp32 arguments, so pow(x_max, alpha) and pow(x_min, alpha) are
+// exactly the largest and smallest entries of the row.  The CTA then writes
+// its slice of channels for its alpha.
 __global__ void __launch_bounds__(256)
-table_minmax_kernel(const float* __restrict__ x, int64_t d_in, int n_grid, int64_t slice,
-                    double* __restrict__ part, int* __restrict__ dev_words) {
-    __shared__ double red_mx[8], red_mn[8];
+table_kernel(const float* __restrict__ x, int64_t d_in, int n_grid, int64_t slice,
+             float* __restrict__ S, float* __restrict__ T, int kind,
+             int* __restrict__ dev_words) {
+    __shared__ float red_mx[8], red_mn[8];
     pdl_launch_dependents();
     const int a = blockIdx.y;
     const int sl = blockIdx.x;
@@ -421,54 +483,41 @@ table_minmax_kernel(const float* __restrict__ x, int64_t d_in, int n_grid, int64
         dev_words[0] = 0;
         dev_words[1] = 0;
     }
-    const double alpha = __ddiv_rn((double)a, (double)n_grid);
-    double mx = 0.0, mn = __longlong_as_double(0x7ff0000000000000ll);
-    const int64_t j0 = (int64_t)sl * slice, j1 = min(d_in, j0 + slice);
-    for (int64_t j = j0 + threadIdx.x; j < j1; j += blockDim.x) {
-        const double sd = table_pow(x, j, alpha);
-        mx = fmax(mx, sd);
-        mn = fmin(mn, sd);
+    float mx = 0.f, mn = __int_as_float(0x7f800000);
+    for (int64_t j = threadIdx.x; j < d_in; j += blockDim.x) {
+        const float v = fmaxf(x[j], 1e-4f);
+        mx = fmaxf(mx, v);
+        mn = fminf(mn, v);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
-        mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        mn = fmin(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
     }
     if ((threadIdx.x & 31) == 0) {
         red_mx[threadIdx.x >> 5] = mx;
         red_mn[threadIdx.x >> 5] = mn;
     }
     __syncthreads();
-    if (threadIdx.x == 0) {
-        for (int k = 1; k < (int)(blockDim.x >> 5); ++k) {
-            mx = fmax(mx, red_mx[k]);
-            mn = fmin(mn, red_mn[k]);
-        }
-        part[((int64_t)a * gridDim.x + sl) * 2 + 0] = fmax(mx, red_mx[0]);
-        part[((int64_t)a * gridDim.x + sl) * 2 + 1] = fmin(mn, red_mn[0]);
+    for (int k = 0; k < (int)(blockDim.x >> 5); ++k) {
+        mx = fmaxf(mx, red_mx[k]);
+        mn = fminf(mn, red_mn[k]);
     }
-}
-
-__global__ void __launch_bounds__(256)
-table_write_kernel(const float* __restrict__ x, int64_t d_in, int n_grid, int64_t slice,
-                   const double* __restrict__ part, float* __restrict__ S,
-                   float* __restrict__ tau, int write_inverse) {
-    pdl_launch_dependents();
-    pdl_wait();
-    const int a = blockIdx.y;
-    const int sl = blockIdx.x;
-    double mx = 0.0, mn = __longlong_as_double(0x7ff0000000000000ll);
-    for (int k = 0; k < (int)gridDim.x; ++k) {   // max and min are order-independent
-        mx = fmax(mx, __ldcg(part + ((int64_t)a * gridDim.x + k) * 2 + 0));
-        mn = fmin(mn, __ldcg(part + ((int64_t)a * gridDim.x + k) * 2 + 1));
-    }
-    const double norm = __dsqrt_rn(__dmul_rn(mx, mn));
     const double alpha = __ddiv_rn((double)a, (double)n_grid);
+    const double norm = __dsqrt_rn(__dmul_rn(table_pow(mx, alpha), table_pow(mn, alpha)));
     const int64_t j0 = (int64_t)sl * slice, j1 = min(d_in, j0 + slice);
     for (int64_t j = j0 + threadIdx.x; j < j1; j += blockDim.x) {
-        const float s = __double2float_rn(__ddiv_rn(table_pow(x, j, alpha), norm));
+        const float xj = x[j];
+        const float s = __double2float_rn(__ddiv_rn(table_pow(xj, alpha), norm));
         S[(int64_t)a * d_in + j] = s;
-        tau[(int64_t)a * d_in + j] = write_inverse ? __frcp_rn(s) : __fdiv_rn(x[j], s);
+        float t;
+        if (kind == kTableInverse) {
+            t = __frcp_rn(s);
+        } else {
+            const double q = __ddiv_rn((double)xj, (double)s);
+            t = __double2float_rn(q * q);
+        }
+        T[(int64_t)a * d_in + j] = t;
     }
 }
 
@@ -486,19 +535,19 @@ finalize_kernel(const double* __restrict__ partial, int n_parts, int n_grid,
 
 struct SearchWs {
     float* S;
-    float* tau;
+    float* tau2;
     double* partial;
     int* dev_words;
 };
 
-size_t max_search_ctas() { return 1024; }
+size_t max_search_ctas() { return kMaxParts; }
 
 SearchWs carve_search_ws(void* ws, int64_t d_in, int n_grid) {
     char* p = static_cast<char*>(ws);
     SearchWs w;
     const size_t tab = align_up((size_t)n_grid * (size_t)d_in * sizeof(float), kWsAlign);
     w.S = reinterpret_cast<float*>(p);
-    w.tau = reinterpret_cast<float*>(p + tab);
+    w.tau2 = reinterpret_cast<float*>(p + tab);
     w.partial = reinterpret_cast<double*>(p + 2 * tab);
     w.dev_words = reinterpret_cast<int*>(
         p + 2 * tab + align_up(max_search_ctas() * kMaxGrid * sizeof(double), kWsAlign));
@@ -547,20 +596,17 @@ size_t scale_search_workspace(int64_t d_in, int group_size, int n_grid) {
 }
 
 cudaError_t launch_scale_table(const float* x_mean, int64_t d_in, int n_grid, float* S,
-                               float* tau, double* part, int* dev_words, int num_sms,
-                               cudaStream_t stream, bool write_inverse) {
+                               float* T, int* dev_words, int num_sms, cudaStream_t stream,
+                               TableKind kind) {
     int64_t slices = (2 * (int64_t)num_sms + n_grid - 1) / n_grid;
     slices = std::min<int64_t>(slices, (d_in + 63) / 64);
     slices = std::max<int64_t>(1, std::min<int64_t>(slices, kMaxTableSlices));
     const int64_t slice = (d_in + slices - 1) / slices;
     slices = (d_in + slice - 1) / slice;
     const dim3 grid((unsigned)slices, (unsigned)n_grid);
-    table_minmax_kernel<<<grid, 256, 0, stream>>>(x_mean, d_in, n_grid, slice, part,
-                                                  dev_words);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    return launch_pdl(table_write_kernel, grid, dim3(256), 0, stream, x_mean, d_in, n_grid,
-                      slice, (const double*)part, S, tau, (int)write_inverse);
+    table_kernel<<<grid, 256, 0, stream>>>(x_mean, d_in, n_grid, slice, S, T, (int)kind,
+                                           dev_words);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_finalize(const double* partial, int n_parts, int n_grid, const float* S,
@@ -591,7 +637,7 @@ awq_status launch_scale_search(int n_seg, const void* const* W, const int64_t* d
     p.flags = flags;
     p.d_in = d_in;
     p.S = w.S;
-    p.tau = w.tau;
+    p.tau2 = w.tau2;
     p.partial = w.partial;
     p.dev_words = w.dev_words;
     p.err = err;
@@ -602,7 +648,8 @@ awq_status launch_scale_search(int n_seg, const void* const* W, const int64_t* d
     for (int k = 0; k < n_seg; ++k) {
         const cuuint64_t gdim[2] = {(cuuint64_t)d_in, (cuuint64_t)d_out[k]};
         const cuuint64_t gstride[1] = {(cuuint64_t)d_in * 2};
-        const cuuint32_t box[2] = {(cuuint32_t)group_size, (cuuint32_t)R};
+        const cuuint32_t box[2] = {(cuuint32_t)group_size,
+                                   (cuuint32_t)std::min(R, kMaxBoxRows)};
         const cuuint32_t estride[2] = {1, 1};
         CUresult r = encode(&p.tmap[k], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
                             const_cast<void*>(W[k]), gdim, gstride, box, estride,
@@ -618,14 +665,14 @@ awq_status launch_scale_search(int n_seg, const void* const* W, const int64_t* d
     p.n_units = units;
 
     const size_t smem = search_smem_bytes(group_size, n_grid);
-    int per_sm = 2;
+    int per_sm = 1;
     while (per_sm > 1 && (size_t)per_sm * (smem + 1024) > dev.max_smem_per_sm) --per_sm;
     int64_t grid = (int64_t)dev.num_sms * per_sm;
     if (grid > units) grid = units;
     if (grid > (int64_t)max_search_ctas()) grid = (int64_t)max_search_ctas();
 
-    if (launch_scale_table(x_mean, d_in, n_grid, w.S, w.tau, w.partial, w.dev_words,
-                           dev.num_sms, stream) != cudaSuccess)
+    if (launch_scale_table(x_mean, d_in, n_grid, w.S, w.tau2, w.dev_words, dev.num_sms,
+                           stream, kTableTauSq) != cudaSuccess)
         return AWQ_ERR_CUDA;
     const cudaError_t e = (flags & AWQ_SCALE_FP32)
                               ? launch_search<true>(L, p, (int)grid, smem, stream)
