@@ -49,7 +49,20 @@ sys.path.insert(0, ROOT)
 
 METRIC = "AWQ search+pack Gparam/s per layer"
 UNIT = "Gparam/s"
-FMA_OPS_PER_PAIR = 6          # FMA-pipe lane ops per (weight, alpha) pair
+# Algorithmic work of the search per (weight, alpha) pair, as the scope of the
+# path counts it (an FMA counts once): multiply w*s, |.| and max, divide by
+# q_scale, round, two clamps, multiply q*q_scale, divide by s, subtract,
+# multiply by x, square-accumulate.
+ALG_OPS_PER_PAIR = 11
+# FMA-pipe lane operations the search kernel actually executes per pair
+# (w*s, the rounding addition and its removal, the residual, the weighted
+# square-accumulate shared by a lane's two rows) -- reported beside it.
+FMA_OPS_PER_PAIR = 5
+# dram__bytes_read.sum + dram__bytes_write.sum of one launch of the dominant
+# kernel from the committed ncu captures (profiles/), for the kernels as they
+# stand; None where no capture of the current kernel exists.
+NCU_TRAFFIC = {"q_proj_4096x4096": 34249472,          # search_kernel<8,0>
+               "down_proj_output_error": 3105129984}  # oe_gemm_kernel, per alpha
 FP32_LANES_PER_SM = 128
 DEFAULT_STEPS = {"single_linear_256x512": 1000, "q_proj_4096x4096": 1000,
                  "qwen3_8b_block": 100, "down_proj_output_error": 10,
@@ -360,7 +373,11 @@ def run_ours(a):
                 "kernel": "awq_output_error (scale table + per alpha: dW builder + tcgen05 "
                           "GEMM with fused square-sum + finalize)",
                 "achieved": achieved / 1e12, "peak": peak_t / 1e12, "unit": "TFLOP/s",
-                "frac": achieved / peak_t, "traffic": None,
+                "frac": achieved / peak_t,
+                "traffic": (NCU_TRAFFIC[a.workload] * n_grid
+                            if a.workload in NCU_TRAFFIC else None),
+                "traffic_basis": "DRAM bytes of the n_grid GEMM launches of one call "
+                                 "(ncu, per launch x n_grid)",
                 "flops_per_step": flops, "executed_flops_per_step": 2 * flops,
                 "peak_basis": "measured bf16 dense GEMM, sustained (fp16 has the same "
                               "nominal tensor rate); algorithmic FLOPs 2*T*d_out*d_in per "
@@ -370,17 +387,22 @@ def run_ours(a):
                                    "executed_TFLOP/s": 2 * achieved / 1e12}
     else:
         peak_ops = n_sms * FP32_LANES_PER_SM * clk_mhz * 1e6          # lane-ops / s
-        ops = params * n_grid * FMA_OPS_PER_PAIR
+        ops = params * n_grid * ALG_OPS_PER_PAIR
         achieved = ops / (ms_search * 1e-3)
+        executed = params * n_grid * FMA_OPS_PER_PAIR / (ms_search * 1e-3)
         roof = {"bound": "alu",
-                "kernel": "awq_scale_search (scale table + fused search + finalize)",
-                "achieved": achieved / 1e12, "peak": peak_ops / 1e12, "unit": "Tlane-op/s",
-                "frac": achieved / peak_ops, "traffic": None,
-                "ops_per_weight_alpha": FMA_OPS_PER_PAIR,
+                "kernel": "awq_scale_search (table kernel + fused search kernel with finalize)",
+                "achieved": achieved / 1e12, "peak": peak_ops / 1e12, "unit": "Top/s",
+                "frac": achieved / peak_ops,
+                "traffic": NCU_TRAFFIC.get(a.workload),
+                "ops_per_weight_alpha": ALG_OPS_PER_PAIR,
+                "executed_fma_pipe_ops_per_weight_alpha": FMA_OPS_PER_PAIR,
+                "executed_frac": executed / peak_ops,
                 "peak_basis": f"{n_sms} SMs x {FP32_LANES_PER_SM} FP32 lanes x "
                               f"{clk_mhz:.0f} MHz (median SM clock sampled in the timed "
                               f"region)"}
-        kernels["scale_search"] = {"ms": ms_search, "Tlane-op/s": achieved / 1e12,
+        kernels["scale_search"] = {"ms": ms_search, "Top/s": achieved / 1e12,
+                                   "executed_Tlane-op/s": executed / 1e12,
                                    "W_GB/s": params * 2 / (ms_search * 1e-3) / 1e9}
     if work.layers == 1:
         par = f"independent layer per rank x{world}"

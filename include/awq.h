@@ -139,8 +139,11 @@ awq_status awq_act_stats(const void *X, int64_t T, int64_t d_in, int64_t ld,
  *               infinite input), -2 if a device-side wait gave up
  *   s_best      fp32 [d_in] device output (NaN when best_idx < 0)
  *   ws          workspace of awq_workspace_size(AWQ_OP_SCALE_SEARCH, ...)
- * err is evaluated in fp32 per row and accumulated in fp64 in a fixed order;
- * it matches the exact score of the same decisions to about 1e-6 relative.
+ * Each term is evaluated in fp32 as (ws - q * q_scale)^2 * (x_mean/s_i)^2,
+ * summed in fp32 over a thread's share of 8 units and in fp64 in a fixed
+ * order after that, so results are deterministic; against the exact score
+ * of the same decisions the relative difference is about 3e-8 on a
+ * 4096 x 4096 layer (the tested bar is 1e-5).
  */
 #define AWQ_MAX_SEGMENTS 8
 awq_status awq_scale_search(int n_seg, const void *const *W,
