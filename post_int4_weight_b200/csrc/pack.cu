@@ -115,6 +115,8 @@ pack_kernel(const uint4* __restrict__ W, int64_t d_out, int64_t d_in,
     int* bad_tile = reinterpret_cast<int*>(qr_tile + KG * kRowStride);  // [KG][kRowStride]
     int* slow_blk = bad_tile + KG * kRowStride;                          // [KG][kBlocks32]
 
+    // a programmatic dependent launch: W and s may come from the kernel before
+    pdl_wait();
     const int tid = threadIdx.x;
     const int64_t col0 = (int64_t)blockIdx.x * kPackCols;
     const int64_t row0 = (int64_t)blockIdx.y * kPackRows;
@@ -147,6 +149,7 @@ pack_kernel(const uint4* __restrict__ W, int64_t d_out, int64_t d_in,
         sabs_tile[sabs_slot(tid)] = fabsf(sv);
     }
     if (tid < KG * kBlocks32) slow_blk[tid] = 0;
+    pdl_launch_dependents();   // the tile is read; the next kernel may start launching
     __syncthreads();
 
     // ---- phase 2: group scale of every (row, group), two threads each.
@@ -253,10 +256,9 @@ cudaError_t launch_pack_G(const void* W, int64_t d_out, int64_t d_in, const floa
     }
     dim3 grid((unsigned)((d_in + kPackCols - 1) / kPackCols),
               (unsigned)((d_out + kPackRows - 1) / kPackRows));
-    pack_kernel<G><<<grid, kPackThreads, smem, stream>>>(
-        static_cast<const uint4*>(W), d_out, d_in, s, zero_point, qweight,
-        static_cast<__half*>(scales), qzeros);
-    return cudaGetLastError();
+    return launch_pdl(pack_kernel<G>, grid, dim3(kPackThreads), smem, stream,
+                      static_cast<const uint4*>(W), d_out, d_in, s, zero_point, qweight,
+                      static_cast<__half*>(scales), qzeros);
 }
 
 }  // namespace

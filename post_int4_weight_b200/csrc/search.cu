@@ -428,6 +428,10 @@ search_kernel(const __grid_constant__ SearchParams p) {
         }
     }
 
+    // the next kernel (e.g. the pack, which waits for this grid to finish)
+    // may start launching while the partials are reduced
+    pdl_launch_dependents();
+
     // drain: never leave the CTA while a TMA copy may still write its smem.
     // The n-th load into a stage completes that barrier's phase n.
     if (tid == 0) {
@@ -476,6 +480,10 @@ table_kernel(const float* __restrict__ x, int64_t d_in, int n_grid, int64_t slic
              float* __restrict__ S, float* __restrict__ T, int kind,
              int* __restrict__ dev_words) {
     __shared__ float red_mx[8], red_mn[8];
+    // Wait for the kernel before (x may come from it) before letting the
+    // search kernel launch: the search reads W before its own wait, so W
+    // must already be final when it starts.
+    pdl_wait();
     pdl_launch_dependents();
     const int a = blockIdx.y;
     const int sl = blockIdx.x;
@@ -604,9 +612,8 @@ cudaError_t launch_scale_table(const float* x_mean, int64_t d_in, int n_grid, fl
     const int64_t slice = (d_in + slices - 1) / slices;
     slices = (d_in + slice - 1) / slice;
     const dim3 grid((unsigned)slices, (unsigned)n_grid);
-    table_kernel<<<grid, 256, 0, stream>>>(x_mean, d_in, n_grid, slice, S, T, (int)kind,
-                                           dev_words);
-    return cudaGetLastError();
+    return launch_pdl(table_kernel, grid, dim3(256), 0, stream, x_mean, d_in, n_grid, slice, S,
+                      T, (int)kind, dev_words);
 }
 
 cudaError_t launch_finalize(const double* partial, int n_parts, int n_grid, const float* S,

@@ -101,6 +101,8 @@ stats_kernel(const uint4* __restrict__ X, int64_t T, int64_t d_in, int64_t ld_ch
     cg::cluster_group cluster = cg::this_cluster();
     const int rank = (int)cluster.block_rank();
 
+    // a programmatic dependent launch: X may be written by the kernel before
+    pdl_wait();
     const int tid = threadIdx.x;
     const int cx = tid % kChunks;
     const int ry = tid / kChunks;
@@ -142,6 +144,7 @@ stats_kernel(const uint4* __restrict__ X, int64_t T, int64_t d_in, int64_t ld_ch
     }
     for (int64_t r = base + sub; r < r1; r += kRowLanes)
         if (active) add_halves(__ldg(p + r * ld_chunks), acc, hmax);
+    pdl_launch_dependents();   // X is read; the next kernel may start launching
     flush(acc, hmax, cx, red, fred);
     __syncthreads();
     if (rank != 0 && tid < kChunks * 8) {
@@ -181,9 +184,8 @@ cudaError_t launch_act_stats(const void* X, int64_t T, int64_t d_in, int64_t ld,
     (void)ws;
     const int64_t col_blocks = (d_in / 8 + kChunks - 1) / kChunks;
     dim3 grid((unsigned)col_blocks, kCluster);
-    stats_kernel<<<grid, kChunks * kRowLanes, 0, stream>>>(static_cast<const uint4*>(X), T,
-                                                            d_in, ld / 8, x_mean);
-    return cudaGetLastError();
+    return launch_pdl(stats_kernel, grid, dim3(kChunks * kRowLanes), 0, stream,
+                      static_cast<const uint4*>(X), T, d_in, ld / 8, x_mean);
 }
 
 }  // namespace awq
