@@ -29,7 +29,9 @@
 // age priority and the later one ends alone on its SM.
 //
 // Register-level formulation of one (weight, alpha) pair: 5 FMA-pipe ops and
-// one max, mostly packed fp32x2 instructions (sm_100).  Each lane holds the
+// one max.  Packed fp32x2 instructions (sm_100) run on the FMA pipe's heavy
+// half only and scalar ones on either half, so the work is split between the
+// two kinds to keep both halves busy while issuing few instructions.  Each lane holds the
 // same 16 channels of two rows r0, r1:
 //   ws = w * s                         (exact fp32 product, as the method)
 //   m  = max(m, |ws|)                  (then shuffled across the L lanes)
@@ -223,6 +225,8 @@ __device__ __forceinline__ float2 rows_errors(const float2* ws0, const float2* w
     if (kClamp && !(qs0 > 0.f)) rq0 = 0.f;
     if (kClamp && !(qs1 > 0.f)) rq1 = 0.f;
     const float2 nqs0 = f2(-qs0, -qs0), nqs1 = f2(-qs1, -qs1);
+    const float2 rq02 = f2(rq0, rq0);
+    const float2 magic2 = f2(kRoundMagic, kRoundMagic), nmagic2 = f2(-kRoundMagic, -kRoundMagic);
     float2 acc2[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
@@ -230,17 +234,19 @@ __device__ __forceinline__ float2 rows_errors(const float2* ws0, const float2* w
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
             const int i = 2 * k + j;
-            float t0x = __fmaf_rn(ws0[i].x, rq0, kRoundMagic);
-            float t0y = __fmaf_rn(ws0[i].y, rq0, kRoundMagic);
+            // row 0 rounds with packed instructions (the FMA pipe's heavy
+            // half), row 1 with scalar ones (either half): this balance
+            // issued fastest
+            float2 t0 = __ffma2_rn(ws0[i], rq02, magic2);
             float t1x = __fmaf_rn(ws1[i].x, rq1, kRoundMagic);
             float t1y = __fmaf_rn(ws1[i].y, rq1, kRoundMagic);
             if (kClamp) {
-                t0x = fminf(fmaxf(t0x, kRoundMagic - 7.f), kRoundMagic + 7.f);
-                t0y = fminf(fmaxf(t0y, kRoundMagic - 7.f), kRoundMagic + 7.f);
+                t0 = f2(fminf(fmaxf(t0.x, kRoundMagic - 7.f), kRoundMagic + 7.f),
+                        fminf(fmaxf(t0.y, kRoundMagic - 7.f), kRoundMagic + 7.f));
                 t1x = fminf(fmaxf(t1x, kRoundMagic - 7.f), kRoundMagic + 7.f);
                 t1y = fminf(fmaxf(t1y, kRoundMagic - 7.f), kRoundMagic + 7.f);
             }
-            const float2 q0 = f2(__fadd_rn(t0x, -kRoundMagic), __fadd_rn(t0y, -kRoundMagic));
+            const float2 q0 = __fadd2_rn(t0, nmagic2);
             const float2 q1 = f2(__fadd_rn(t1x, -kRoundMagic), __fadd_rn(t1y, -kRoundMagic));
             const float2 d0 = __ffma2_rn(q0, nqs0, ws0[i]);
             const float2 d1 = __ffma2_rn(q1, nqs1, ws1[i]);
@@ -318,8 +324,6 @@ search_kernel(const __grid_constant__ SearchParams p) {
     pdl_wait();          // the scale table (and the cleared counters) are ready
     __syncthreads();
 
-    const float2 magic2 = f2(kRoundMagic, kRoundMagic);
-    const float2 nmagic2 = f2(-kRoundMagic, -kRoundMagic);
     int cur_grp = -1;
     // Once any bounded wait gives up, the CTA stops computing but keeps the
     // same barrier sequence (no thread leaves a __syncthreads behind).
