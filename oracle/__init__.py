@@ -37,7 +37,14 @@ def _load():
         lib.orc_weighted_error.argtypes = [p, i64, i64, p, p, i64, i32]
         lib.orc_weighted_error.restype = f64
         lib.orc_scale_search.argtypes = [i32, p, p, i64, p, i64, i32, i32, p, p, p]
-        lib.orc_quantize_pack.argtypes = [p, i64, i64, p, i64, i32, p, p, p]
+        lib.orc_quantize_pack.argtypes = [p, i64, i64, p, p, i64, i32, p, p, p]
+        lib.orc_clip_ratio.argtypes = [i32]
+        lib.orc_clip_ratio.restype = ctypes.c_float
+        lib.orc_fake_quant_group_clip.argtypes = [p, p, i64, i32, ctypes.c_float, p, p]
+        lib.orc_fake_quant_group_clip.restype = i32
+        lib.orc_clip_group_error.argtypes = [p, p, p, i64, i32, ctypes.c_float]
+        lib.orc_clip_group_error.restype = f64
+        lib.orc_clip_search.argtypes = [p, i64, i64, p, p, i64, i32, i32, p, p]
         lib.orc_unpack.argtypes = [p, i64, i64, p]
         lib.orc_output_error.argtypes = [p, i64, p, i64, i64, p, i64, i32, i32, p]
         _lib = lib
@@ -111,9 +118,10 @@ def scale_search(Ws, x, group_size: int = 128, n_grid: int = 20, flags: int = 0)
     return err, int(best[0]), s_best
 
 
-def quantize_pack(W, s=None, group_size: int = 128, zero_point: int = 8):
+def quantize_pack(W, s=None, group_size: int = 128, zero_point: int = 8, clip_idx=None):
     """AutoAWQ GEMM layout: (qweight int32[d_in, d_out/8],
-    scales fp16[d_in/g, d_out], qzeros int32[d_in/g, d_out/8])."""
+    scales fp16[d_in/g, d_out], qzeros int32[d_in/g, d_out/8]).
+    clip_idx: optional uint8 [d_out, d_in/g] clip ratio indices."""
     W = _f16(W)
     d_out, d_in = W.shape
     G = d_in // group_size
@@ -121,11 +129,53 @@ def quantize_pack(W, s=None, group_size: int = 128, zero_point: int = 8):
     scales = np.empty((G, d_out), np.float16)
     qzeros = np.empty((G, d_out // 8), np.int32)
     s_arr = None if s is None else _f32(s)
+    c_arr = None if clip_idx is None else np.ascontiguousarray(clip_idx, dtype=np.uint8)
+    if c_arr is not None and c_arr.shape != (d_out, G):
+        raise ValueError("clip_idx must be [d_out, d_in / group_size]")
     _load().orc_quantize_pack(_ptr(W), d_out, d_in,
                               None if s_arr is None else _ptr(s_arr),
+                              None if c_arr is None else _ptr(c_arr),
                               group_size, zero_point, _ptr(qweight),
                               _ptr(scales), _ptr(qzeros))
     return qweight, scales, qzeros
+
+
+def clip_ratio(i: int) -> float:
+    """Clip ratio of grid index i: (20 - i) / 20 rounded to fp32."""
+    return float(_load().orc_clip_ratio(int(i)))
+
+
+def fake_quant_group_clip(w, s, c: float, flags: int = 0):
+    """Codes and group scale of one group with the range shrunk to c*max|ws|."""
+    w, s = _f32(w), _f32(s)
+    q = np.empty(w.shape[0], np.int8)
+    qs = np.empty(1, np.float32)
+    _load().orc_fake_quant_group_clip(_ptr(w), _ptr(s), w.shape[0], flags,
+                                      ctypes.c_float(c), _ptr(q), _ptr(qs))
+    return q, float(qs[0])
+
+
+def clip_group_error(w, s, x, c: float, flags: int = 0) -> float:
+    """Weighted error of one group at clip ratio c (fp64)."""
+    w, s, x = _f32(w), _f32(s), _f32(x)
+    return float(_load().orc_clip_group_error(_ptr(w), _ptr(s), _ptr(x), w.shape[0],
+                                              flags, ctypes.c_float(c)))
+
+
+def clip_search(W, x, s=None, group_size: int = 128, n_clip: int = 10, flags: int = 0):
+    """Per (row, group) clip ratio index (uint8 [d_out, d_in/g]) and the
+    totals (error without clipping, error with the chosen ratios)."""
+    W = _f16(W)
+    x = _f32(x)
+    d_out, d_in = W.shape
+    G = d_in // group_size
+    idx = np.empty((d_out, G), np.uint8)
+    err = np.empty(2, np.float64)
+    s_arr = None if s is None else _f32(s)
+    _load().orc_clip_search(_ptr(W), d_out, d_in, _ptr(x),
+                            None if s_arr is None else _ptr(s_arr), group_size, n_clip,
+                            flags, _ptr(idx), _ptr(err))
+    return idx, err
 
 
 def unpack(qweight, d_out: int) -> np.ndarray:

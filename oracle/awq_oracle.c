@@ -14,6 +14,11 @@
  *        code" and "Quantization, storage and packing".
  *   [P4] "Weight-Only Quantization: GPTQ and AWQ", section 4 "Tiny example"
  *        and sections 6-9 "Under the hood: the packed format".
+ *   Clip search: [P3] "The pipeline end to end", step 5 (an optional search
+ *        of a clipping range per output channel that shrinks the
+ *        quantisation range); [P5] "AWQ, Reproduced" (the paper also clips
+ *        the weight range).  The pages give no formula; the reading used
+ *        here is listed in the design doc.
  *
  * Precision (readings are listed in the design doc):
  *   - every decision that produces an integer (a code, the group scale, the
@@ -196,6 +201,123 @@ double orc_weighted_error(const uint16_t *W, int64_t d_out, int64_t d_in,
     return total;
 }
 
+/* ------------------------------------------------------------- clipping --
+ * Clip ratio i of the grid: c_i = (20 - i) / 20 rounded to fp32, so c_0 = 1
+ * (no clipping) and each step shrinks the range by 5% of the group maximum.
+ */
+#define ORC_CLIP_DEN 20
+
+float orc_clip_ratio(int i)
+{
+    return (float)((double)(ORC_CLIP_DEN - i) / (double)ORC_CLIP_DEN);
+}
+
+/* The group fake-quantisation with the range shrunk to c * max|w s|:
+ *   m_c = fl32(c * max|ws|),  q_scale = fp16_rne(fl32(m_c / 7)),
+ *   q = clamp(rint(ws / q_scale), -7, 7)
+ * (values beyond the shrunk range saturate at +-7).  With c = 1 every
+ * operation is the one of orc_fake_quant_group. */
+int orc_fake_quant_group_clip(const float *w, const float *s, int64_t n, int flags,
+                              float c, int8_t *q, float *q_scale)
+{
+    float m = 0.0f;
+    int nonfinite = 0;
+    for (int64_t j = 0; j < n; ++j) {
+        float ws = w[j] * s[j];
+        if (!isfinite(ws)) nonfinite = 1;
+        float a = fabsf(ws);
+        if (a > m) m = a;
+    }
+    if (nonfinite) {
+        for (int64_t j = 0; j < n; ++j) q[j] = 0;
+        *q_scale = NAN;
+        return 1;
+    }
+    float mc = m * c;
+    float qs = mc / 7.0f;
+    if (!(flags & ORC_SCALE_FP32)) {
+        qs = h2f(f2h(qs));
+        if (isinf(qs)) qs = 65504.0f;
+    }
+    for (int64_t j = 0; j < n; ++j) {
+        if (qs == 0.0f) { q[j] = 0; continue; }
+        float ws = w[j] * s[j];
+        float r = rintf(ws / qs);
+        if (r > 7.0f) r = 7.0f;
+        if (r < -7.0f) r = -7.0f;
+        q[j] = (int8_t)r;
+    }
+    *q_scale = qs;
+    return 0;
+}
+
+/* Weighted error of one group (n weights) at clip ratio c, in fp64:
+ * sum_j ((w_j - q_j q_scale / s_j) x_j)^2; NaN for a non-finite group. */
+double orc_clip_group_error(const float *w, const float *s, const float *x, int64_t n,
+                            int flags, float c)
+{
+    int8_t q[n];
+    float qs;
+    if (orc_fake_quant_group_clip(w, s, n, flags, c, q, &qs)) return NAN;
+    double acc = 0.0;
+    for (int64_t j = 0; j < n; ++j) {
+        double what = (double)q[j] * (double)qs / (double)s[j];
+        double e = ((double)w[j] - what) * (double)x[j];
+        acc += e * e;
+    }
+    return acc;
+}
+
+/* Clip search at a fixed scale s (normally the scale search's s_best):
+ * for every row r and group k, the first ratio index i < n_clip with the
+ * smallest weighted error of that group wins (strict '<').
+ *   clip_idx[r * G + k]  the chosen index (0 for a non-finite group)
+ *   err[0]               total error with no clipping (index 0 everywhere)
+ *   err[1]               total error with the chosen indices
+ * Totals are summed per row, then over rows in order.  s == NULL: s = 1. */
+void orc_clip_search(const uint16_t *W, int64_t d_out, int64_t d_in, const float *x,
+                     const float *s, int64_t g, int n_clip, int flags,
+                     uint8_t *clip_idx, double *err)
+{
+    int64_t G = d_in / g;
+    double *row0 = (double *)malloc((size_t)d_out * sizeof(double));
+    double *row1 = (double *)malloc((size_t)d_out * sizeof(double));
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < d_out; ++r) {
+        float w[g], ones[g];
+        for (int64_t j = 0; j < g; ++j) ones[j] = 1.0f;
+        double a0 = 0.0, a1 = 0.0;
+        for (int64_t k = 0; k < G; ++k) {
+            for (int64_t j = 0; j < g; ++j) w[j] = h2f(W[r * d_in + k * g + j]);
+            const float *sk = s ? s + k * g : ones;
+            double best = orc_clip_group_error(w, sk, x + k * g, g, flags, orc_clip_ratio(0));
+            double e0 = best;
+            int b = 0;
+            for (int i = 1; i < n_clip; ++i) {
+                double e = orc_clip_group_error(w, sk, x + k * g, g, flags, orc_clip_ratio(i));
+                if (e < best) {
+                    best = e;
+                    b = i;
+                }
+            }
+            clip_idx[r * G + k] = (uint8_t)b;
+            a0 += e0;
+            a1 += best;
+        }
+        row0[r] = a0;
+        row1[r] = a1;
+    }
+    double t0 = 0.0, t1 = 0.0;
+    for (int64_t r = 0; r < d_out; ++r) {
+        t0 += row0[r];
+        t1 += row1[r];
+    }
+    err[0] = t0;
+    err[1] = t1;
+    free(row0);
+    free(row1);
+}
+
 /* ---------------------------------------------------------- scale search --
  * [P3] "The scale search as code" + [P1] "AWQ scaling": for every grid
  * index i the error of every weight segment that shares the input x is
@@ -240,14 +362,16 @@ void orc_scale_search(int n_seg, const uint16_t *const *W, const int64_t *d_out,
  *                     u[8c + order[p], j],  order = {0,2,4,6,1,3,5,7}
  *   scales[k, r]    = fp16 group scale of row r, group k
  *   qzeros[k, c]    = zero_point in all eight nibbles
- * s == NULL means s = 1 (plain round-to-nearest).  A non-finite group stores
- * code zero_point and scale NaN.
+ * s == NULL means s = 1 (plain round-to-nearest).  clip_idx (or NULL for
+ * none) gives each (row, group) a clip ratio index as in orc_clip_search.
+ * A non-finite group stores code zero_point and scale NaN.
  */
 static const int kOrder[8] = {0, 2, 4, 6, 1, 3, 5, 7};
 
 void orc_quantize_pack(const uint16_t *W, int64_t d_out, int64_t d_in,
-                       const float *s, int64_t g, int zero_point,
-                       int32_t *qweight, uint16_t *scales, int32_t *qzeros)
+                       const float *s, const uint8_t *clip_idx, int64_t g,
+                       int zero_point, int32_t *qweight, uint16_t *scales,
+                       int32_t *qzeros)
 {
     int64_t G = d_in / g, C = d_out / 8;
     uint8_t *u = (uint8_t *)malloc((size_t)d_out * (size_t)d_in);
@@ -260,7 +384,11 @@ void orc_quantize_pack(const uint16_t *W, int64_t d_out, int64_t d_in,
         for (int64_t k = 0; k < G; ++k) {
             for (int64_t j = 0; j < g; ++j) w[j] = h2f(W[r * d_in + k * g + j]);
             float qs;
-            orc_fake_quant_group(w, s ? s + k * g : ones, g, 0, q, &qs);
+            if (clip_idx)
+                orc_fake_quant_group_clip(w, s ? s + k * g : ones, g, 0,
+                                          orc_clip_ratio(clip_idx[r * G + k]), q, &qs);
+            else
+                orc_fake_quant_group(w, s ? s + k * g : ones, g, 0, q, &qs);
             scales[k * d_out + r] = isnan(qs) ? (uint16_t)0x7E00 : f2h(qs);
             for (int64_t j = 0; j < g; ++j)
                 u[r * d_in + k * g + j] = (uint8_t)(q[j] + zero_point);

@@ -343,3 +343,134 @@ def test_output_mode_token_additivity_and_scaling():
     assert np.allclose(e, e1 + e2, rtol=1e-12)
     e4 = oracle.output_error((2 * X.astype(np.float32)).astype(np.float16), W, x, g, 20)
     assert np.allclose(e4, 4 * e, rtol=1e-12)
+
+
+# ------------------------------------------------------------- clip search --
+# The pages name the clip search (pipeline step 5 of the AWQ architecture
+# page: shrink the quantisation range per output channel to cut rounding
+# error on outliers) without a formula; the reading pinned here: ratios
+# c_i = (20 - i) / 20, range c_i * max|w s|, codes saturating at +-7, the
+# same activation-weighted error, first minimum per (row, group).
+
+def test_clip_ratio_grid():
+    assert oracle.clip_ratio(0) == 1.0
+    assert oracle.clip_ratio(10) == 0.5          # exactly representable
+    for i in range(20):
+        assert oracle.clip_ratio(i) == float(np.float32((20 - i) / 20))
+
+
+def test_clip_ratio_one_is_the_unclipped_quantiser():
+    rng = np.random.default_rng(41)
+    for _ in range(100):
+        n = 128
+        w = (rng.standard_normal(n) * 0.02).astype(np.float16).astype(np.float32)
+        s = np.exp(rng.standard_normal(n)).astype(np.float32)
+        q0, qs0, _ = oracle.fake_quant_group(w, s, 0)
+        q1, qs1 = oracle.fake_quant_group_clip(w, s, 1.0, 0)
+        assert np.array_equal(q0, q1) and qs0 == qs1
+
+
+@pytest.mark.parametrize("i", [1, 3, 6, 9, 14])
+def test_clipped_codes_are_nearest_of_15_levels(i):
+    """With the range shrunk to c * max|ws|, every code is the nearest of the
+    15 levels -7..7 to the IEEE quotient (saturating beyond the range), and
+    the scale is fp16(fl32(fl32(c m) / 7))."""
+    rng = np.random.default_rng(42 + i)
+    c = np.float32(oracle.clip_ratio(i))
+    for _ in range(50):
+        n = 64
+        w = (rng.standard_normal(n) * 0.02).astype(np.float16).astype(np.float32)
+        s = np.exp(rng.standard_normal(n)).astype(np.float32)
+        q, qs = oracle.fake_quant_group_clip(w, s, float(c), 0)
+        ws = (w * s).astype(np.float32)
+        m = np.float32(np.max(np.abs(ws)))
+        assert qs == float(np.float16(np.float32(m * c) / np.float32(7)))
+        for j in range(n):
+            quot = np.float32(ws[j]) / np.float32(qs)
+            assert q[j] == _nearest_level(quot)
+
+
+def test_clip_search_never_worse_and_first_minimum():
+    rng = np.random.default_rng(43)
+    d_out, d_in, g, n_clip = 24, 256, 64, 10
+    W = (rng.standard_normal((d_out, d_in)) * 0.02).astype(np.float16)
+    W[3, 5] = np.float16(0.3)                     # a lone outlier in one group
+    x = np.exp(rng.standard_normal(d_in)).astype(np.float32)
+    s = np.exp(rng.standard_normal(d_in) * 0.5).astype(np.float32)
+    idx, err = oracle.clip_search(W, x, s, g, n_clip)
+    assert err[1] <= err[0]
+    Wf = W.astype(np.float32)
+    total0 = total1 = 0.0
+    for r in range(d_out):
+        for k in range(d_in // g):
+            sl = slice(k * g, (k + 1) * g)
+            e = [oracle.clip_group_error(Wf[r, sl], s[sl], x[sl], oracle.clip_ratio(i))
+                 for i in range(n_clip)]
+            b = int(np.argmin(e))                  # numpy argmin: first minimum
+            assert idx[r, k] == b
+            total0 += e[0]
+            total1 += e[b]
+    assert math.isclose(err[0], total0, rel_tol=1e-12)
+    assert math.isclose(err[1], total1, rel_tol=1e-12)
+    assert idx[3, 0] > 0                           # the outlier's group is clipped
+
+
+def test_clip_search_one_ratio_is_the_weighted_error():
+    rng = np.random.default_rng(44)
+    W = (rng.standard_normal((16, 256)) * 0.02).astype(np.float16)
+    x = np.exp(rng.standard_normal(256)).astype(np.float32)
+    s = np.exp(rng.standard_normal(256) * 0.5).astype(np.float32)
+    idx, err = oracle.clip_search(W, x, s, 128, 1)
+    assert not idx.any()
+    e = oracle.weighted_error(W, x, s, 128)
+    assert err[0] == err[1]
+    assert math.isclose(err[0], e, rel_tol=1e-12)
+
+
+def test_clip_constant_magnitude_group_keeps_full_range():
+    """|w s| equal across a group: the unclipped codes are all +-7 and any
+    shrink saturates every weight below its value, so index 0 wins."""
+    g = 32
+    rng = np.random.default_rng(45)
+    signs = np.where(rng.standard_normal((8, g)) > 0, 1.0, -1.0)
+    W = (signs * 0.0123).astype(np.float16)
+    x = np.ones(g, np.float32)
+    idx, err = oracle.clip_search(W, x, None, g, 20)
+    assert not idx.any()
+    assert err[0] == err[1]
+
+
+def test_clip_scaling_by_power_of_two():
+    """Scaling W by 2 leaves every decision unchanged and multiplies the
+    errors by 4 (every rounding step commutes with a power of two)."""
+    rng = np.random.default_rng(46)
+    W = (rng.standard_normal((16, 256)) * 0.02).astype(np.float16)
+    x = np.exp(rng.standard_normal(256)).astype(np.float32)
+    idx1, err1 = oracle.clip_search(W, x, None, 64, 10)
+    idx2, err2 = oracle.clip_search((W.astype(np.float32) * 2).astype(np.float16), x, None, 64, 10)
+    assert np.array_equal(idx1, idx2)
+    assert np.allclose(err2, 4 * err1, rtol=1e-12)
+
+
+def test_clip_pack_matches_clipped_groups():
+    """The pack with clip indices stores the clipped group's codes and fp16
+    scale; index 0 everywhere is the unclipped pack."""
+    rng = np.random.default_rng(47)
+    d_out, d_in, g = 16, 256, 64
+    W = (rng.standard_normal((d_out, d_in)) * 0.02).astype(np.float16)
+    s = np.exp(rng.standard_normal(d_in) * 0.5).astype(np.float32)
+    idx = rng.integers(0, 10, size=(d_out, d_in // g)).astype(np.uint8)
+    qw, sc, qz = oracle.quantize_pack(W, s, g, 8, idx)
+    u = oracle.unpack(qw, d_out)
+    Wf = W.astype(np.float32)
+    for r in range(d_out):
+        for k in range(d_in // g):
+            sl = slice(k * g, (k + 1) * g)
+            q, qs = oracle.fake_quant_group_clip(Wf[r, sl], s[sl], oracle.clip_ratio(idx[r, k]), 0)
+            assert np.array_equal(u[r, sl].astype(np.int32), q.astype(np.int32) + 8)
+            assert sc[k, r] == np.float16(qs)
+    zero = np.zeros_like(idx)
+    a = oracle.quantize_pack(W, s, g, 8, zero)
+    b = oracle.quantize_pack(W, s, g, 8)
+    for t1, t2 in zip(a, b):
+        assert np.array_equal(t1.view(np.uint8), t2.view(np.uint8))
