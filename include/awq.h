@@ -61,6 +61,12 @@ typedef enum awq_status {
 #define AWQ_OP_ACT_STATS    0
 #define AWQ_OP_SCALE_SEARCH 1
 #define AWQ_OP_OUTPUT_ERROR 2
+#define AWQ_OP_CLIP_SEARCH  3
+
+/* Clip ratios: index i stands for c_i = (AWQ_CLIP_DEN - i) / AWQ_CLIP_DEN
+ * rounded to fp32; 0 is no clipping, at most AWQ_CLIP_MAX ratios. */
+#define AWQ_CLIP_DEN 20
+#define AWQ_CLIP_MAX 20
 
 /* Human-readable name of a status code (static storage; never NULL). */
 const char *awq_status_string(int status);
@@ -77,7 +83,8 @@ const char *awq_last_error(void);
  * Bytes of workspace that `op` needs for the given sizes.  For
  * AWQ_OP_ACT_STATS only d_in matters; for AWQ_OP_SCALE_SEARCH d_in, the
  * group size and n_grid; for AWQ_OP_OUTPUT_ERROR all of them (T is the token
- * count, d_out_total the rows of W).  Writes *bytes; returns
+ * count, d_out_total the rows of W); for AWQ_OP_CLIP_SEARCH only the group
+ * size is checked (the workspace is a fixed 16.6 KB).  Writes *bytes; returns
  * AWQ_ERR_INVALID_ARG for an unknown op or out-of-range size.
  */
 awq_status awq_workspace_size(int op, int64_t T, int64_t d_out_total,
@@ -198,6 +205,11 @@ awq_status awq_scale_search_noalloc(int n_seg, const void *const *W,
  *   W           fp16 [d_out, d_in] device
  *   d_out       multiple of 8;  d_in multiple of group_size
  *   s           fp32 [d_in] device scale (s_best), or NULL for s = 1 (RTN)
+ *   clip_idx    uint8 [d_out, d_in / group_size] device clip ratio indices
+ *               from awq_clip_search, or NULL for none: group (r, k) uses the
+ *               range c * max|ws| with c = (20 - i) / 20 (indices above 19
+ *               count as 19), q_scale = fp16(fl32(fl32(c m) / 7)), and codes
+ *               beyond the range saturate at +-7
  *   group_size  32, 64 or 128
  *   zero_point  7 or 8 (8: codes 1..15; 7: codes 0..14)
  *   qweight     int32 [d_in, d_out / 8] device output
@@ -207,9 +219,48 @@ awq_status awq_scale_search_noalloc(int n_seg, const void *const *W,
  * zero_point for all its weights.
  */
 awq_status awq_quantize_pack(const void *W, int64_t d_out, int64_t d_in,
-                             const float *s, int group_size, int zero_point,
-                             int32_t *qweight, void *scales, int32_t *qzeros,
-                             void *stream);
+                             const float *s, const uint8_t *clip_idx,
+                             int group_size, int zero_point, int32_t *qweight,
+                             void *scales, int32_t *qzeros, void *stream);
+
+/*
+ * Per (row, group) clip search at a fixed scale ("AWQ architecture ...",
+ * section "The pipeline end to end", step 5: an optional search of a
+ * clipping range per output channel that shrinks the quantisation range to
+ * cut rounding error on outliers; the pages give no formula, the reading
+ * is this one).  For every row r, group k and i < n_clip, with
+ * c_i = (20 - i) / 20 rounded to fp32:
+ *
+ *   q_scale_i = fp16_rne(fl32(fl32(c_i * max_j |w_j s_j|) / 7))
+ *   q_j       = clamp(rint(w_j s_j / q_scale_i), -7, 7)
+ *   e_i       = sum_j ((w_j - q_j q_scale_i / s_j) * x_mean_j)^2
+ *
+ * and clip_idx[r, k] = the first i with the smallest e_i.  err[0] is the
+ * total error without clipping (i = 0 everywhere), err[1] the total with
+ * the chosen ratios; both are reduced in a fixed order (deterministic).
+ * Each e_i is summed in fp32 (so two ratios within ~1e-6 of each other may
+ * be ordered differently from an exact evaluation); codes use an
+ * approximate reciprocal of q_scale (the stored codes come from
+ * awq_quantize_pack's exact quotient).
+ *
+ *   W           fp16 [d_out, d_in] device;  d_out >= 1
+ *   d_in        multiple of group_size
+ *   x_mean      fp32 [d_in] device
+ *   s           fp32 [d_in] device (normally s_best), or NULL for s = 1
+ *   group_size  32, 64 or 128
+ *   n_clip      1..AWQ_CLIP_MAX ratios (10: down to 0.55)
+ *   flags       AWQ_SCALE_FP16 or AWQ_SCALE_FP32
+ *   clip_idx    uint8 [d_out, d_in / group_size] device output
+ *   err         fp64 [2] device output (NaN if W holds a non-finite value;
+ *               such a group keeps index 0)
+ *   ws          workspace of awq_workspace_size(AWQ_OP_CLIP_SEARCH, ...),
+ *               256-byte aligned
+ */
+awq_status awq_clip_search(const void *W, int64_t d_out, int64_t d_in,
+                           const float *x_mean, const float *s, int group_size,
+                           int n_clip, int flags, uint8_t *clip_idx,
+                           double *err, void *ws, size_t ws_bytes,
+                           void *stream);
 
 /*
  * Optional output-space scoring of every grid point ("AWQ architecture

@@ -21,6 +21,8 @@ SCALE_FP32 = 1
 OP_ACT_STATS = 0
 OP_SCALE_SEARCH = 1
 OP_OUTPUT_ERROR = 2
+OP_CLIP_SEARCH = 3
+CLIP_DEN = 20
 MAX_SEGMENTS = 8
 
 LIB_PATH = _build.LIB
@@ -60,8 +62,10 @@ def lib() -> ctypes.CDLL:
         L.awq_act_stats.restype = i32
         L.awq_scale_search.argtypes = [i32, p, p, i64, p, i32, i32, i32, p, p, p, p, sz, p]
         L.awq_scale_search.restype = i32
-        L.awq_quantize_pack.argtypes = [p, i64, i64, p, i32, i32, p, p, p, p]
+        L.awq_quantize_pack.argtypes = [p, i64, i64, p, p, i32, i32, p, p, p, p]
         L.awq_quantize_pack.restype = i32
+        L.awq_clip_search.argtypes = [p, i64, i64, p, p, i32, i32, i32, p, p, p, sz, p]
+        L.awq_clip_search.restype = i32
         L.awq_output_error.argtypes = [p, i64, p, i64, i64, p, i32, i32, i32, p, p, p, p, sz, p]
         L.awq_output_error.restype = i32
         _lib = L
@@ -153,13 +157,18 @@ def scale_search(Ws: Sequence[torch.Tensor], x: torch.Tensor, group_size: int = 
 
 
 def quantize_pack(W: torch.Tensor, s: Optional[torch.Tensor] = None, group_size: int = 128,
-                  zero_point: int = 8, out=None):
+                  zero_point: int = 8, out=None, clip_idx: Optional[torch.Tensor] = None):
     """AutoAWQ GEMM packing: (qweight int32 [d_in, d_out/8],
-    scales fp16 [d_in/g, d_out], qzeros int32 [d_in/g, d_out/8])."""
+    scales fp16 [d_in/g, d_out], qzeros int32 [d_in/g, d_out/8]).
+    clip_idx: optional uint8 [d_out, d_in/g] from clip_search."""
     _cuda(W, torch.float16, "W")
     d_out, d_in = W.shape
     if s is not None:
         _cuda(s, torch.float32, "s")
+    if clip_idx is not None:
+        _cuda(clip_idx, torch.uint8, "clip_idx")
+        if tuple(clip_idx.shape) != (d_out, d_in // group_size):
+            raise ValueError("clip_idx must be [d_out, d_in / group_size]")
     dev = W.device
     G = d_in // group_size
     if out is None:
@@ -168,11 +177,38 @@ def quantize_pack(W: torch.Tensor, s: Optional[torch.Tensor] = None, group_size:
                torch.empty(G, d_out // 8, dtype=torch.int32, device=dev))
     qw, sc, qz = out
     _check(lib().awq_quantize_pack(W.data_ptr(), d_out, d_in,
-                                   None if s is None else s.data_ptr(), group_size,
-                                   zero_point, qw.data_ptr(), sc.data_ptr(), qz.data_ptr(),
-                                   _stream(dev)),
+                                   None if s is None else s.data_ptr(),
+                                   None if clip_idx is None else clip_idx.data_ptr(),
+                                   group_size, zero_point, qw.data_ptr(), sc.data_ptr(),
+                                   qz.data_ptr(), _stream(dev)),
            "awq_quantize_pack")
     return qw, sc, qz
+
+
+def clip_search(W: torch.Tensor, x: torch.Tensor, s: Optional[torch.Tensor] = None,
+                group_size: int = 128, n_clip: int = 10, flags: int = SCALE_FP16,
+                out: Optional[Tuple[torch.Tensor, torch.Tensor]] = None,
+                ws: Optional[torch.Tensor] = None):
+    """Per (row, group) clip ratio search at scale s: (clip_idx uint8
+    [d_out, d_in/g], err fp64[2] = (no clipping, chosen ratios))."""
+    _cuda(W, torch.float16, "W")
+    _cuda(x, torch.float32, "x")
+    if s is not None:
+        _cuda(s, torch.float32, "s")
+    d_out, d_in = W.shape
+    dev = W.device
+    if out is None:
+        out = (torch.empty(d_out, d_in // group_size, dtype=torch.uint8, device=dev),
+               torch.empty(2, dtype=torch.float64, device=dev))
+    idx, err = out
+    if ws is None:
+        ws = workspace(OP_CLIP_SEARCH, dev, 1, d_out, d_in, group_size, 1)
+    _check(lib().awq_clip_search(W.data_ptr(), d_out, d_in, x.data_ptr(),
+                                 None if s is None else s.data_ptr(), group_size, n_clip, flags,
+                                 idx.data_ptr(), err.data_ptr(), ws.data_ptr(), ws.numel(),
+                                 _stream(dev)),
+           "awq_clip_search")
+    return idx, err
 
 
 def output_error(X: torch.Tensor, W: torch.Tensor, x: torch.Tensor, group_size: int = 128,

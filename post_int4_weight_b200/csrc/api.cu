@@ -84,6 +84,10 @@ awq_status awq_workspace_size(int op, int64_t T, int64_t d_out_total, int64_t d_
             if (!valid_group(group_size) || n_grid < 1 || n_grid > 32) return AWQ_ERR_INVALID_ARG;
             *bytes = scale_search_workspace(d_in, group_size, n_grid);
             return AWQ_OK;
+        case AWQ_OP_CLIP_SEARCH:
+            if (!valid_group(group_size)) return AWQ_ERR_INVALID_ARG;
+            *bytes = clip_search_workspace();
+            return AWQ_OK;
         case AWQ_OP_OUTPUT_ERROR:
             if (!valid_group(group_size) || n_grid < 1 || n_grid > 32 || T < 1 ||
                 d_out_total < 1)
@@ -137,8 +141,8 @@ awq_status awq_scale_search(int n_seg, const void* const* W, const int64_t* d_ou
 }
 
 awq_status awq_quantize_pack(const void* W, int64_t d_out, int64_t d_in, const float* s,
-                             int group_size, int zero_point, int32_t* qweight, void* scales,
-                             int32_t* qzeros, void* stream) {
+                             const uint8_t* clip_idx, int group_size, int zero_point,
+                             int32_t* qweight, void* scales, int32_t* qzeros, void* stream) {
     if (!W || !qweight || !scales || !qzeros) return AWQ_ERR_INVALID_ARG;
     if (!valid_group(group_size)) return AWQ_ERR_UNSUPPORTED;
     if (zero_point != 7 && zero_point != 8) return AWQ_ERR_INVALID_ARG;
@@ -148,8 +152,32 @@ awq_status awq_quantize_pack(const void* W, int64_t d_out, int64_t d_in, const f
     if (!aligned16(W) || !aligned16(qweight) || !aligned16(scales) || !aligned16(qzeros))
         return AWQ_ERR_ALIGNMENT;
     if (s && !aligned16(s)) return AWQ_ERR_ALIGNMENT;
-    if (launch_quantize_pack(W, d_out, d_in, s, group_size, zero_point, qweight, scales,
-                             qzeros, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    if (note_cuda(launch_quantize_pack(W, d_out, d_in, s, clip_idx, group_size, zero_point,
+                                       qweight, scales, qzeros,
+                                       static_cast<cudaStream_t>(stream)),
+                  "quantize_pack launch") != cudaSuccess)
+        return AWQ_ERR_CUDA;
+    return AWQ_OK;
+}
+
+awq_status awq_clip_search(const void* W, int64_t d_out, int64_t d_in, const float* x_mean,
+                           const float* s, int group_size, int n_clip, int flags,
+                           uint8_t* clip_idx, double* err, void* ws, size_t ws_bytes,
+                           void* stream) {
+    if (!W || !x_mean || !clip_idx || !err) return AWQ_ERR_INVALID_ARG;
+    if (!valid_group(group_size)) return AWQ_ERR_UNSUPPORTED;
+    if (n_clip < 1 || n_clip > AWQ_CLIP_MAX) return AWQ_ERR_INVALID_ARG;
+    if (flags != AWQ_SCALE_FP16 && flags != AWQ_SCALE_FP32) return AWQ_ERR_INVALID_ARG;
+    if (d_out < 1 || d_out > (int64_t(1) << 31)) return AWQ_ERR_INVALID_ARG;
+    if (d_in < group_size || d_in % group_size || d_in > (int64_t(1) << 24))
+        return AWQ_ERR_INVALID_ARG;
+    if (!aligned16(W) || !aligned16(x_mean) || !aligned16(err) || (s && !aligned16(s)))
+        return AWQ_ERR_ALIGNMENT;
+    if (!ws || ws_bytes < clip_search_workspace()) return AWQ_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(ws) & (kWsAlign - 1)) != 0) return AWQ_ERR_ALIGNMENT;
+    if (note_cuda(launch_clip_search(W, d_out, d_in, x_mean, s, group_size, n_clip, flags,
+                                     clip_idx, err, ws, static_cast<cudaStream_t>(stream)),
+                  "clip_search launch") != cudaSuccess)
         return AWQ_ERR_CUDA;
     return AWQ_OK;
 }

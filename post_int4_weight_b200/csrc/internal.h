@@ -46,9 +46,15 @@ awq_status launch_scale_search(int n_seg, const void* const* W, const int64_t* d
 
 // ---- quantise + pack
 cudaError_t launch_quantize_pack(const void* W, int64_t d_out, int64_t d_in,
-                                 const float* s, int group_size, int zero_point,
-                                 int32_t* qweight, void* scales, int32_t* qzeros,
-                                 cudaStream_t stream);
+                                 const float* s, const uint8_t* clip_idx, int group_size,
+                                 int zero_point, int32_t* qweight, void* scales,
+                                 int32_t* qzeros, cudaStream_t stream);
+
+// ---- clip search
+size_t clip_search_workspace();
+cudaError_t launch_clip_search(const void* W, int64_t d_out, int64_t d_in, const float* x_mean,
+                               const float* s, int group_size, int n_clip, int flags,
+                               uint8_t* clip_idx, double* err, void* ws, cudaStream_t stream);
 
 // ---- output-space scoring
 size_t output_error_workspace(int64_t T, int64_t d_out, int64_t d_in, int group_size,

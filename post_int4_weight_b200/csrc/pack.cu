@@ -36,6 +36,8 @@ constexpr int kPackCols = 128;
 constexpr int kPackChunks = kPackCols / 8;     // 16-byte chunks per tile row
 constexpr int kPackThreads = 256;
 constexpr int kBlocks32 = kPackRows / 32;      // 32-row blocks per tile
+constexpr int kClipDen = 20;                   // clip ratio c_i = (20 - i) / 20
+constexpr int kClipMaxIndex = 19;
 
 __device__ __forceinline__ int pack_swz(int r) { return (r ^ (r >> 4)) & 7; }
 
@@ -104,8 +106,9 @@ __device__ __forceinline__ void pack_columns(const uint4* tile, const float2* qr
 template <int G>
 __global__ void __launch_bounds__(kPackThreads, 5)
 pack_kernel(const uint4* __restrict__ W, int64_t d_out, int64_t d_in,
-            const float* __restrict__ s, int zero_point, int32_t* __restrict__ qweight,
-            __half* __restrict__ scales, int32_t* __restrict__ qzeros) {
+            const float* __restrict__ s, const uint8_t* __restrict__ clip_idx, int zero_point,
+            int32_t* __restrict__ qweight, __half* __restrict__ scales,
+            int32_t* __restrict__ qzeros) {
     constexpr int KG = kPackCols / G;               // groups per tile
     extern __shared__ __align__(16) unsigned char smem[];
     uint4* tile = reinterpret_cast<uint4*>(smem);                       // 32 KB
@@ -182,12 +185,22 @@ pack_kernel(const uint4* __restrict__ W, int64_t d_out, int64_t d_in,
         }
         if (half == 0) {
             const bool bad = !(m <= 3.402823466e38f);      // a NaN or an infinity
+            const int64_t gr = row0 + r, gk = col0 / G + kk;
+            // clipping shrinks the range to c * m, c = RN((20 - i) / 20); codes
+            // beyond it saturate, so the block takes the clamping path
+            bool clipped = false;
+            if (clip_idx && gr < d_out && gk * G < d_in) {
+                const int ci = min((int)clip_idx[gr * (d_in / G) + gk], kClipMaxIndex);
+                if (ci > 0) {
+                    m = __fmul_rn(m, __fdiv_rn((float)(kClipDen - ci), (float)kClipDen));
+                    clipped = true;
+                }
+            }
             bool in_range;
             const float qs = bad ? 1.0f : group_scale(m, false, &in_range);
             qr_tile[row_slot(kk, r)] = make_float2(qs, (qs > 0.f) ? __frcp_rn(qs) : 0.f);
             bad_tile[row_slot(kk, r)] = bad;
-            if (bad || !in_range) slow_blk[kk * kBlocks32 + r / 32] = 1;
-            const int64_t gr = row0 + r, gk = col0 / G + kk;
+            if (bad || clipped || !in_range) slow_blk[kk * kBlocks32 + r / 32] = 1;
             if (gr < d_out && gk * G < d_in)
                 scales[gk * d_out + gr] = bad ? __ushort_as_half((unsigned short)0x7E00)
                                               : __float2half_rn(qs);
@@ -238,8 +251,8 @@ pack_kernel(const uint4* __restrict__ W, int64_t d_out, int64_t d_in,
 
 template <int G>
 cudaError_t launch_pack_G(const void* W, int64_t d_out, int64_t d_in, const float* s,
-                          int zero_point, int32_t* qweight, void* scales, int32_t* qzeros,
-                          cudaStream_t stream) {
+                          const uint8_t* clip_idx, int zero_point, int32_t* qweight,
+                          void* scales, int32_t* qzeros, cudaStream_t stream) {
     constexpr int KG = kPackCols / G;
     const size_t smem = (size_t)kPackRows * kPackCols * 2 + (2 * kPackCols + 8) * sizeof(float) +
                         (size_t)KG * kRowStride * (sizeof(float2) + sizeof(int)) +
@@ -257,25 +270,26 @@ cudaError_t launch_pack_G(const void* W, int64_t d_out, int64_t d_in, const floa
     dim3 grid((unsigned)((d_in + kPackCols - 1) / kPackCols),
               (unsigned)((d_out + kPackRows - 1) / kPackRows));
     return launch_pdl(pack_kernel<G>, grid, dim3(kPackThreads), smem, stream,
-                      static_cast<const uint4*>(W), d_out, d_in, s, zero_point, qweight,
-                      static_cast<__half*>(scales), qzeros);
+                      static_cast<const uint4*>(W), d_out, d_in, s, clip_idx, zero_point,
+                      qweight, static_cast<__half*>(scales), qzeros);
 }
 
 }  // namespace
 
 cudaError_t launch_quantize_pack(const void* W, int64_t d_out, int64_t d_in, const float* s,
-                                 int group_size, int zero_point, int32_t* qweight,
-                                 void* scales, int32_t* qzeros, cudaStream_t stream) {
+                                 const uint8_t* clip_idx, int group_size, int zero_point,
+                                 int32_t* qweight, void* scales, int32_t* qzeros,
+                                 cudaStream_t stream) {
     switch (group_size) {
         case 32:
-            return launch_pack_G<32>(W, d_out, d_in, s, zero_point, qweight, scales, qzeros,
-                                     stream);
+            return launch_pack_G<32>(W, d_out, d_in, s, clip_idx, zero_point, qweight, scales,
+                                     qzeros, stream);
         case 64:
-            return launch_pack_G<64>(W, d_out, d_in, s, zero_point, qweight, scales, qzeros,
-                                     stream);
+            return launch_pack_G<64>(W, d_out, d_in, s, clip_idx, zero_point, qweight, scales,
+                                     qzeros, stream);
         case 128:
-            return launch_pack_G<128>(W, d_out, d_in, s, zero_point, qweight, scales, qzeros,
-                                      stream);
+            return launch_pack_G<128>(W, d_out, d_in, s, clip_idx, zero_point, qweight, scales,
+                                      qzeros, stream);
         default:
             return cudaErrorInvalidValue;
     }

@@ -89,10 +89,23 @@ def test_host_validation_without_a_gpu():
     assert L.awq_scale_search(1, W, d, 256, fake, 128, 20, 0, fake, fake, fake, fake,
                               16, None) == 4
     # quantize_pack
-    assert L.awq_quantize_pack(fake, 12, 256, None, 128, 8, fake, fake, fake, None) == 1
-    assert L.awq_quantize_pack(fake, 64, 256, None, 128, 9, fake, fake, fake, None) == 1
-    assert L.awq_quantize_pack(fake, 64, 256, None, 48, 8, fake, fake, fake, None) == 2
-    assert L.awq_quantize_pack(fake, 64, 256, odd, 128, 8, fake, fake, fake, None) == 3
+    assert L.awq_quantize_pack(fake, 12, 256, None, None, 128, 8, fake, fake, fake, None) == 1
+    assert L.awq_quantize_pack(fake, 64, 256, None, None, 128, 9, fake, fake, fake, None) == 1
+    assert L.awq_quantize_pack(fake, 64, 256, None, None, 48, 8, fake, fake, fake, None) == 2
+    assert L.awq_quantize_pack(fake, 64, 256, odd, None, 128, 8, fake, fake, fake, None) == 3
+    # clip_search
+    assert L.awq_clip_search(fake, 64, 256, fake, None, 128, 0, 0, fake, fake, fake,
+                             1 << 20, None) == 1
+    assert L.awq_clip_search(fake, 64, 256, fake, None, 128, 21, 0, fake, fake, fake,
+                             1 << 20, None) == 1
+    assert L.awq_clip_search(fake, 64, 256, fake, None, 48, 10, 0, fake, fake, fake,
+                             1 << 20, None) == 2
+    assert L.awq_clip_search(fake, 64, 200, fake, None, 128, 10, 0, fake, fake, fake,
+                             1 << 20, None) == 1
+    assert L.awq_clip_search(fake, 64, 256, fake, odd, 128, 10, 0, fake, fake, fake,
+                             1 << 20, None) == 3
+    assert L.awq_clip_search(fake, 64, 256, fake, None, 128, 10, 0, fake, fake, fake,
+                             64, None) == 4
     # output_error
     assert L.awq_output_error(fake, 0, fake, 64, 256, fake, 128, 20, 0, fake, fake,
                               None, fake, 1 << 30, None) == 1
