@@ -79,6 +79,9 @@ def _args():
     ap.add_argument("--workload", default="q_proj_4096x4096")
     ap.add_argument("--group-size", type=int, default=0,
                     help="group size (default: the workload's first)")
+    ap.add_argument("--clip", type=int, default=0,
+                    help="also run the clip search with this many ratios per member "
+                         "(0: off, the method's default path)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-graph", action="store_true",
@@ -214,7 +217,7 @@ def run_ours(a):
     for li in layer_inputs:
         for Ws, X in li:
             jobs.append(pipeline.GroupJob([W.to(dev) for W in Ws], X.to(dev), g, n_grid,
-                                          work.output_mode))
+                                          work.output_mode, n_clip=a.clip))
     if work.layers == 1:
         host_layer = [([W.pin_memory() for W in Ws], X.pin_memory()) for Ws, X in layer_inputs[0]]
     else:
@@ -239,6 +242,10 @@ def run_ours(a):
         for j in jobs:
             j.pack()
 
+    def call_clip():
+        for j in jobs:
+            j.clip(wss.clip)
+
     def step():
         for j in jobs:
             j.run(wss)
@@ -256,8 +263,9 @@ def run_ours(a):
     graphs = None
     if not a.no_graph:
         graphs = {}
-        for name, fn in (("step", step), ("stats", call_stats), ("search", call_search),
-                         ("pack", call_pack)):
+        calls = [("step", step), ("stats", call_stats), ("search", call_search),
+                 ("pack", call_pack)] + ([("clip", call_clip)] if a.clip > 0 else [])
+        for name, fn in calls:
             gr = torch.cuda.CUDAGraph()
             with torch.cuda.graph(gr):
                 fn()
@@ -267,7 +275,9 @@ def run_ours(a):
             graphs["step"].replay()
         torch.cuda.synchronize(dev)
     run = {k: (graphs[k].replay if graphs else f) for k, f in
-           (("step", step), ("stats", call_stats), ("search", call_search), ("pack", call_pack))}
+           (("step", step), ("stats", call_stats), ("search", call_search), ("pack", call_pack),
+            ("clip", call_clip))
+           if a.clip > 0 or k != "clip"}
 
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(a.steps)]
@@ -288,29 +298,28 @@ def run_ours(a):
 
     # per-call breakdown (separately timed passes, L2 flushed before each)
     n_br = max(3, min(200, a.steps))
-    br = {"stats": [], "search": [], "pack": []}
+    names = ["stats", "search"] + (["clip"] if a.clip > 0 else []) + ["pack"]
+    br = {k: [] for k in names}
     for _ in range(n_br):
         do_flush()
-        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
         ev[0].record(stream)
-        run["stats"]()
-        ev[1].record(stream)
-        run["search"]()
-        ev[2].record(stream)
-        run["pack"]()
-        ev[3].record(stream)
+        for i, k in enumerate(names):
+            run[k]()
+            ev[i + 1].record(stream)
         torch.cuda.synchronize(dev)
-        br["stats"].append(ev[0].elapsed_time(ev[1]))
-        br["search"].append(ev[1].elapsed_time(ev[2]))
-        br["pack"].append(ev[2].elapsed_time(ev[3]))
+        for i, k in enumerate(names):
+            br[k].append(ev[i].elapsed_time(ev[i + 1]))
     ms_stats = sum(br["stats"]) / n_br
     ms_search = sum(br["search"]) / n_br
     ms_pack = sum(br["pack"]) / n_br
+    ms_clip = sum(br["clip"]) / n_br if a.clip > 0 else None
     del graphs
 
     # --- end to end: the same work streamed from pinned host memory
     template = layer_inputs[0]
-    streamer = pipeline.LayerStreamer(template, dev, g, n_grid, work.output_mode)
+    streamer = pipeline.LayerStreamer(template, dev, g, n_grid, work.output_mode,
+                                      n_clip=a.clip)
     if work.layers == 1:
         n_e2e = max(5, min(50, a.steps // 20))
         host_layers = [host_layer] * n_e2e
@@ -401,6 +410,11 @@ def run_ours(a):
                 "peak_basis": f"{n_sms} SMs x {FP32_LANES_PER_SM} FP32 lanes x "
                               f"{clk_mhz:.0f} MHz (median SM clock sampled in the timed "
                               f"region)"}
+        if a.clip > 0:
+            clip_ops = params * a.clip * ALG_OPS_PER_PAIR
+            kernels["clip_search"] = {"ms": ms_clip, "n_clip": a.clip,
+                                      "Top/s": clip_ops / (ms_clip * 1e-3) / 1e12,
+                                      "frac_of_alu_peak": clip_ops / (ms_clip * 1e-3) / peak_ops}
         kernels["scale_search"] = {"ms": ms_search, "Top/s": achieved / 1e12,
                                    "executed_Tlane-op/s": executed / 1e12,
                                    "W_GB/s": params * 2 / (ms_search * 1e-3) / 1e9}
@@ -415,7 +429,7 @@ def run_ours(a):
         "vs_baseline": None, "dtype": "f16" if work.output_mode else "f32",
         "data": "synthetic",
         "config": {"workload": a.workload, "layers": work.layers, "tokens": work.tokens,
-                   "group_size": g, "n_grid": n_grid,
+                   "group_size": g, "n_grid": n_grid, "n_clip": a.clip,
                    "params_per_step": _total_params(work, world, params),
                    "params_rank0": params,
                    "l2": ("flushed (256 MB write) between timed steps" if flush_l2 else
@@ -430,7 +444,7 @@ def run_ours(a):
         "launch": "CUDA graph per step" if not a.no_graph else "eager",
     }
     if world == 1 and not a.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(work, g, a.cpu_seconds)
+        out["cpu_baseline"] = cpu_baseline(work, g, a.cpu_seconds, a.clip)
     print(json.dumps(out), flush=True)
     if world > 1:
         dist.destroy_process_group()
@@ -480,7 +494,7 @@ def oracle_sample(work, g, row_cap=256, out_rows=16, out_tokens=None):
     return out, params, "; ".join(parts) + f" ({mode})"
 
 
-def _oracle_pass(sample, g, n_grid, output_mode):
+def _oracle_pass(sample, g, n_grid, output_mode, n_clip=0):
     import oracle
     for Ws, X in sample:
         x = oracle.act_stats(X)
@@ -490,18 +504,21 @@ def _oracle_pass(sample, g, n_grid, output_mode):
         else:
             err, best, s = oracle.scale_search(Ws, x, g, n_grid)
         for W in Ws:
-            oracle.quantize_pack(W, s, g, 8)
+            idx = oracle.clip_search(W, x, s, g, n_clip)[0] if n_clip > 0 else None
+            oracle.quantize_pack(W, s, g, 8, idx)
 
 
-def cpu_baseline(work, g, seconds):
+def cpu_baseline(work, g, seconds, n_clip=0):
     """Passes of the CPU oracle over a bounded sample of the workload until
     `seconds` have elapsed."""
     import oracle
     sample, params, text = oracle_sample(work, g)
+    if n_clip > 0:
+        text += f" + {n_clip}-ratio clip search"
     n = 0
     t0 = time.perf_counter()
     while True:
-        _oracle_pass(sample, g, work.n_grid, work.output_mode)
+        _oracle_pass(sample, g, work.n_grid, work.output_mode, n_clip)
         n += 1
         if time.perf_counter() - t0 >= seconds:
             break
@@ -521,11 +538,13 @@ def run_reference(a):
     g = _group_size(a, work)
     # a small sample per step, so that even thousands of steps end in minutes
     sample, params, text = oracle_sample(work, g, row_cap=64, out_rows=8, out_tokens=1024)
+    if a.clip > 0:
+        text += f" + {a.clip}-ratio clip search"
     for _ in range(max(a.warmup, 3)):
-        _oracle_pass(sample, g, work.n_grid, work.output_mode)
+        _oracle_pass(sample, g, work.n_grid, work.output_mode, a.clip)
     t0 = time.perf_counter()
     for _ in range(a.steps):
-        _oracle_pass(sample, g, work.n_grid, work.output_mode)
+        _oracle_pass(sample, g, work.n_grid, work.output_mode, a.clip)
     dt = time.perf_counter() - t0
     v = a.steps * params / dt / 1e9
     print(json.dumps({
@@ -534,7 +553,7 @@ def run_reference(a):
         "higher_is_better": True, "scaling": "strong" if work.layers > 1 else "weak",
         "vs_baseline": None, "dtype": "f64" if work.output_mode else "f32",
         "data": "synthetic", "config": {"workload": a.workload, "group_size": g,
-                                        "n_grid": work.n_grid},
+                                        "n_grid": work.n_grid, "n_clip": a.clip},
         "cpu_baseline": {"value": v, "unit": UNIT, "cores": oracle.threads(),
                          "kind": "oracle", "sample": f"per step, one pass over {text}"},
         "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},

@@ -7,7 +7,9 @@ in the library's kernels through the calls of :mod:`awq`.
 The unit of work is a *search group*: the linears that read one input X
 (q/k/v, gate/up, or a linear alone).  Its path is awq_act_stats on X, the
 scale search (weight-space, or output-space with ``output_mode``) over all
-members at once, then awq_quantize_pack of every member at the chosen scale
+members at once, optionally a clip search per member (``n_clip`` > 0; the
+architecture page's pipeline step 5), then awq_quantize_pack of every member
+at the chosen scale (and clip ratios)
 ("From-Scratch AWQ INT4 Quantization on Qwen3-8B", pipeline and AWQ scaling
 sections; "AWQ architecture, in depth", section "The scale search as code").
 """
@@ -21,12 +23,13 @@ from . import awq
 
 # kernels each call launches (the library's own count, used for reporting)
 LAUNCHES_STATS = 1
-LAUNCHES_SEARCH = 3            # scale table (2) + fused search with finalize
+LAUNCHES_SEARCH = 2            # scale table + fused search with finalize
+LAUNCHES_CLIP = 1              # per member (plus a 4-byte memset of its counter)
 
 
 def launches_output_error(n_grid: int) -> int:
-    """Scale table (2) + one dW builder and one GEMM per grid point + finalize."""
-    return 2 + 2 * n_grid + 1
+    """Scale table + one dW builder and one GEMM per grid point + finalize."""
+    return 1 + 2 * n_grid + 1
 
 
 def shard_layers(n_layers: int, world: int, rank: int) -> List[int]:
@@ -61,7 +64,8 @@ class GroupJob:
     """
 
     def __init__(self, Ws: Sequence[torch.Tensor], X: torch.Tensor, group_size: int = 128,
-                 n_grid: int = 20, output_mode: bool = False, zero_point: int = 8):
+                 n_grid: int = 20, output_mode: bool = False, zero_point: int = 8,
+                 n_clip: int = 0):
         if output_mode and len(Ws) != 1:
             raise ValueError("the output-space score takes one linear per call")
         self.Ws = list(Ws)
@@ -70,6 +74,7 @@ class GroupJob:
         self.n_grid = n_grid
         self.output_mode = output_mode
         self.zero_point = zero_point
+        self.n_clip = n_clip
         dev = X.device
         T, d_in = X.shape
         self.x = torch.empty(d_in, dtype=torch.float32, device=dev)
@@ -81,6 +86,10 @@ class GroupJob:
                        torch.empty(G, W.shape[0], dtype=torch.float16, device=dev),
                        torch.empty(G, W.shape[0] // 8, dtype=torch.int32, device=dev))
                       for W in self.Ws]
+        # clip ratio indices and (unclipped, clipped) error totals per member
+        self.clips = [(torch.zeros(W.shape[0], G, dtype=torch.uint8, device=dev),
+                       torch.zeros(2, dtype=torch.float64, device=dev))
+                      for W in self.Ws] if n_clip > 0 else []
 
     @property
     def params(self) -> int:
@@ -89,16 +98,19 @@ class GroupJob:
     @property
     def launches(self) -> int:
         search = launches_output_error(self.n_grid) if self.output_mode else LAUNCHES_SEARCH
-        return LAUNCHES_STATS + search + len(self.Ws)
+        clip = LAUNCHES_CLIP * len(self.Ws) if self.n_clip > 0 else 0
+        return LAUNCHES_STATS + search + clip + len(self.Ws)
 
-    def workspace_bytes(self) -> Tuple[int, int]:
-        """(act_stats, search) workspace bytes of this job."""
+    def workspace_bytes(self) -> Tuple[int, int, int]:
+        """(act_stats, search, clip) workspace bytes of this job."""
         T, d_in = self.X.shape
         d_out = sum(W.shape[0] for W in self.Ws)
         st = awq.workspace_size(awq.OP_ACT_STATS, T, 8, d_in, self.g, self.n_grid)
         op = awq.OP_OUTPUT_ERROR if self.output_mode else awq.OP_SCALE_SEARCH
         se = awq.workspace_size(op, T, d_out, d_in, self.g, self.n_grid)
-        return st, se
+        cl = awq.workspace_size(awq.OP_CLIP_SEARCH, T, d_out, d_in, self.g, 1) \
+            if self.n_clip > 0 else 0
+        return st, se, cl
 
     def stats(self, ws: torch.Tensor):
         awq.act_stats(self.X, out=self.x, ws=ws)
@@ -110,13 +122,20 @@ class GroupJob:
         else:
             awq.scale_search(self.Ws, self.x, self.g, self.n_grid, out=out, ws=ws)
 
+    def clip(self, ws: torch.Tensor):
+        for W, cl in zip(self.Ws, self.clips):
+            awq.clip_search(W, self.x, self.s_best, self.g, self.n_clip, out=cl, ws=ws)
+
     def pack(self):
-        for W, pk in zip(self.Ws, self.packs):
-            awq.quantize_pack(W, self.s_best, self.g, self.zero_point, out=pk)
+        for m, (W, pk) in enumerate(zip(self.Ws, self.packs)):
+            awq.quantize_pack(W, self.s_best, self.g, self.zero_point, out=pk,
+                              clip_idx=self.clips[m][0] if self.n_clip > 0 else None)
 
     def run(self, ws: "Workspaces"):
         self.stats(ws.stats)
         self.search(ws.search)
+        if self.n_clip > 0:
+            self.clip(ws.clip)
         self.pack()
 
 
@@ -126,10 +145,13 @@ class Workspaces:
     concurrently need their own."""
 
     def __init__(self, jobs: Sequence[GroupJob], device):
-        st = max([j.workspace_bytes()[0] for j in jobs] + [1])
-        se = max([j.workspace_bytes()[1] for j in jobs] + [1])
+        sizes = [j.workspace_bytes() for j in jobs]
+        st = max([b[0] for b in sizes] + [1])
+        se = max([b[1] for b in sizes] + [1])
+        cl = max([b[2] for b in sizes] + [1])
         self.stats = torch.empty(st, dtype=torch.uint8, device=device)
         self.search = torch.empty(se, dtype=torch.uint8, device=device)
+        self.clip = torch.empty(cl, dtype=torch.uint8, device=device)
 
 
 def _pinned_like(t: torch.Tensor) -> torch.Tensor:
@@ -148,7 +170,8 @@ class LayerStreamer:
     """
 
     def __init__(self, template, device, group_size: int = 128, n_grid: int = 20,
-                 output_mode: bool = False, zero_point: int = 8, depth: int = 2):
+                 output_mode: bool = False, zero_point: int = 8, depth: int = 2,
+                 n_clip: int = 0):
         self.device = torch.device(device)
         self.depth = depth
         self.slots = []
@@ -157,7 +180,8 @@ class LayerStreamer:
             for Ws, X in template:
                 dWs = [torch.empty(W.shape, dtype=torch.float16, device=self.device) for W in Ws]
                 dX = torch.empty(X.shape, dtype=torch.float16, device=self.device)
-                jobs.append(GroupJob(dWs, dX, group_size, n_grid, output_mode, zero_point))
+                jobs.append(GroupJob(dWs, dX, group_size, n_grid, output_mode, zero_point,
+                                     n_clip))
             self.slots.append(jobs)
         self.ws = Workspaces(self.slots[0], self.device)
         self.h2d = torch.cuda.Stream(self.device)
@@ -177,17 +201,25 @@ class LayerStreamer:
 
     def host_outputs(self):
         """Pinned host buffers for one layer's results:
-        [(err, best, s_best, [(qweight, scales, qzeros) per member]) per group]."""
-        return [(_pinned_like(j.err), _pinned_like(j.best), _pinned_like(j.s_best),
-                 [tuple(_pinned_like(t) for t in pk) for pk in j.packs])
-                for j in self.slots[0]]
+        [(err, best, s_best, [(qweight, scales, qzeros[, clip_idx]) per member])
+        per group]."""
+        out = []
+        for j in self.slots[0]:
+            packs = []
+            for m, pk in enumerate(j.packs):
+                ts = list(pk) + ([j.clips[m][0]] if j.n_clip > 0 else [])
+                packs.append(tuple(_pinned_like(t) for t in ts))
+            out.append((_pinned_like(j.err), _pinned_like(j.best), _pinned_like(j.s_best),
+                        packs))
+        return out
 
     def bytes_per_layer(self) -> Tuple[int, int]:
         """(host-to-device, device-to-host) bytes copied per layer."""
         jobs = self.slots[0]
         h2d = sum(j.X.numel() * 2 + sum(W.numel() * 2 for W in j.Ws) for j in jobs)
         d2h = sum(j.err.numel() * 8 + 4 + j.s_best.numel() * 4 +
-                  sum(t.numel() * t.element_size() for pk in j.packs for t in pk)
+                  sum(t.numel() * t.element_size() for pk in j.packs for t in pk) +
+                  sum(c[0].numel() for c in j.clips)
                   for j in jobs)
         return h2d, d2h
 
@@ -221,8 +253,9 @@ class LayerStreamer:
                     err.copy_(job.err, non_blocking=True)
                     best.copy_(job.best, non_blocking=True)
                     s_best.copy_(job.s_best, non_blocking=True)
-                    for pk_h, pk in zip(packs, job.packs):
-                        for th, t in zip(pk_h, pk):
+                    for m, (pk_h, pk) in enumerate(zip(packs, job.packs)):
+                        src = list(pk) + ([job.clips[m][0]] if job.n_clip > 0 else [])
+                        for th, t in zip(pk_h, src):
                             th.copy_(t, non_blocking=True)
             self.drained[k].record(self.d2h)
         cur = torch.cuda.current_stream(self.device)

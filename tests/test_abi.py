@@ -123,11 +123,16 @@ def test_pipeline_workspace_sizes_from_host_query():
     Ws = [torch.zeros(256, 512, dtype=torch.float16), torch.zeros(128, 512, dtype=torch.float16)]
     X = torch.zeros(64, 512, dtype=torch.float16)
     j = pipeline.GroupJob(Ws, X, 128, 20)
-    st, se = j.workspace_bytes()
-    assert st >= 0 and se > 0
+    st, se, cl = j.workspace_bytes()
+    assert st >= 0 and se > 0 and cl == 0
     jo = pipeline.GroupJob(Ws[:1], X, 128, 20, output_mode=True)
-    st_o, se_o = jo.workspace_bytes()
+    st_o, se_o, _ = jo.workspace_bytes()
     assert se_o >= 2 * 256 * 512 * 2            # the hi/lo dW buffer at least
-    assert j.launches == 1 + 3 + 2 and jo.launches == 1 + 43 + 1
-    ws = pipeline.Workspaces([j, jo], "cpu")
+    jc = pipeline.GroupJob(Ws, X, 128, 20, n_clip=10)
+    assert jc.workspace_bytes()[2] > 0
+    # stats 1; search 2 (table, search); output mode 1 + 2 * 20 + 1; clip 1 per member;
+    # pack 1 per member
+    assert j.launches == 1 + 2 + 2 and jo.launches == 1 + 42 + 1
+    assert jc.launches == 1 + 2 + 2 + 2
+    ws = pipeline.Workspaces([j, jo, jc], "cpu")
     assert ws.search.numel() == max(se, se_o)

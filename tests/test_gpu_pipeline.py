@@ -98,3 +98,38 @@ def test_stack36_layer_full_parity():
         got = (j.x.cpu().numpy(), j.err.cpu().numpy(), int(j.best.cpu()[0]),
                j.s_best.cpu().numpy(), [tuple(t.cpu().numpy() for t in pk) for pk in j.packs])
         _compare(got, [W.numpy() for W in Ws], X.numpy(), 128, work.n_grid, False)
+
+
+def test_layer_streamer_with_clip_search():
+    """Three layers streamed with the clip search on: for every member the
+    clip indices agree with the oracle at the chosen scale (ties within 1e-6
+    exempt) and the packed output equals the oracle's pack of those indices."""
+    g, n_grid, n_clip = 128, 20, 10
+    layers = [_small_layer(2000 + 10 * l) for l in range(3)]
+    host = [[([W.pin_memory() for W in Ws], X.pin_memory()) for Ws, X in lay]
+            for lay in layers]
+    st = pipeline.LayerStreamer(layers[0], "cuda", g, n_grid, False, n_clip=n_clip)
+    out = [st.host_outputs() for _ in range(3)]
+    st.run(host, out)
+    torch.cuda.synchronize()
+    for lay, res in zip(layers, out):
+        for (Ws, X), (err, best, s, packs) in zip(lay, res):
+            x = oracle.act_stats(X.numpy())
+            err_o, best_o, s_o = oracle.scale_search([W.numpy() for W in Ws], x, g, n_grid)
+            assert int(best[0]) == best_o
+            assert np.array_equal(s.numpy(), s_o)
+            for W, pk in zip(Ws, packs):
+                qw, sc, qz, idx = (t.numpy() for t in pk)
+                idx_o, _ = oracle.clip_search(W.numpy(), x, s_o, g, n_clip)
+                Wf = W.numpy().astype(np.float32)
+                for r, k in np.argwhere(idx != idx_o):
+                    sl = slice(k * g, (k + 1) * g)
+                    e1 = oracle.clip_group_error(Wf[r, sl], s_o[sl], x[sl],
+                                                 oracle.clip_ratio(idx[r, k]))
+                    e2 = oracle.clip_group_error(Wf[r, sl], s_o[sl], x[sl],
+                                                 oracle.clip_ratio(idx_o[r, k]))
+                    assert abs(e1 - e2) <= TIE_RTOL * e2
+                qw_o, sc_o, qz_o = oracle.quantize_pack(W.numpy(), s_o, g, 8, idx)
+                assert np.array_equal(qw, qw_o)
+                assert np.array_equal(sc.view(np.uint16), sc_o.view(np.uint16))
+                assert np.array_equal(qz, qz_o)
