@@ -38,6 +38,7 @@ def _load():
         lib.orc_weighted_error.restype = f64
         lib.orc_scale_search.argtypes = [i32, p, p, i64, p, i64, i32, i32, p, p, p]
         lib.orc_quantize_pack.argtypes = [p, i64, i64, p, p, i64, i32, p, p, p]
+        lib.orc_geomean_scales.argtypes = [i32, p, i64, p]
         lib.orc_clip_ratio.argtypes = [i32]
         lib.orc_clip_ratio.restype = ctypes.c_float
         lib.orc_fake_quant_group_clip.argtypes = [p, p, i64, i32, ctypes.c_float, p, p]
@@ -138,6 +139,16 @@ def quantize_pack(W, s=None, group_size: int = 128, zero_point: int = 8, clip_id
                               group_size, zero_point, _ptr(qweight),
                               _ptr(scales), _ptr(qzeros))
     return qweight, scales, qzeros
+
+
+def geomean_scales(ss) -> np.ndarray:
+    """Per-channel geometric mean of the member linears' scales (fp32)."""
+    ss = [_f32(x) for x in ss]
+    d_in = ss[0].shape[0]
+    ptrs = (ctypes.c_void_p * len(ss))(*[x.ctypes.data for x in ss])
+    out = np.empty(d_in, np.float32)
+    _load().orc_geomean_scales(len(ss), ptrs, d_in, _ptr(out))
+    return out
 
 
 def clip_ratio(i: int) -> float:

@@ -14,6 +14,9 @@
  *        code" and "Quantization, storage and packing".
  *   [P4] "Weight-Only Quantization: GPTQ and AWQ", section 4 "Tiny example"
  *        and sections 6-9 "Under the hood: the packed format".
+ *   Norm-group scales: [P1] "AutoAWQ / HF-AWQ GEMM on-disk format",
+ *        exporter steps 1-2 (one shared scale per norm group: the geometric
+ *        mean of the member linears' scales, then re-quantisation with it).
  *   Clip search: [P3] "The pipeline end to end", step 5 (an optional search
  *        of a clipping range per output channel that shrinks the
  *        quantisation range); [P5] "AWQ, Reproduced" (the paper also clips
@@ -199,6 +202,28 @@ double orc_weighted_error(const uint16_t *W, int64_t d_out, int64_t d_in,
     for (int64_t r = 0; r < d_out; ++r) total += row_err[r];
     free(row_err);
     return total;
+}
+
+/* ---------------------------------------------------- norm-group scales --
+ * [P1] exporter step 1: the linears that follow one norm (q/k/v; gate/up)
+ * each get their own searched scale s_m; the norm can absorb only one, so
+ * they share the per-channel geometric mean
+ *     s_shared[j] = (prod_m s_m[j])^(1/n)
+ * evaluated as the fp64 product in member order, then sqrt for n = 2 and
+ * pow(., 1/n) otherwise, rounded once to fp32 (n = 1 copies s_0).
+ */
+void orc_geomean_scales(int n, const float *const *s, int64_t d_in, float *out)
+{
+    for (int64_t j = 0; j < d_in; ++j) {
+        if (n == 1) {
+            out[j] = s[0][j];
+            continue;
+        }
+        double p = 1.0;
+        for (int m = 0; m < n; ++m) p *= (double)s[m][j];
+        double r = (n == 2) ? sqrt(p) : pow(p, 1.0 / (double)n);
+        out[j] = (float)r;
+    }
 }
 
 /* ------------------------------------------------------------- clipping --

@@ -474,3 +474,38 @@ def test_clip_pack_matches_clipped_groups():
     b = oracle.quantize_pack(W, s, g, 8)
     for t1, t2 in zip(a, b):
         assert np.array_equal(t1.view(np.uint8), t2.view(np.uint8))
+
+
+# ----------------------------------------------------- norm-group scales --
+# "From-Scratch AWQ INT4 Quantization on Qwen3-8B", exporter steps 1-2: one
+# shared scale per norm group, the geometric mean of the members' scales.
+
+def test_geomean_closed_forms():
+    rng = np.random.default_rng(51)
+    a = np.exp(rng.standard_normal(1000)).astype(np.float32)
+    b = np.exp(rng.standard_normal(1000)).astype(np.float32)
+    assert np.array_equal(oracle.geomean_scales([a]), a)
+    assert np.array_equal(oracle.geomean_scales([a, a]), a)          # sqrt(a^2) = a exactly
+    # (a^3)^(1/3) is within ~1e-16 of the fp32 value a, far inside half an fp32 ulp
+    assert np.array_equal(oracle.geomean_scales([a, a, a]), a)
+    # two members: the correctly rounded sqrt of the exact product
+    two = oracle.geomean_scales([a, b])
+    exact = np.array([math.sqrt(float(x) * float(y)) for x, y in zip(a, b)])
+    assert np.array_equal(two, exact.astype(np.float32))
+    # powers of two pass through: 4 and 16 give 8; 2, 4, 8 give 4
+    assert oracle.geomean_scales([np.float32([4.0]), np.float32([16.0])])[0] == 8.0
+    assert oracle.geomean_scales([np.float32([2.0]), np.float32([4.0]),
+                                  np.float32([8.0])])[0] == np.float32(4.0)
+
+
+def test_geomean_bounds_and_homogeneity():
+    rng = np.random.default_rng(52)
+    ss = [np.exp(rng.standard_normal(500) * 2).astype(np.float32) for _ in range(3)]
+    g = oracle.geomean_scales(ss).astype(np.float64)
+    lo = np.minimum.reduce([x.astype(np.float64) for x in ss])
+    hi = np.maximum.reduce([x.astype(np.float64) for x in ss])
+    am = sum(x.astype(np.float64) for x in ss) / 3
+    assert np.all(g >= lo * (1 - 1e-7)) and np.all(g <= hi * (1 + 1e-7))
+    assert np.all(g <= am * (1 + 1e-7))                               # AM-GM
+    g2 = oracle.geomean_scales([x * np.float32(8.0) for x in ss])     # scaling by 2^3
+    assert np.array_equal(g2, (g * 8).astype(np.float32))
