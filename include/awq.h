@@ -224,6 +224,27 @@ awq_status awq_quantize_pack(const void *W, int64_t d_out, int64_t d_in,
                              void *scales, int32_t *qzeros, void *stream);
 
 /*
+ * One shared scale for the linears that follow one norm ("From-Scratch AWQ
+ * ...", section "AutoAWQ / HF-AWQ GEMM on-disk format", exporter steps 1-2:
+ * the per-linear scales of q/k/v, or of gate/up, are aggregated into one
+ * scale per norm group by their geometric mean, folded into the norm, and
+ * the members are re-quantised with it by awq_quantize_pack):
+ *
+ *   s_shared[j] = (s_0[j] * ... * s_{n-1}[j])^(1/n)
+ *
+ * evaluated as the fp64 product in member order, then sqrt for n = 2 and
+ * pow(., 1/n) otherwise, rounded once to fp32; n = 1 copies s_0.
+ *
+ *   n          1..AWQ_MAX_SEGMENTS member scales
+ *   s          HOST array of n DEVICE pointers, fp32 [d_in] each (each
+ *              normally the s_best of a one-segment awq_scale_search)
+ *   d_in       1..2^24 channels
+ *   s_shared   fp32 [d_in] device output
+ */
+awq_status awq_norm_group_scale(int n, const float *const *s, int64_t d_in,
+                                float *s_shared, void *stream);
+
+/*
  * Per (row, group) clip search at a fixed scale ("AWQ architecture ...",
  * section "The pipeline end to end", step 5: an optional search of a
  * clipping range per output channel that shrinks the quantisation range to

@@ -66,6 +66,9 @@ def lib() -> ctypes.CDLL:
         L.awq_quantize_pack.restype = i32
         L.awq_clip_search.argtypes = [p, i64, i64, p, p, i32, i32, i32, p, p, p, sz, p]
         L.awq_clip_search.restype = i32
+        L.awq_norm_group_scale.argtypes = [i32, p, i64, p, p]
+        L.awq_norm_group_scale.restype = i32
+        L.awq_clip_search.restype = i32
         L.awq_output_error.argtypes = [p, i64, p, i64, i64, p, i32, i32, i32, p, p, p, p, sz, p]
         L.awq_output_error.restype = i32
         _lib = L
@@ -183,6 +186,23 @@ def quantize_pack(W: torch.Tensor, s: Optional[torch.Tensor] = None, group_size:
                                    qz.data_ptr(), _stream(dev)),
            "awq_quantize_pack")
     return qw, sc, qz
+
+
+def norm_group_scale(ss: Sequence[torch.Tensor], out: Optional[torch.Tensor] = None):
+    """Per-channel geometric mean of the member linears' scales (fp32)."""
+    ss = [_cuda(x, torch.float32, "s") for x in ss]
+    d_in = ss[0].shape[0]
+    for x in ss:
+        if x.dim() != 1 or x.shape[0] != d_in:
+            raise ValueError("every scale must be [d_in]")
+    dev = ss[0].device
+    if out is None:
+        out = torch.empty(d_in, dtype=torch.float32, device=dev)
+    n = len(ss)
+    ptrs = (ctypes.c_void_p * n)(*[x.data_ptr() for x in ss])
+    _check(lib().awq_norm_group_scale(n, ptrs, d_in, out.data_ptr(), _stream(dev)),
+           "awq_norm_group_scale")
+    return out
 
 
 def clip_search(W: torch.Tensor, x: torch.Tensor, s: Optional[torch.Tensor] = None,

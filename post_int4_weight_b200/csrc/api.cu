@@ -160,6 +160,24 @@ awq_status awq_quantize_pack(const void* W, int64_t d_out, int64_t d_in, const f
     return AWQ_OK;
 }
 
+awq_status awq_norm_group_scale(int n, const float* const* s, int64_t d_in, float* s_shared,
+                               void* stream) {
+    if (n < 1 || n > AWQ_MAX_SEGMENTS || !s || !s_shared) return AWQ_ERR_INVALID_ARG;
+    if (d_in < 1 || d_in > (int64_t(1) << 24)) return AWQ_ERR_INVALID_ARG;
+    for (int m = 0; m < n; ++m) {
+        if (!s[m]) return AWQ_ERR_INVALID_ARG;
+        if (!aligned16(s[m])) return AWQ_ERR_ALIGNMENT;
+    }
+    if (!aligned16(s_shared)) return AWQ_ERR_ALIGNMENT;
+    DeviceInfo dev;
+    if (note_cuda(query_device(&dev), "device query") != cudaSuccess) return AWQ_ERR_CUDA;
+    if (note_cuda(launch_norm_group_scale(n, s, d_in, s_shared, dev.num_sms,
+                                          static_cast<cudaStream_t>(stream)),
+                  "norm_group_scale launch") != cudaSuccess)
+        return AWQ_ERR_CUDA;
+    return AWQ_OK;
+}
+
 awq_status awq_clip_search(const void* W, int64_t d_out, int64_t d_in, const float* x_mean,
                            const float* s, int group_size, int n_clip, int flags,
                            uint8_t* clip_idx, double* err, void* ws, size_t ws_bytes,

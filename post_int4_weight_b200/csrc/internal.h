@@ -50,6 +50,10 @@ cudaError_t launch_quantize_pack(const void* W, int64_t d_out, int64_t d_in,
                                  int zero_point, int32_t* qweight, void* scales,
                                  int32_t* qzeros, cudaStream_t stream);
 
+// ---- norm-group shared scale
+cudaError_t launch_norm_group_scale(int n, const float* const* s, int64_t d_in, float* out,
+                                    int num_sms, cudaStream_t stream);
+
 // ---- clip search
 size_t clip_search_workspace();
 cudaError_t launch_clip_search(const void* W, int64_t d_out, int64_t d_in, const float* x_mean,

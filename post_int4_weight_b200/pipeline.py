@@ -7,7 +7,9 @@ in the library's kernels through the calls of :mod:`awq`.
 The unit of work is a *search group*: the linears that read one input X
 (q/k/v, gate/up, or a linear alone).  Its path is awq_act_stats on X, the
 scale search (weight-space, or output-space with ``output_mode``) over all
-members at once, optionally a clip search per member (``n_clip`` > 0; the
+members at once -- or, with ``scale_mode="geomean"``, one search per member
+and the geometric mean of their scales (the Qwen3-8B page's exporter steps
+1-2: one scale per norm group) -- optionally a clip search per member (``n_clip`` > 0; the
 architecture page's pipeline step 5), then awq_quantize_pack of every member
 at the chosen scale (and clip ratios)
 ("From-Scratch AWQ INT4 Quantization on Qwen3-8B", pipeline and AWQ scaling
@@ -65,9 +67,11 @@ class GroupJob:
 
     def __init__(self, Ws: Sequence[torch.Tensor], X: torch.Tensor, group_size: int = 128,
                  n_grid: int = 20, output_mode: bool = False, zero_point: int = 8,
-                 n_clip: int = 0):
+                 n_clip: int = 0, scale_mode: str = "joint"):
         if output_mode and len(Ws) != 1:
             raise ValueError("the output-space score takes one linear per call")
+        if scale_mode not in ("joint", "geomean"):
+            raise ValueError("scale_mode is 'joint' or 'geomean'")
         self.Ws = list(Ws)
         self.X = X
         self.g = group_size
@@ -75,11 +79,22 @@ class GroupJob:
         self.output_mode = output_mode
         self.zero_point = zero_point
         self.n_clip = n_clip
+        # geomean with one member is the joint search
+        self.geomean = scale_mode == "geomean" and len(self.Ws) > 1
         dev = X.device
         T, d_in = X.shape
+        M = len(self.Ws)
         self.x = torch.empty(d_in, dtype=torch.float32, device=dev)
-        self.err = torch.empty(n_grid, dtype=torch.float64, device=dev)
-        self.best = torch.empty(1, dtype=torch.int32, device=dev)
+        if self.geomean:
+            # per member: errors, chosen index and scale; s_best is their
+            # geometric mean
+            # (rows padded to 16 bytes: the library wants aligned outputs)
+            self.err = torch.empty(M, (n_grid + 1) // 2 * 2, dtype=torch.float64, device=dev)
+            self.best = torch.empty(M, 4, dtype=torch.int32, device=dev)
+            self.member_s = torch.empty(M, d_in, dtype=torch.float32, device=dev)
+        else:
+            self.err = torch.empty(n_grid, dtype=torch.float64, device=dev)
+            self.best = torch.empty(1, dtype=torch.int32, device=dev)
         self.s_best = torch.empty(d_in, dtype=torch.float32, device=dev)
         G = d_in // group_size
         self.packs = [(torch.empty(d_in, W.shape[0] // 8, dtype=torch.int32, device=dev),
@@ -97,7 +112,12 @@ class GroupJob:
 
     @property
     def launches(self) -> int:
-        search = launches_output_error(self.n_grid) if self.output_mode else LAUNCHES_SEARCH
+        if self.output_mode:
+            search = launches_output_error(self.n_grid)
+        elif self.geomean:
+            search = LAUNCHES_SEARCH * len(self.Ws) + 1
+        else:
+            search = LAUNCHES_SEARCH
         clip = LAUNCHES_CLIP * len(self.Ws) if self.n_clip > 0 else 0
         return LAUNCHES_STATS + search + clip + len(self.Ws)
 
@@ -116,6 +136,13 @@ class GroupJob:
         awq.act_stats(self.X, out=self.x, ws=ws)
 
     def search(self, ws: torch.Tensor):
+        if self.geomean:
+            for m, W in enumerate(self.Ws):
+                awq.scale_search([W], self.x, self.g, self.n_grid,
+                                 out=(self.err[m, :self.n_grid], self.best[m, :1],
+                                      self.member_s[m]), ws=ws)
+            awq.norm_group_scale(list(self.member_s), out=self.s_best)
+            return
         out = (self.err, self.best, self.s_best)
         if self.output_mode:
             awq.output_error(self.X, self.Ws[0], self.x, self.g, self.n_grid, out=out, ws=ws)
@@ -171,7 +198,7 @@ class LayerStreamer:
 
     def __init__(self, template, device, group_size: int = 128, n_grid: int = 20,
                  output_mode: bool = False, zero_point: int = 8, depth: int = 2,
-                 n_clip: int = 0):
+                 n_clip: int = 0, scale_mode: str = "joint"):
         self.device = torch.device(device)
         self.depth = depth
         self.slots = []
@@ -181,7 +208,7 @@ class LayerStreamer:
                 dWs = [torch.empty(W.shape, dtype=torch.float16, device=self.device) for W in Ws]
                 dX = torch.empty(X.shape, dtype=torch.float16, device=self.device)
                 jobs.append(GroupJob(dWs, dX, group_size, n_grid, output_mode, zero_point,
-                                     n_clip))
+                                     n_clip, scale_mode))
             self.slots.append(jobs)
         self.ws = Workspaces(self.slots[0], self.device)
         self.h2d = torch.cuda.Stream(self.device)
@@ -217,7 +244,7 @@ class LayerStreamer:
         """(host-to-device, device-to-host) bytes copied per layer."""
         jobs = self.slots[0]
         h2d = sum(j.X.numel() * 2 + sum(W.numel() * 2 for W in j.Ws) for j in jobs)
-        d2h = sum(j.err.numel() * 8 + 4 + j.s_best.numel() * 4 +
+        d2h = sum(j.err.numel() * 8 + j.best.numel() * 4 + j.s_best.numel() * 4 +
                   sum(t.numel() * t.element_size() for pk in j.packs for t in pk) +
                   sum(c[0].numel() for c in j.clips)
                   for j in jobs)

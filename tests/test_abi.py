@@ -93,6 +93,13 @@ def test_host_validation_without_a_gpu():
     assert L.awq_quantize_pack(fake, 64, 256, None, None, 128, 9, fake, fake, fake, None) == 1
     assert L.awq_quantize_pack(fake, 64, 256, None, None, 48, 8, fake, fake, fake, None) == 2
     assert L.awq_quantize_pack(fake, 64, 256, odd, None, 128, 8, fake, fake, fake, None) == 3
+    # norm_group_scale
+    ptrs1 = (ctypes.c_void_p * 1)(fake)
+    ptrs_odd = (ctypes.c_void_p * 2)(fake, odd)
+    assert L.awq_norm_group_scale(0, ptrs1, 256, fake, None) == 1
+    assert L.awq_norm_group_scale(9, ptrs1, 256, fake, None) == 1
+    assert L.awq_norm_group_scale(2, ptrs_odd, 256, fake, None) == 3
+    assert L.awq_norm_group_scale(1, ptrs1, 256, odd, None) == 3
     # clip_search
     assert L.awq_clip_search(fake, 64, 256, fake, None, 128, 0, 0, fake, fake, fake,
                              1 << 20, None) == 1

@@ -133,3 +133,45 @@ def test_layer_streamer_with_clip_search():
                 assert np.array_equal(qw, qw_o)
                 assert np.array_equal(sc.view(np.uint16), sc_o.view(np.uint16))
                 assert np.array_equal(qz, qz_o)
+
+
+def test_norm_group_geomean_kernel_bit_exact():
+    from post_int4_weight_b200 import awq
+    rng = np.random.default_rng(61)
+    for n in (1, 2, 3, 5, 8):
+        ss = [np.exp(rng.standard_normal(4096) * 3).astype(np.float32) for _ in range(n)]
+        ss[0][:4] = [1e-30, 1e30, 1.0, 3.0e-8]          # extremes of the fp32 range
+        g = awq.norm_group_scale([torch.from_numpy(x).cuda() for x in ss])
+        torch.cuda.synchronize()
+        assert np.array_equal(g.cpu().numpy(), oracle.geomean_scales(ss)), n
+
+
+def test_norm_group_mode_qkv_block_group():
+    """The Qwen3-8B q/k/v group (4096 + 1024 + 1024 rows x 4096, 16384 tokens)
+    in geomean mode: per-member searches, the shared scale and the three
+    re-quantised linears against the oracle."""
+    work = wl.WORKLOADS["qwen3_8b_block"]
+    grp, Ws, X = wl.group_inputs(work)[0]
+    dev = torch.device("cuda")
+    job = pipeline.GroupJob([W.to(dev) for W in Ws], X.to(dev), 128, 20, scale_mode="geomean")
+    job.run(pipeline.Workspaces([job], dev))
+    torch.cuda.synchronize()
+    x = oracle.act_stats(X.numpy())
+    assert np.array_equal(job.x.cpu().numpy(), x)
+    ss = []
+    for m, W in enumerate(Ws):
+        err_o, best_o, s_o = oracle.scale_search([W.numpy()], x, 128, 20)
+        np.testing.assert_allclose(job.err[m, :20].cpu().numpy(), err_o, rtol=ERR_RTOL, atol=0)
+        b = int(job.best[m, 0].cpu())
+        if b != best_o:
+            assert abs(err_o[b] - err_o[best_o]) <= TIE_RTOL * err_o[best_o]
+            s_o = oracle.scale_table(x, 20)[b]        # follow the GPU's tie choice
+        assert np.array_equal(job.member_s[m].cpu().numpy(), s_o)
+        ss.append(s_o)
+    s_shared = oracle.geomean_scales(ss)
+    assert np.array_equal(job.s_best.cpu().numpy(), s_shared)
+    for W, pk in zip(Ws, job.packs):
+        qw_o, sc_o, qz_o = oracle.quantize_pack(W.numpy(), s_shared, 128, 8)
+        assert np.array_equal(pk[0].cpu().numpy(), qw_o)
+        assert np.array_equal(pk[1].cpu().numpy().view(np.uint16), sc_o.view(np.uint16))
+        assert np.array_equal(pk[2].cpu().numpy(), qz_o)
