@@ -19,6 +19,7 @@ import numpy as np
 from . import build as _build
 
 SCALE_FP32 = 1  # keep the group scale unrounded (fp32) instead of fp16
+DUO = 2         # duo scaling candidates in the scale search
 
 _lib = None
 
@@ -39,6 +40,8 @@ def _load():
         lib.orc_scale_search.argtypes = [i32, p, p, i64, p, i64, i32, i32, p, p, p]
         lib.orc_quantize_pack.argtypes = [p, i64, i64, p, p, i64, i32, p, p, p]
         lib.orc_geomean_scales.argtypes = [i32, p, i64, p]
+        lib.orc_weight_mean.argtypes = [i32, p, p, i64, p]
+        lib.orc_scale_table_duo.argtypes = [p, p, i64, i32, p]
         lib.orc_clip_ratio.argtypes = [i32]
         lib.orc_clip_ratio.restype = ctypes.c_float
         lib.orc_fake_quant_group_clip.argtypes = [p, p, i64, i32, ctypes.c_float, p, p]
@@ -139,6 +142,26 @@ def quantize_pack(W, s=None, group_size: int = 128, zero_point: int = 8, clip_id
                               group_size, zero_point, _ptr(qweight),
                               _ptr(scales), _ptr(qzeros))
     return qweight, scales, qzeros
+
+
+def weight_mean(Ws) -> np.ndarray:
+    """Duo scaling's per-channel mean of |w| / (row max |w|), fp64 [d_in]."""
+    Ws = [_f16(W) for W in Ws]
+    d_in = Ws[0].shape[1]
+    ptrs = (ctypes.c_void_p * len(Ws))(*[W.ctypes.data for W in Ws])
+    d_out = (ctypes.c_int64 * len(Ws))(*[W.shape[0] for W in Ws])
+    out = np.empty(d_in, np.float64)
+    _load().orc_weight_mean(len(Ws), ptrs, d_out, d_in, _ptr(out))
+    return out
+
+
+def scale_table_duo(x, w_mean, n_grid: int = 20) -> np.ndarray:
+    """Duo scale table S[i, j] (fp32) from x and the fp64 weight mean."""
+    x = _f32(x)
+    w_mean = np.ascontiguousarray(w_mean, dtype=np.float64)
+    S = np.empty((n_grid, x.shape[0]), np.float32)
+    _load().orc_scale_table_duo(_ptr(x), _ptr(w_mean), x.shape[0], n_grid, _ptr(S))
+    return S
 
 
 def geomean_scales(ss) -> np.ndarray:

@@ -14,6 +14,9 @@
  *        code" and "Quantization, storage and packing".
  *   [P4] "Weight-Only Quantization: GPTQ and AWQ", section 4 "Tiny example"
  *        and sections 6-9 "Under the hood: the packed format".
+ *   Duo scaling: [P3] "The scale search as code" (with duo scaling the
+ *        candidate is also divided by the mean normalised weight magnitude
+ *        raised to 1 - r).
  *   Norm-group scales: [P1] "AutoAWQ / HF-AWQ GEMM on-disk format",
  *        exporter steps 1-2 (one shared scale per norm group: the geometric
  *        mean of the member linears' scales, then re-quantisation with it).
@@ -45,6 +48,7 @@
 #include <string.h>
 
 #define ORC_SCALE_FP32 1   /* flag: keep the group scale unrounded (fp32) */
+#define ORC_DUO 2          /* flag: duo scaling candidates (see orc_scale_table_duo) */
 
 /* ---------------------------------------------------------------- fp16 -- */
 
@@ -161,6 +165,61 @@ int orc_fake_quant_group(const float *w, const float *s, int64_t n, int flags,
     }
     *q_scale = qs;
     return 0;
+}
+
+/* ---------------------------------------------------------- duo scaling --
+ * [P3] "The scale search as code", duo scaling: per input channel the mean,
+ * over every row of the concatenated member linears, of |w| divided by its
+ * row's largest |w|:
+ *     w_mean[j] = (1 / R) sum_r |W[r, j]| / max_k |W[r, k]|
+ * each quotient correctly rounded in fp64 (an all-zero row contributes 0),
+ * summed in fp64 in segment and row order.
+ */
+void orc_weight_mean(int n_seg, const uint16_t *const *W, const int64_t *d_out, int64_t d_in,
+                     double *w_mean)
+{
+    int64_t rows = 0;
+    for (int64_t j = 0; j < d_in; ++j) w_mean[j] = 0.0;
+    for (int k = 0; k < n_seg; ++k) {
+        for (int64_t r = 0; r < d_out[k]; ++r) {
+            const uint16_t *row = W[k] + r * d_in;
+            double mx = 0.0;
+            for (int64_t j = 0; j < d_in; ++j) {
+                double a = fabs((double)h2f(row[j]));
+                if (a > mx) mx = a;
+            }
+            for (int64_t j = 0; j < d_in; ++j)
+                w_mean[j] += mx > 0.0 ? fabs((double)h2f(row[j])) / mx : 0.0;
+        }
+        rows += d_out[k];
+    }
+    for (int64_t j = 0; j < d_in; ++j) w_mean[j] /= (double)rows;
+}
+
+/* Duo scale table ([P3] "The scale search as code"): for r = i / n_grid
+ *     s[j] = x[j]^r / (w_mean[j]^(1 - r) + 1e-4),  then max(s, 1e-4),
+ *     S[i][j] = s[j] / sqrt(max_j s * min_j s)
+ * in fp64 (x as given, the clamp on s as the page writes it), rounded once
+ * to fp32. */
+void orc_scale_table_duo(const float *x, const double *w_mean, int64_t d_in, int n_grid,
+                         float *S)
+{
+    double *sd = (double *)malloc((size_t)d_in * sizeof(double));
+    for (int i = 0; i < n_grid; ++i) {
+        double r = (double)i / (double)n_grid;
+        double mx = -INFINITY, mn = INFINITY;
+        for (int64_t j = 0; j < d_in; ++j) {
+            double v = pow((double)x[j], r) / (pow(w_mean[j], 1.0 - r) + 1e-4);
+            if (v < 1e-4) v = 1e-4;
+            sd[j] = v;
+            if (v > mx) mx = v;
+            if (v < mn) mn = v;
+        }
+        double norm = sqrt(mx * mn);
+        for (int64_t j = 0; j < d_in; ++j)
+            S[(int64_t)i * d_in + j] = (float)(sd[j] / norm);
+    }
+    free(sd);
 }
 
 /* ------------------------------------------------- weight-space scoring --
@@ -347,15 +406,23 @@ void orc_clip_search(const uint16_t *W, int64_t d_out, int64_t d_in, const float
  * [P3] "The scale search as code" + [P1] "AWQ scaling": for every grid
  * index i the error of every weight segment that shares the input x is
  * summed; the first index with the smallest error wins (strict '<', so the
- * smallest alpha wins a tie).  s_best receives that row of the scale table.
- * best = -1 (and s_best NaN) when any error is not finite.
+ * smallest alpha wins a tie).  s_best receives that row of the scale table
+ * (the duo table with ORC_DUO in flags).  best = -1 (and s_best NaN) when
+ * any error is not finite.
  */
 void orc_scale_search(int n_seg, const uint16_t *const *W, const int64_t *d_out,
                       int64_t d_in, const float *x, int64_t g, int n_grid,
                       int flags, double *err, int32_t *best, float *s_best)
 {
     float *S = (float *)malloc((size_t)n_grid * (size_t)d_in * sizeof(float));
-    orc_scale_table(x, d_in, n_grid, S);
+    if (flags & ORC_DUO) {
+        double *wm = (double *)malloc((size_t)d_in * sizeof(double));
+        orc_weight_mean(n_seg, W, d_out, d_in, wm);
+        orc_scale_table_duo(x, wm, d_in, n_grid, S);
+        free(wm);
+    } else {
+        orc_scale_table(x, d_in, n_grid, S);
+    }
     for (int i = 0; i < n_grid; ++i) {
         double e = 0.0;
         for (int k = 0; k < n_seg; ++k)

@@ -509,3 +509,59 @@ def test_geomean_bounds_and_homogeneity():
     assert np.all(g <= am * (1 + 1e-7))                               # AM-GM
     g2 = oracle.geomean_scales([x * np.float32(8.0) for x in ss])     # scaling by 2^3
     assert np.array_equal(g2, (g * 8).astype(np.float32))
+
+
+# ------------------------------------------------------------ duo scaling --
+# "AWQ architecture, in depth", section "The scale search as code": with duo
+# scaling the candidate is x^r / (w_mean^(1-r) + 1e-4), w_mean the mean over
+# rows of |w| divided by its row's largest |w|; clamped at 1e-4, normalised.
+
+def test_weight_mean_closed_forms():
+    W = np.array([[1, 0.5, 0.25, 1], [2, 2, 1, 0.5]], np.float16)
+    # rows divided by their maxima 1 and 2: [1, .5, .25, 1] and [1, 1, .5, .25]
+    assert np.array_equal(oracle.weight_mean([W]), np.array([1, 0.75, 0.375, 0.625]))
+    # split into two segments: the same rows, the same mean
+    assert np.array_equal(oracle.weight_mean([W[:1], W[1:]]), np.array([1, 0.75, 0.375, 0.625]))
+    # an all-zero row adds 0 to every channel and counts as a row
+    Z = np.vstack([W, np.zeros((1, 4), np.float16)])
+    assert np.array_equal(oracle.weight_mean([Z]), np.array([1, 0.75, 0.375, 0.625]) * 2 / 3)
+
+
+def test_weight_mean_row_scaling_invariance():
+    """Each row is divided by its own maximum, so scaling rows by powers of
+    two leaves w_mean unchanged (and signs do not matter).  Scaling up only:
+    that is exact in fp16 for every value, subnormals included."""
+    rng = np.random.default_rng(71)
+    W = (rng.standard_normal((32, 256)) * 0.02).astype(np.float16)
+    f = (2.0 ** rng.integers(0, 4, size=(32, 1))) * np.where(rng.random((32, 1)) > 0.5, 1, -1)
+    W2 = (W.astype(np.float32) * f).astype(np.float16)
+    assert np.array_equal(oracle.weight_mean([W]), oracle.weight_mean([W2]))
+
+
+def test_duo_table_r0_closed_form_and_constant_weights():
+    x = np.array([0.5, 2.0, 8.0, 1e-6], np.float32)
+    wm = np.array([1, 0.75, 0.375, 0.625])
+    S = oracle.scale_table_duo(x, wm, 20)
+    s0 = [max(1.0 / (w + 1e-4), 1e-4) for w in wm]        # r = 0: x^0 = 1
+    norm = math.sqrt(max(s0) * min(s0))
+    assert np.array_equal(S[0], np.array([v / norm for v in s0]).astype(np.float32))
+    # every |w| equal: w_mean = 1, the constant 1/(1 + 1e-4) cancels in the
+    # normalisation, leaving the plain table (x well above the clamps)
+    x2 = np.exp(np.random.default_rng(72).standard_normal(300)).astype(np.float32)
+    Sd = oracle.scale_table_duo(x2, np.ones(300), 20)
+    Sp = oracle.scale_table(x2, 20)
+    ulp = np.abs(Sd.view(np.int32).astype(np.int64) - Sp.view(np.int32).astype(np.int64))
+    assert ulp.max() <= 1
+
+
+def test_duo_search_uses_duo_table():
+    rng = np.random.default_rng(73)
+    W = (rng.standard_normal((48, 256)) * 0.02).astype(np.float16)
+    X = (rng.standard_normal((64, 256)) * np.exp(rng.standard_normal(256))).astype(np.float16)
+    x = oracle.act_stats(X)
+    err, best, s = oracle.scale_search([W], x, 128, 20, oracle.DUO)
+    S = oracle.scale_table_duo(x, oracle.weight_mean([W]), 20)
+    assert np.array_equal(s, S[best])
+    for i in (0, best, 19):
+        assert math.isclose(err[i], oracle.weighted_error(W, x, S[i], 128), rel_tol=1e-12)
+    assert err[best] == err.min() and best == int(np.argmin(err))
