@@ -82,6 +82,8 @@ def _args():
     ap.add_argument("--scale-mode", choices=["joint", "geomean"], default="joint",
                     help="joint: one search over a shared-input group's linears; geomean: "
                          "one search per linear, then their geometric mean (norm group)")
+    ap.add_argument("--duo", action="store_true",
+                    help="duo scaling candidates (weights' row-normalised mean) in the search")
     ap.add_argument("--clip", type=int, default=0,
                     help="also run the clip search with this many ratios per member "
                          "(0: off, the method's default path)")
@@ -221,7 +223,7 @@ def run_ours(a):
         for Ws, X in li:
             jobs.append(pipeline.GroupJob([W.to(dev) for W in Ws], X.to(dev), g, n_grid,
                                           work.output_mode, n_clip=a.clip,
-                                          scale_mode=a.scale_mode))
+                                          scale_mode=a.scale_mode, duo=a.duo))
     if work.layers == 1:
         host_layer = [([W.pin_memory() for W in Ws], X.pin_memory()) for Ws, X in layer_inputs[0]]
     else:
@@ -323,7 +325,7 @@ def run_ours(a):
     # --- end to end: the same work streamed from pinned host memory
     template = layer_inputs[0]
     streamer = pipeline.LayerStreamer(template, dev, g, n_grid, work.output_mode,
-                                      n_clip=a.clip, scale_mode=a.scale_mode)
+                                      n_clip=a.clip, scale_mode=a.scale_mode, duo=a.duo)
     if work.layers == 1:
         n_e2e = max(5, min(50, a.steps // 20))
         host_layers = [host_layer] * n_e2e
@@ -434,7 +436,7 @@ def run_ours(a):
         "data": "synthetic",
         "config": {"workload": a.workload, "layers": work.layers, "tokens": work.tokens,
                    "group_size": g, "n_grid": n_grid, "n_clip": a.clip,
-                   "scale_mode": a.scale_mode,
+                   "scale_mode": a.scale_mode, "duo": a.duo,
                    "params_per_step": _total_params(work, world, params),
                    "params_rank0": params,
                    "l2": ("flushed (256 MB write) between timed steps" if flush_l2 else
@@ -449,7 +451,8 @@ def run_ours(a):
         "launch": "CUDA graph per step" if not a.no_graph else "eager",
     }
     if world == 1 and not a.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(work, g, a.cpu_seconds, a.clip, a.scale_mode)
+        out["cpu_baseline"] = cpu_baseline(work, g, a.cpu_seconds, a.clip, a.scale_mode,
+                                           a.duo)
     print(json.dumps(out), flush=True)
     if world > 1:
         dist.destroy_process_group()
@@ -499,23 +502,25 @@ def oracle_sample(work, g, row_cap=256, out_rows=16, out_tokens=None):
     return out, params, "; ".join(parts) + f" ({mode})"
 
 
-def _oracle_pass(sample, g, n_grid, output_mode, n_clip=0, scale_mode="joint"):
+def _oracle_pass(sample, g, n_grid, output_mode, n_clip=0, scale_mode="joint", duo=False):
     import oracle
+    fl = oracle.DUO if duo else 0
     for Ws, X in sample:
         x = oracle.act_stats(X)
         if output_mode:
             err = oracle.output_error(X, Ws[0], x, g, n_grid)
             s = oracle.scale_table(x, n_grid)[int(err.argmin())]
         elif scale_mode == "geomean" and len(Ws) > 1:
-            s = oracle.geomean_scales([oracle.scale_search([W], x, g, n_grid)[2] for W in Ws])
+            s = oracle.geomean_scales([oracle.scale_search([W], x, g, n_grid, fl)[2]
+                                       for W in Ws])
         else:
-            err, best, s = oracle.scale_search(Ws, x, g, n_grid)
+            err, best, s = oracle.scale_search(Ws, x, g, n_grid, fl)
         for W in Ws:
             idx = oracle.clip_search(W, x, s, g, n_clip)[0] if n_clip > 0 else None
             oracle.quantize_pack(W, s, g, 8, idx)
 
 
-def cpu_baseline(work, g, seconds, n_clip=0, scale_mode="joint"):
+def cpu_baseline(work, g, seconds, n_clip=0, scale_mode="joint", duo=False):
     """Passes of the CPU oracle over a bounded sample of the workload until
     `seconds` have elapsed."""
     import oracle
@@ -525,7 +530,7 @@ def cpu_baseline(work, g, seconds, n_clip=0, scale_mode="joint"):
     n = 0
     t0 = time.perf_counter()
     while True:
-        _oracle_pass(sample, g, work.n_grid, work.output_mode, n_clip, scale_mode)
+        _oracle_pass(sample, g, work.n_grid, work.output_mode, n_clip, scale_mode, duo)
         n += 1
         if time.perf_counter() - t0 >= seconds:
             break
@@ -548,10 +553,10 @@ def run_reference(a):
     if a.clip > 0:
         text += f" + {a.clip}-ratio clip search"
     for _ in range(max(a.warmup, 3)):
-        _oracle_pass(sample, g, work.n_grid, work.output_mode, a.clip, a.scale_mode)
+        _oracle_pass(sample, g, work.n_grid, work.output_mode, a.clip, a.scale_mode, a.duo)
     t0 = time.perf_counter()
     for _ in range(a.steps):
-        _oracle_pass(sample, g, work.n_grid, work.output_mode, a.clip, a.scale_mode)
+        _oracle_pass(sample, g, work.n_grid, work.output_mode, a.clip, a.scale_mode, a.duo)
     dt = time.perf_counter() - t0
     v = a.steps * params / dt / 1e9
     print(json.dumps({
@@ -561,7 +566,7 @@ def run_reference(a):
         "vs_baseline": None, "dtype": "f64" if work.output_mode else "f32",
         "data": "synthetic", "config": {"workload": a.workload, "group_size": g,
                                         "n_grid": work.n_grid, "n_clip": a.clip,
-                                        "scale_mode": a.scale_mode},
+                                        "scale_mode": a.scale_mode, "duo": a.duo},
         "cpu_baseline": {"value": v, "unit": UNIT, "cores": oracle.threads(),
                          "kind": "oracle", "sample": f"per step, one pass over {text}"},
         "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},

@@ -53,15 +53,22 @@ typedef enum awq_status {
     AWQ_ERR_NONFINITE = 6      /* reserved: non-finite data (see outputs)      */
 } awq_status;
 
-/* Flags of awq_scale_search / awq_output_error. */
+/* Flags of awq_scale_search / awq_output_error / awq_clip_search. */
 #define AWQ_SCALE_FP16 0  /* group scale rounded to fp16 (the stored format) */
 #define AWQ_SCALE_FP32 1  /* group scale kept in fp32 (the worked example)  */
+/* awq_scale_search only: duo scaling candidates ("AWQ architecture ...",
+ * section "The scale search as code"): s_i = max(x^r / (w_mean^(1-r) +
+ * 1e-4), 1e-4), normalised as usual, with w_mean[j] the mean over every row
+ * of the segments of |W[r, j]| / max_k |W[r, k]| (fp64); needs
+ * d_in <= 16384 and the AWQ_OP_SCALE_SEARCH_DUO workspace. */
+#define AWQ_DUO_SCALING 2
 
 /* Operation ids of awq_workspace_size. */
 #define AWQ_OP_ACT_STATS    0
 #define AWQ_OP_SCALE_SEARCH 1
 #define AWQ_OP_OUTPUT_ERROR 2
 #define AWQ_OP_CLIP_SEARCH  3
+#define AWQ_OP_SCALE_SEARCH_DUO 4   /* awq_scale_search with AWQ_DUO_SCALING */
 
 /* Clip ratios: index i stands for c_i = (AWQ_CLIP_DEN - i) / AWQ_CLIP_DEN
  * rounded to fp32; 0 is no clipping, at most AWQ_CLIP_MAX ratios. */

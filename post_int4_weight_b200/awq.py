@@ -22,6 +22,8 @@ OP_ACT_STATS = 0
 OP_SCALE_SEARCH = 1
 OP_OUTPUT_ERROR = 2
 OP_CLIP_SEARCH = 3
+OP_SCALE_SEARCH_DUO = 4
+DUO_SCALING = 2
 CLIP_DEN = 20
 MAX_SEGMENTS = 8
 
@@ -148,7 +150,8 @@ def scale_search(Ws: Sequence[torch.Tensor], x: torch.Tensor, group_size: int = 
                torch.empty(d_in, dtype=torch.float32, device=dev))
     err, best, s_best = out
     if ws is None:
-        ws = workspace(OP_SCALE_SEARCH, dev, 1, 8, d_in, group_size, n_grid)
+        op = OP_SCALE_SEARCH_DUO if flags & DUO_SCALING else OP_SCALE_SEARCH
+        ws = workspace(op, dev, 1, 8, d_in, group_size, n_grid)
     n = len(Ws)
     ptrs = (ctypes.c_void_p * n)(*[W.data_ptr() for W in Ws])
     d_out = (ctypes.c_int64 * n)(*[W.shape[0] for W in Ws])

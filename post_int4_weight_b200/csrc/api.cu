@@ -84,6 +84,12 @@ awq_status awq_workspace_size(int op, int64_t T, int64_t d_out_total, int64_t d_
             if (!valid_group(group_size) || n_grid < 1 || n_grid > 32) return AWQ_ERR_INVALID_ARG;
             *bytes = scale_search_workspace(d_in, group_size, n_grid);
             return AWQ_OK;
+        case AWQ_OP_SCALE_SEARCH_DUO:
+            if (!valid_group(group_size) || n_grid < 1 || n_grid > 32 || d_in > kDuoMaxDin)
+                return AWQ_ERR_INVALID_ARG;
+            *bytes = scale_search_workspace(d_in, group_size, n_grid) +
+                     duo_workspace_bound(d_in, n_grid);
+            return AWQ_OK;
         case AWQ_OP_CLIP_SEARCH:
             if (!valid_group(group_size)) return AWQ_ERR_INVALID_ARG;
             *bytes = clip_search_workspace();
@@ -123,7 +129,9 @@ awq_status awq_scale_search(int n_seg, const void* const* W, const int64_t* d_ou
     if (!x_mean || !err || !best_idx || !s_best) return AWQ_ERR_INVALID_ARG;
     if (!valid_group(group_size)) return AWQ_ERR_UNSUPPORTED;
     if (n_grid < 1 || n_grid > 32) return AWQ_ERR_INVALID_ARG;
-    if (flags != AWQ_SCALE_FP16 && flags != AWQ_SCALE_FP32) return AWQ_ERR_INVALID_ARG;
+    if (flags & ~(AWQ_SCALE_FP32 | AWQ_DUO_SCALING)) return AWQ_ERR_INVALID_ARG;
+    const bool duo = (flags & AWQ_DUO_SCALING) != 0;
+    if (duo && d_in > kDuoMaxDin) return AWQ_ERR_UNSUPPORTED;
     if (d_in < group_size || d_in % group_size || d_in > (int64_t(1) << 24))
         return AWQ_ERR_INVALID_ARG;
     for (int k = 0; k < n_seg; ++k) {
@@ -133,8 +141,9 @@ awq_status awq_scale_search(int n_seg, const void* const* W, const int64_t* d_ou
     }
     if (!aligned16(x_mean) || !aligned16(err) || !aligned16(best_idx) || !aligned16(s_best))
         return AWQ_ERR_ALIGNMENT;
-    if (!ws || ws_bytes < scale_search_workspace(d_in, group_size, n_grid))
-        return AWQ_ERR_WORKSPACE;
+    const size_t need = scale_search_workspace(d_in, group_size, n_grid) +
+                        (duo ? duo_workspace_bound(d_in, n_grid) : 0);
+    if (!ws || ws_bytes < need) return AWQ_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(ws) & (kWsAlign - 1)) != 0) return AWQ_ERR_ALIGNMENT;
     return launch_scale_search(n_seg, W, d_out, d_in, x_mean, group_size, n_grid, flags, err,
                                best_idx, s_best, ws, static_cast<cudaStream_t>(stream));

@@ -157,6 +157,20 @@ __device__ __forceinline__ float div_rn_rcp(float a, float b, float y) {
     return __fmaf_rn(r, y, q);
 }
 
+// RN(a / b) in fp64 for finite a >= 0 and b > 0 from y = RN(1 / b): the
+// product a*y is within about one ulp of the quotient, and each residual
+// a - q*b (exact in an FMA) corrects it (Markstein's construction); two
+// corrections give the correctly rounded quotient.  Used for |w| / max|w|
+// of fp16 values, checked against __ddiv_rn for every pair of non-negative
+// fp16 values.
+__device__ __forceinline__ double ddiv_rn_rcp(double a, double b, double y) {
+    double q = __dmul_rn(a, y);
+    double r = __fma_rn(-q, b, a);
+    q = __fma_rn(r, y, q);
+    r = __fma_rn(-q, b, a);
+    return __fma_rn(r, y, q);
+}
+
 // Group scale from the group's largest |w * s| (round-to-nearest-even
 // throughout): fp32 quotient by 7, then fp16 unless fp32 scales are asked
 // for.  An fp16 overflow is held at 65504; a non-finite maximum gives NaN.

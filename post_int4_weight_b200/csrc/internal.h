@@ -50,6 +50,16 @@ cudaError_t launch_quantize_pack(const void* W, int64_t d_out, int64_t d_in,
                                  int zero_point, int32_t* qweight, void* scales,
                                  int32_t* qzeros, cudaStream_t stream);
 
+// ---- duo scaling (the scale table from x and the weights' row-normalised
+// mean); its workspace follows the search workspace
+constexpr int kDuoMaxSms = 160;        // weight-mean CTAs (one per SM, at most this many)
+constexpr int64_t kDuoMaxDin = 16384;  // the weight-mean pass keeps d_in fp64 sums in smem
+size_t duo_workspace(int64_t d_in, int num_sms, int n_grid);
+size_t duo_workspace_bound(int64_t d_in, int n_grid);
+cudaError_t launch_duo_table(int n_seg, const void* const* W, const int64_t* d_out, int64_t d_in,
+                             const float* x_mean, int n_grid, float* S, float* T,
+                             int* dev_words, void* duo_ws, int num_sms, cudaStream_t stream);
+
 // ---- norm-group shared scale
 cudaError_t launch_norm_group_scale(int n, const float* const* s, int64_t d_in, float* out,
                                     int num_sms, cudaStream_t stream);

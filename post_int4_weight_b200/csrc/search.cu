@@ -682,9 +682,16 @@ awq_status launch_scale_search(int n_seg, const void* const* W, const int64_t* d
     if (grid > units) grid = units;
     if (grid > (int64_t)max_search_ctas()) grid = (int64_t)max_search_ctas();
 
-    if (launch_scale_table(x_mean, d_in, n_grid, w.S, w.tau2, w.dev_words, dev.num_sms,
-                           stream, kTableTauSq) != cudaSuccess)
-        return AWQ_ERR_CUDA;
+    cudaError_t te;
+    if (flags & AWQ_DUO_SCALING) {
+        char* duo_ws = static_cast<char*>(ws) + scale_search_workspace(d_in, group_size, n_grid);
+        te = launch_duo_table(n_seg, W, d_out, d_in, x_mean, n_grid, w.S, w.tau2, w.dev_words,
+                              duo_ws, dev.num_sms, stream);
+    } else {
+        te = launch_scale_table(x_mean, d_in, n_grid, w.S, w.tau2, w.dev_words, dev.num_sms,
+                                stream, kTableTauSq);
+    }
+    if (note_cuda(te, "scale table launch") != cudaSuccess) return AWQ_ERR_CUDA;
     const cudaError_t e = (flags & AWQ_SCALE_FP32)
                               ? launch_search<true>(L, p, (int)grid, smem, stream)
                               : launch_search<false>(L, p, (int)grid, smem, stream);

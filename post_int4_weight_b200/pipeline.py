@@ -67,7 +67,7 @@ class GroupJob:
 
     def __init__(self, Ws: Sequence[torch.Tensor], X: torch.Tensor, group_size: int = 128,
                  n_grid: int = 20, output_mode: bool = False, zero_point: int = 8,
-                 n_clip: int = 0, scale_mode: str = "joint"):
+                 n_clip: int = 0, scale_mode: str = "joint", duo: bool = False):
         if output_mode and len(Ws) != 1:
             raise ValueError("the output-space score takes one linear per call")
         if scale_mode not in ("joint", "geomean"):
@@ -79,6 +79,9 @@ class GroupJob:
         self.output_mode = output_mode
         self.zero_point = zero_point
         self.n_clip = n_clip
+        self.flags = awq.DUO_SCALING if duo else awq.SCALE_FP16
+        if duo and output_mode:
+            raise ValueError("duo scaling is a weight-space search option")
         # geomean with one member is the joint search
         self.geomean = scale_mode == "geomean" and len(self.Ws) > 1
         dev = X.device
@@ -114,6 +117,10 @@ class GroupJob:
     def launches(self) -> int:
         if self.output_mode:
             search = launches_output_error(self.n_grid)
+        elif self.flags & awq.DUO_SCALING:
+            # weight mean (2) + duo table (2) + search, per search call
+            n = len(self.Ws) if self.geomean else 1
+            search = 5 * n + (1 if self.geomean else 0)
         elif self.geomean:
             search = LAUNCHES_SEARCH * len(self.Ws) + 1
         else:
@@ -126,7 +133,8 @@ class GroupJob:
         T, d_in = self.X.shape
         d_out = sum(W.shape[0] for W in self.Ws)
         st = awq.workspace_size(awq.OP_ACT_STATS, T, 8, d_in, self.g, self.n_grid)
-        op = awq.OP_OUTPUT_ERROR if self.output_mode else awq.OP_SCALE_SEARCH
+        op = awq.OP_OUTPUT_ERROR if self.output_mode else (
+            awq.OP_SCALE_SEARCH_DUO if self.flags & awq.DUO_SCALING else awq.OP_SCALE_SEARCH)
         se = awq.workspace_size(op, T, d_out, d_in, self.g, self.n_grid)
         cl = awq.workspace_size(awq.OP_CLIP_SEARCH, T, d_out, d_in, self.g, 1) \
             if self.n_clip > 0 else 0
@@ -138,7 +146,7 @@ class GroupJob:
     def search(self, ws: torch.Tensor):
         if self.geomean:
             for m, W in enumerate(self.Ws):
-                awq.scale_search([W], self.x, self.g, self.n_grid,
+                awq.scale_search([W], self.x, self.g, self.n_grid, self.flags,
                                  out=(self.err[m, :self.n_grid], self.best[m, :1],
                                       self.member_s[m]), ws=ws)
             awq.norm_group_scale(list(self.member_s), out=self.s_best)
@@ -147,7 +155,7 @@ class GroupJob:
         if self.output_mode:
             awq.output_error(self.X, self.Ws[0], self.x, self.g, self.n_grid, out=out, ws=ws)
         else:
-            awq.scale_search(self.Ws, self.x, self.g, self.n_grid, out=out, ws=ws)
+            awq.scale_search(self.Ws, self.x, self.g, self.n_grid, self.flags, out=out, ws=ws)
 
     def clip(self, ws: torch.Tensor):
         for W, cl in zip(self.Ws, self.clips):
@@ -198,7 +206,7 @@ class LayerStreamer:
 
     def __init__(self, template, device, group_size: int = 128, n_grid: int = 20,
                  output_mode: bool = False, zero_point: int = 8, depth: int = 2,
-                 n_clip: int = 0, scale_mode: str = "joint"):
+                 n_clip: int = 0, scale_mode: str = "joint", duo: bool = False):
         self.device = torch.device(device)
         self.depth = depth
         self.slots = []
@@ -208,7 +216,7 @@ class LayerStreamer:
                 dWs = [torch.empty(W.shape, dtype=torch.float16, device=self.device) for W in Ws]
                 dX = torch.empty(X.shape, dtype=torch.float16, device=self.device)
                 jobs.append(GroupJob(dWs, dX, group_size, n_grid, output_mode, zero_point,
-                                     n_clip, scale_mode))
+                                     n_clip, scale_mode, duo))
             self.slots.append(jobs)
         self.ws = Workspaces(self.slots[0], self.device)
         self.h2d = torch.cuda.Stream(self.device)

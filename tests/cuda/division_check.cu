@@ -46,26 +46,47 @@ __global__ void check_div_rcp(unsigned long long* bad, uint32_t* first_bad_b) {
     }
 }
 
+// every pair (a, b) of non-negative finite fp16 values with b > 0 (blockIdx.x
+// selects b): ddiv_rn_rcp against the IEEE fp64 quotient __ddiv_rn
+__global__ void check_ddiv_rcp(unsigned long long* bad, uint32_t* first_bad_b) {
+    const uint32_t hb = blockIdx.x + 1;           // 0x0001 .. 0x7bff
+    const double b = (double)__half2float(__ushort_as_half((unsigned short)hb));
+    const double y = __drcp_rn(b);
+    for (uint32_t ha = threadIdx.x; ha <= 0x7bffu; ha += blockDim.x) {
+        const double a = (double)__half2float(__ushort_as_half((unsigned short)ha));
+        const double q = awq::ddiv_rn_rcp(a, b, y);
+        const double r = __ddiv_rn(a, b);
+        if (__double_as_longlong(q) != __double_as_longlong(r)) {
+            atomicAdd(bad, 1ull);
+            atomicMin(first_bad_b, hb);
+        }
+    }
+}
+
 extern "C" int run_checks(unsigned long long* out) {
     // out[0]: div7 mismatches, out[1]: first bad bits, out[2]: div_rcp
-    // mismatches, out[3]: first bad fp16 divisor
+    // mismatches, out[3]: first bad fp16 divisor, out[4]: ddiv_rcp
+    // mismatches, out[5]: its first bad fp16 divisor
     unsigned long long* d_bad;
     uint32_t* d_first;
-    if (cudaMalloc(&d_bad, 2 * sizeof(unsigned long long)) != cudaSuccess) return 1;
-    if (cudaMalloc(&d_first, 2 * sizeof(uint32_t)) != cudaSuccess) return 1;
-    cudaMemset(d_bad, 0, 2 * sizeof(unsigned long long));
-    cudaMemset(d_first, 0xff, 2 * sizeof(uint32_t));
+    if (cudaMalloc(&d_bad, 3 * sizeof(unsigned long long)) != cudaSuccess) return 1;
+    if (cudaMalloc(&d_first, 3 * sizeof(uint32_t)) != cudaSuccess) return 1;
+    cudaMemset(d_bad, 0, 3 * sizeof(unsigned long long));
+    cudaMemset(d_first, 0xff, 3 * sizeof(uint32_t));
     check_div7<<<4096, 256>>>(0u, 0x7f800000u, d_bad, d_first);
     check_div_rcp<<<0x7bff, 256>>>(d_bad + 1, d_first + 1);
+    check_ddiv_rcp<<<0x7bff, 256>>>(d_bad + 2, d_first + 2);
     if (cudaDeviceSynchronize() != cudaSuccess) return 2;
-    unsigned long long h_bad[2];
-    uint32_t h_first[2];
+    unsigned long long h_bad[3];
+    uint32_t h_first[3];
     cudaMemcpy(h_bad, d_bad, sizeof h_bad, cudaMemcpyDeviceToHost);
     cudaMemcpy(h_first, d_first, sizeof h_first, cudaMemcpyDeviceToHost);
     out[0] = h_bad[0];
     out[1] = h_first[0];
     out[2] = h_bad[1];
     out[3] = h_first[1];
+    out[4] = h_bad[2];
+    out[5] = h_first[2];
     cudaFree(d_bad);
     cudaFree(d_first);
     return 0;

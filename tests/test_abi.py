@@ -82,12 +82,18 @@ def test_host_validation_without_a_gpu():
     assert search(n=9) == 1
     assert search(g=96) == 2
     assert search(n_grid=0) == 1 and search(n_grid=33) == 1
-    assert search(flags=2) == 1
+    assert search(flags=4) == 1                      # an unknown flag bit
+    assert search(flags=2, d_in=32768) == 2           # duo scaling: d_in <= 16384
     assert search(d_in=200) == 1
     assert search(W=(ctypes.c_void_p * 1)(odd)) == 3
     assert search(d=(ctypes.c_int64 * 1)(0)) == 1
     assert L.awq_scale_search(1, W, d, 256, fake, 128, 20, 0, fake, fake, fake, fake,
                               16, None) == 4
+    plain = awq.workspace_size(awq.OP_SCALE_SEARCH, 1, 64, 256, 128, 20)
+    duo = awq.workspace_size(awq.OP_SCALE_SEARCH_DUO, 1, 64, 256, 128, 20)
+    assert duo > plain
+    assert L.awq_scale_search(1, W, d, 256, fake, 128, 20, 2, fake, fake, fake, fake,
+                              plain, None) == 4
     # quantize_pack
     assert L.awq_quantize_pack(fake, 12, 256, None, None, 128, 8, fake, fake, fake, None) == 1
     assert L.awq_quantize_pack(fake, 64, 256, None, None, 128, 9, fake, fake, fake, None) == 1
