@@ -20,6 +20,7 @@ from . import build as _build
 
 SCALE_FP32 = 1  # keep the group scale unrounded (fp32) instead of fp16
 DUO = 2         # duo scaling candidates in the scale search
+ASYM = 4        # asymmetric INT4 (16 levels, per-group zero point)
 
 _lib = None
 
@@ -40,6 +41,8 @@ def _load():
         lib.orc_scale_search.argtypes = [i32, p, p, i64, p, i64, i32, i32, p, p, p]
         lib.orc_quantize_pack.argtypes = [p, i64, i64, p, p, i64, i32, p, p, p]
         lib.orc_geomean_scales.argtypes = [i32, p, i64, p]
+        lib.orc_fake_quant_group_asym.argtypes = [p, p, i64, i32, p, p, p]
+        lib.orc_fake_quant_group_asym.restype = i32
         lib.orc_weight_mean.argtypes = [i32, p, p, i64, p]
         lib.orc_scale_table_duo.argtypes = [p, p, i64, i32, p]
         lib.orc_clip_ratio.argtypes = [i32]
@@ -142,6 +145,17 @@ def quantize_pack(W, s=None, group_size: int = 128, zero_point: int = 8, clip_id
                               group_size, zero_point, _ptr(qweight),
                               _ptr(scales), _ptr(qzeros))
     return qweight, scales, qzeros
+
+
+def fake_quant_group_asym(w, s, flags: int = 0):
+    """Asymmetric INT4 of one group: (codes uint8 0..15, q_scale, zero point)."""
+    w, s = _f32(w), _f32(s)
+    q = np.empty(w.shape[0], np.uint8)
+    qs = np.empty(1, np.float32)
+    z = np.empty(1, np.int32)
+    _load().orc_fake_quant_group_asym(_ptr(w), _ptr(s), w.shape[0], flags, _ptr(q), _ptr(qs),
+                                      _ptr(z))
+    return q, float(qs[0]), int(z[0])
 
 
 def weight_mean(Ws) -> np.ndarray:

@@ -14,6 +14,11 @@
  *        code" and "Quantization, storage and packing".
  *   [P4] "Weight-Only Quantization: GPTQ and AWQ", section 4 "Tiny example"
  *        and sections 6-9 "Under the hood: the packed format".
+ *   Asymmetric INT4: [P3] "Quantization, storage and packing" (a 16-bit
+ *        scale and a 4-bit zero point per group and output channel) and
+ *        "The scale search as code" (the worked example: values up to 0.5
+ *        in magnitude give a step of about 1/15 and a worst rounding error
+ *        of about 0.033); the formula is a reading listed in the design doc.
  *   Duo scaling: [P3] "The scale search as code" (with duo scaling the
  *        candidate is also divided by the mean normalised weight magnitude
  *        raised to 1 - r).
@@ -49,6 +54,7 @@
 
 #define ORC_SCALE_FP32 1   /* flag: keep the group scale unrounded (fp32) */
 #define ORC_DUO 2          /* flag: duo scaling candidates (see orc_scale_table_duo) */
+#define ORC_ASYM 4         /* flag: asymmetric INT4 (see orc_fake_quant_group_asym) */
 
 /* ---------------------------------------------------------------- fp16 -- */
 
@@ -222,6 +228,54 @@ void orc_scale_table_duo(const float *x, const double *w_mean, int64_t d_in, int
     free(sd);
 }
 
+/* ------------------------------------------------------- asymmetric INT4 --
+ * 16 levels 0..15 with a per-group zero point (min-max grid):
+ *   ws = fl32(w s);  range = max(fl32(max ws - min ws), 1e-5)
+ *   q_scale = fp16_rne(fl32(range / 15))        (unrounded with ORC_SCALE_FP32)
+ *   zero    = clamp(rint(fl32(-min ws / q_scale)), 0, 15)
+ *   q       = clamp(rint(fl32(ws / q_scale)) + zero, 0, 15)
+ *   w_hat   = (q - zero) q_scale / s
+ * A non-finite group gives q_scale NaN, zero 8 and codes 8 (return 1).
+ */
+int orc_fake_quant_group_asym(const float *w, const float *s, int64_t n, int flags,
+                              uint8_t *q, float *q_scale, int *zero)
+{
+    float mx = -INFINITY, mn = INFINITY;
+    int nonfinite = 0;
+    for (int64_t j = 0; j < n; ++j) {
+        float ws = w[j] * s[j];
+        if (!isfinite(ws)) nonfinite = 1;
+        if (ws > mx) mx = ws;
+        if (ws < mn) mn = ws;
+    }
+    if (nonfinite) {
+        for (int64_t j = 0; j < n; ++j) q[j] = 8;
+        *q_scale = NAN;
+        *zero = 8;
+        return 1;
+    }
+    float range = mx - mn;
+    if (range < 1e-5f) range = 1e-5f;
+    float qs = range / 15.0f;
+    if (!(flags & ORC_SCALE_FP32)) {
+        qs = h2f(f2h(qs));
+        if (isinf(qs)) qs = 65504.0f;
+    }
+    float z = rintf(-mn / qs);
+    if (z < 0.0f) z = 0.0f;
+    if (z > 15.0f) z = 15.0f;
+    for (int64_t j = 0; j < n; ++j) {
+        float ws = w[j] * s[j];
+        float r = rintf(ws / qs) + z;
+        if (r < 0.0f) r = 0.0f;
+        if (r > 15.0f) r = 15.0f;
+        q[j] = (uint8_t)r;
+    }
+    *q_scale = qs;
+    *zero = (int)z;
+    return 0;
+}
+
 /* ------------------------------------------------- weight-space scoring --
  * Activation-weighted reconstruction error of one candidate scale vector s
  * over one weight matrix W[d_out, d_in] (fp16, row-major)
@@ -240,17 +294,23 @@ double orc_weighted_error(const uint16_t *W, int64_t d_out, int64_t d_in,
     for (int64_t r = 0; r < d_out; ++r) {
         float w[g];
         int8_t q[g];
+        uint8_t u[g];
         double acc = 0.0;
         for (int64_t k = 0; k < d_in / g; ++k) {
             const uint16_t *row = W + r * d_in + k * g;
             for (int64_t j = 0; j < g; ++j) w[j] = h2f(row[j]);
             float qs;
-            if (orc_fake_quant_group(w, s + k * g, g, flags, q, &qs)) {
+            int z = 0;
+            int bad = (flags & ORC_ASYM)
+                          ? orc_fake_quant_group_asym(w, s + k * g, g, flags, u, &qs, &z)
+                          : orc_fake_quant_group(w, s + k * g, g, flags, q, &qs);
+            if (bad) {
                 acc = NAN;
                 continue;
             }
             for (int64_t j = 0; j < g; ++j) {
-                double what = (double)q[j] * (double)qs / (double)s[k * g + j];
+                double level = (flags & ORC_ASYM) ? (double)((int)u[j] - z) : (double)q[j];
+                double what = level * (double)qs / (double)s[k * g + j];
                 double e = ((double)w[j] - what) * (double)x[k * g + j];
                 acc += e * e;
             }
@@ -456,6 +516,9 @@ void orc_scale_search(int n_seg, const uint16_t *const *W, const int64_t *d_out,
  *   qzeros[k, c]    = zero_point in all eight nibbles
  * s == NULL means s = 1 (plain round-to-nearest).  clip_idx (or NULL for
  * none) gives each (row, group) a clip ratio index as in orc_clip_search.
+ * zero_point = -1 selects the asymmetric grid: codes 0..15 from
+ * orc_fake_quant_group_asym and qzeros holding each (group, row)'s zero
+ * point in the same nibble order (clip_idx is ignored then).
  * A non-finite group stores code zero_point and scale NaN.
  */
 static const int kOrder[8] = {0, 2, 4, 6, 1, 3, 5, 7};
@@ -470,12 +533,22 @@ void orc_quantize_pack(const uint16_t *W, int64_t d_out, int64_t d_in,
     float *w = (float *)malloc((size_t)g * sizeof(float));
     float *ones = (float *)malloc((size_t)g * sizeof(float));
     int8_t *q = (int8_t *)malloc((size_t)g);
+    uint8_t *ua = (uint8_t *)malloc((size_t)g);
+    uint8_t *zeros = (uint8_t *)malloc((size_t)d_out * (size_t)G);
     for (int64_t j = 0; j < g; ++j) ones[j] = 1.0f;
 
     for (int64_t r = 0; r < d_out; ++r) {
         for (int64_t k = 0; k < G; ++k) {
             for (int64_t j = 0; j < g; ++j) w[j] = h2f(W[r * d_in + k * g + j]);
             float qs;
+            if (zero_point < 0) {
+                int z;
+                orc_fake_quant_group_asym(w, s ? s + k * g : ones, g, 0, ua, &qs, &z);
+                zeros[r * G + k] = (uint8_t)z;
+                for (int64_t j = 0; j < g; ++j) u[r * d_in + k * g + j] = ua[j];
+                scales[k * d_out + r] = isnan(qs) ? (uint16_t)0x7E00 : f2h(qs);
+                continue;
+            }
             if (clip_idx)
                 orc_fake_quant_group_clip(w, s ? s + k * g : ones, g, 0,
                                           orc_clip_ratio(clip_idx[r * G + k]), q, &qs);
@@ -495,10 +568,23 @@ void orc_quantize_pack(const uint16_t *W, int64_t d_out, int64_t d_in,
             qweight[j * C + c] = (int32_t)word;
         }
     }
-    uint32_t zword = 0;
-    for (int p = 0; p < 8; ++p) zword |= (uint32_t)(zero_point & 0xF) << (4 * p);
-    for (int64_t k = 0; k < G; ++k)
-        for (int64_t c = 0; c < C; ++c) qzeros[k * C + c] = (int32_t)zword;
+    if (zero_point < 0) {
+        /* per (group, row) zero points, packed like the codes along rows */
+        for (int64_t k = 0; k < G; ++k)
+            for (int64_t c = 0; c < C; ++c) {
+                uint32_t word = 0;
+                for (int p = 0; p < 8; ++p)
+                    word |= (uint32_t)(zeros[(8 * c + kOrder[p]) * G + k] & 0xF) << (4 * p);
+                qzeros[k * C + c] = (int32_t)word;
+            }
+    } else {
+        uint32_t zword = 0;
+        for (int p = 0; p < 8; ++p) zword |= (uint32_t)(zero_point & 0xF) << (4 * p);
+        for (int64_t k = 0; k < G; ++k)
+            for (int64_t c = 0; c < C; ++c) qzeros[k * C + c] = (int32_t)zword;
+    }
+    free(ua);
+    free(zeros);
     free(u);
     free(w);
     free(ones);

@@ -565,3 +565,105 @@ def test_duo_search_uses_duo_table():
     for i in (0, best, 19):
         assert math.isclose(err[i], oracle.weighted_error(W, x, S[i], 128), rel_tol=1e-12)
     assert err[best] == err.min() and best == int(np.argmin(err))
+
+
+# ------------------------------------------------------- asymmetric INT4 --
+# "AWQ architecture, in depth": a 16-bit scale and a 4-bit zero point per
+# group and output channel; the worked example in "The scale search as code"
+# (values up to 0.5: step about 1/15 = 0.067, worst rounding error about
+# 0.033).  Reading: min-max grid of 16 levels, zero = rint(-min / scale).
+
+def _nearest_int_in(v, lo, hi):
+    """Nearest integer in [lo, hi] to v, ties to even (by enumeration)."""
+    v = float(v)
+    return min(range(lo, hi + 1), key=lambda c: (abs(v - c), c % 2))
+
+
+def test_asym_worked_example_step_and_error():
+    w = np.linspace(-0.5, 0.5, 128).astype(np.float16).astype(np.float32)
+    s = np.ones(128, np.float32)
+    q, qs, z = oracle.fake_quant_group_asym(w, s)
+    assert qs == float(np.float16(np.float32(1.0) / np.float32(15)))   # 0.06665...
+    assert abs(qs - 1 / 15) < 1e-4
+    err = np.abs(w.astype(np.float64) - (q.astype(np.float64) - z) * qs)
+    inside = (q > 0) & (q < 15)
+    assert np.all(err[inside] <= qs / 2 * (1 + 1e-6))
+    # the page's "about 0.033": the fp16 step is a little under 1/15, so the
+    # largest value lands just past the top level and clamps (0.0334)
+    assert abs(err.max() - 1 / 30) < 1e-3
+
+
+def test_asym_codes_zero_and_scale_bruteforce():
+    rng = np.random.default_rng(81)
+    for trial in range(200):
+        n = 64
+        w = (rng.standard_normal(n) * 0.02 + (0.01 if trial % 3 == 0 else 0.0)
+             ).astype(np.float16).astype(np.float32)
+        s = np.exp(rng.standard_normal(n)).astype(np.float32)
+        q, qs, z = oracle.fake_quant_group_asym(w, s)
+        ws = (w * s).astype(np.float32)
+        rng_ = max(np.float32(ws.max() - ws.min()), np.float32(1e-5))
+        assert qs == float(np.float16(np.float32(rng_) / np.float32(15)))
+        assert z == _nearest_int_in(np.float32(-ws.min()) / np.float32(qs), 0, 15)
+        for j in range(n):
+            quot = np.float32(ws[j]) / np.float32(qs)
+            assert q[j] == _nearest_int_in(float(quot) + z, 0, 15) or \
+                abs(abs(float(quot) + z - q[j]) - 0.5) < 1e-6   # a tie in the shifted grid
+            assert q[j] == min(15, max(0, int(np.rint(quot)) + z))
+
+
+def test_asym_zero_group_and_nonfinite():
+    q, qs, z = oracle.fake_quant_group_asym(np.zeros(32, np.float32), np.ones(32, np.float32))
+    assert z == 0 and not q.any()
+    assert qs == float(np.float16(np.float32(1e-5) / np.float32(15)))
+    w = np.ones(32, np.float32)
+    w[3] = np.inf
+    q, qs, z = oracle.fake_quant_group_asym(w, np.ones(32, np.float32))
+    assert np.isnan(qs) and z == 8 and (q == 8).all()
+
+
+def test_asym_dequant_within_half_step():
+    rng = np.random.default_rng(82)
+    for _ in range(100):
+        w = (rng.standard_normal(128) * 0.02).astype(np.float16).astype(np.float32)
+        s = np.exp(rng.standard_normal(128)).astype(np.float32)
+        q, qs, z = oracle.fake_quant_group_asym(w, s)
+        ws = (w * s).astype(np.float64)
+        err = np.abs(ws - (q.astype(np.float64) - z) * qs)
+        inside = (q > 0) & (q < 15)
+        assert np.all(err[inside] <= qs / 2 * (1 + 1e-6))
+
+
+@pytest.mark.parametrize("g", [32, 128])
+def test_asym_pack_roundtrip(g):
+    """Codes and per-group zero points unpack exactly; the runtime dequant
+    (u - zero) * scale equals the group dequant (q - zero) * q_scale."""
+    rng = np.random.default_rng(83 + g)
+    d_out, d_in = 24, 256
+    W = (rng.standard_normal((d_out, d_in)) * 0.02).astype(np.float16)
+    s = np.exp(rng.standard_normal(d_in) * 0.5).astype(np.float32)
+    qw, sc, qz = oracle.quantize_pack(W, s, g, -1)
+    u = oracle.unpack(qw, d_out)
+    zz = oracle.unpack(qz, d_out)          # [d_out, G]: the zeros use the same packing
+    Wf = W.astype(np.float32)
+    for r in range(d_out):
+        for k in range(d_in // g):
+            sl = slice(k * g, (k + 1) * g)
+            q, qs, z = oracle.fake_quant_group_asym(Wf[r, sl], s[sl])
+            assert np.array_equal(u[r, sl], q) and zz[r, k] == z
+            assert sc[k, r] == np.float16(qs)
+            assert np.array_equal((u[r, sl].astype(np.float64) - zz[r, k]) * float(sc[k, r]),
+                                  (q.astype(np.float64) - z) * qs)
+
+
+def test_asym_search_alpha0_is_asym_rtn():
+    rng = np.random.default_rng(84)
+    W = (rng.standard_normal((32, 256)) * 0.02).astype(np.float16)
+    X = (rng.standard_normal((64, 256)) * np.exp(rng.standard_normal(256))).astype(np.float16)
+    x = oracle.act_stats(X)
+    err, best, s = oracle.scale_search([W], x, 128, 20, oracle.ASYM)
+    e0 = oracle.weighted_error(W, x, np.ones(256, np.float32), 128, oracle.ASYM)
+    assert math.isclose(err[0], e0, rel_tol=1e-12)
+    assert err[best] <= err[0]
+    e_sym = oracle.weighted_error(W, x, np.ones(256, np.float32), 128)
+    assert e0 != e_sym
