@@ -82,6 +82,8 @@ def _args():
     ap.add_argument("--scale-mode", choices=["joint", "geomean"], default="joint",
                     help="joint: one search over a shared-input group's linears; geomean: "
                          "one search per linear, then their geometric mean (norm group)")
+    ap.add_argument("--asym", action="store_true",
+                    help="asymmetric INT4 grid (per-group zero points) in search and pack")
     ap.add_argument("--duo", action="store_true",
                     help="duo scaling candidates (weights' row-normalised mean) in the search")
     ap.add_argument("--clip", type=int, default=0,
@@ -223,7 +225,8 @@ def run_ours(a):
         for Ws, X in li:
             jobs.append(pipeline.GroupJob([W.to(dev) for W in Ws], X.to(dev), g, n_grid,
                                           work.output_mode, n_clip=a.clip,
-                                          scale_mode=a.scale_mode, duo=a.duo))
+                                          scale_mode=a.scale_mode, duo=a.duo,
+                                          asym=a.asym))
     if work.layers == 1:
         host_layer = [([W.pin_memory() for W in Ws], X.pin_memory()) for Ws, X in layer_inputs[0]]
     else:
@@ -325,7 +328,8 @@ def run_ours(a):
     # --- end to end: the same work streamed from pinned host memory
     template = layer_inputs[0]
     streamer = pipeline.LayerStreamer(template, dev, g, n_grid, work.output_mode,
-                                      n_clip=a.clip, scale_mode=a.scale_mode, duo=a.duo)
+                                      n_clip=a.clip, scale_mode=a.scale_mode, duo=a.duo,
+                                      asym=a.asym)
     if work.layers == 1:
         n_e2e = max(5, min(50, a.steps // 20))
         host_layers = [host_layer] * n_e2e
@@ -436,7 +440,7 @@ def run_ours(a):
         "data": "synthetic",
         "config": {"workload": a.workload, "layers": work.layers, "tokens": work.tokens,
                    "group_size": g, "n_grid": n_grid, "n_clip": a.clip,
-                   "scale_mode": a.scale_mode, "duo": a.duo,
+                   "scale_mode": a.scale_mode, "duo": a.duo, "asym": a.asym,
                    "params_per_step": _total_params(work, world, params),
                    "params_rank0": params,
                    "l2": ("flushed (256 MB write) between timed steps" if flush_l2 else
@@ -452,7 +456,7 @@ def run_ours(a):
     }
     if world == 1 and not a.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(work, g, a.cpu_seconds, a.clip, a.scale_mode,
-                                           a.duo)
+                                           a.duo, a.asym)
     print(json.dumps(out), flush=True)
     if world > 1:
         dist.destroy_process_group()
@@ -502,9 +506,11 @@ def oracle_sample(work, g, row_cap=256, out_rows=16, out_tokens=None):
     return out, params, "; ".join(parts) + f" ({mode})"
 
 
-def _oracle_pass(sample, g, n_grid, output_mode, n_clip=0, scale_mode="joint", duo=False):
+def _oracle_pass(sample, g, n_grid, output_mode, n_clip=0, scale_mode="joint", duo=False,
+                 asym=False):
     import oracle
-    fl = oracle.DUO if duo else 0
+    fl = (oracle.DUO if duo else 0) | (oracle.ASYM if asym else 0)
+    zp = -1 if asym else 8
     for Ws, X in sample:
         x = oracle.act_stats(X)
         if output_mode:
@@ -517,10 +523,10 @@ def _oracle_pass(sample, g, n_grid, output_mode, n_clip=0, scale_mode="joint", d
             err, best, s = oracle.scale_search(Ws, x, g, n_grid, fl)
         for W in Ws:
             idx = oracle.clip_search(W, x, s, g, n_clip)[0] if n_clip > 0 else None
-            oracle.quantize_pack(W, s, g, 8, idx)
+            oracle.quantize_pack(W, s, g, zp, idx)
 
 
-def cpu_baseline(work, g, seconds, n_clip=0, scale_mode="joint", duo=False):
+def cpu_baseline(work, g, seconds, n_clip=0, scale_mode="joint", duo=False, asym=False):
     """Passes of the CPU oracle over a bounded sample of the workload until
     `seconds` have elapsed."""
     import oracle
@@ -530,7 +536,7 @@ def cpu_baseline(work, g, seconds, n_clip=0, scale_mode="joint", duo=False):
     n = 0
     t0 = time.perf_counter()
     while True:
-        _oracle_pass(sample, g, work.n_grid, work.output_mode, n_clip, scale_mode, duo)
+        _oracle_pass(sample, g, work.n_grid, work.output_mode, n_clip, scale_mode, duo, asym)
         n += 1
         if time.perf_counter() - t0 >= seconds:
             break
@@ -553,10 +559,12 @@ def run_reference(a):
     if a.clip > 0:
         text += f" + {a.clip}-ratio clip search"
     for _ in range(max(a.warmup, 3)):
-        _oracle_pass(sample, g, work.n_grid, work.output_mode, a.clip, a.scale_mode, a.duo)
+        _oracle_pass(sample, g, work.n_grid, work.output_mode, a.clip, a.scale_mode, a.duo,
+                     a.asym)
     t0 = time.perf_counter()
     for _ in range(a.steps):
-        _oracle_pass(sample, g, work.n_grid, work.output_mode, a.clip, a.scale_mode, a.duo)
+        _oracle_pass(sample, g, work.n_grid, work.output_mode, a.clip, a.scale_mode, a.duo,
+                     a.asym)
     dt = time.perf_counter() - t0
     v = a.steps * params / dt / 1e9
     print(json.dumps({
@@ -566,7 +574,8 @@ def run_reference(a):
         "vs_baseline": None, "dtype": "f64" if work.output_mode else "f32",
         "data": "synthetic", "config": {"workload": a.workload, "group_size": g,
                                         "n_grid": work.n_grid, "n_clip": a.clip,
-                                        "scale_mode": a.scale_mode, "duo": a.duo},
+                                        "scale_mode": a.scale_mode, "duo": a.duo,
+                                        "asym": a.asym},
         "cpu_baseline": {"value": v, "unit": UNIT, "cores": oracle.threads(),
                          "kind": "oracle", "sample": f"per step, one pass over {text}"},
         "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},

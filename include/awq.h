@@ -62,6 +62,16 @@ typedef enum awq_status {
  * of the segments of |W[r, j]| / max_k |W[r, k]| (fp64); needs
  * d_in <= 16384 and the AWQ_OP_SCALE_SEARCH_DUO workspace. */
 #define AWQ_DUO_SCALING 2
+/* awq_scale_search only: the asymmetric INT4 grid ("AWQ architecture ...",
+ * section "Quantization, storage and packing": a 16-bit scale and a 4-bit
+ * zero point per group and output channel).  Per group, with ws = w * s:
+ * range = max(max ws - min ws, 1e-5), q_scale = fp16(range / 15),
+ * zero = clamp(rint(-min ws / q_scale), 0, 15),
+ * q = clamp(rint(ws / q_scale) + zero, 0, 15), w_hat = (q - zero) q_scale / s.
+ * Pack the result with awq_quantize_pack(zero_point = AWQ_ZERO_POINT_ASYM). */
+#define AWQ_ASYMMETRIC 4
+/* zero_point argument of awq_quantize_pack selecting the asymmetric grid */
+#define AWQ_ZERO_POINT_ASYM (-1)
 
 /* Operation ids of awq_workspace_size. */
 #define AWQ_OP_ACT_STATS    0
@@ -218,7 +228,12 @@ awq_status awq_scale_search_noalloc(int n_seg, const void *const *W,
  *               count as 19), q_scale = fp16(fl32(fl32(c m) / 7)), and codes
  *               beyond the range saturate at +-7
  *   group_size  32, 64 or 128
- *   zero_point  7 or 8 (8: codes 1..15; 7: codes 0..14)
+ *   zero_point  7 or 8 (8: codes 1..15; 7: codes 0..14), or
+ *               AWQ_ZERO_POINT_ASYM for the asymmetric grid of
+ *               AWQ_ASYMMETRIC: codes 0..15 and qzeros holding each (group,
+ *               row)'s zero point in the same nibble order as qweight
+ *               (clip_idx must then be NULL); a non-finite group stores
+ *               scale NaN, zero point 8 and codes 8
  *   qweight     int32 [d_in, d_out / 8] device output
  *   scales      fp16 [d_in / group_size, d_out] device output
  *   qzeros      int32 [d_in / group_size, d_out / 8] device output

@@ -24,6 +24,8 @@ OP_OUTPUT_ERROR = 2
 OP_CLIP_SEARCH = 3
 OP_SCALE_SEARCH_DUO = 4
 DUO_SCALING = 2
+ASYMMETRIC = 4
+ZERO_POINT_ASYM = -1
 CLIP_DEN = 20
 MAX_SEGMENTS = 8
 

@@ -129,7 +129,7 @@ awq_status awq_scale_search(int n_seg, const void* const* W, const int64_t* d_ou
     if (!x_mean || !err || !best_idx || !s_best) return AWQ_ERR_INVALID_ARG;
     if (!valid_group(group_size)) return AWQ_ERR_UNSUPPORTED;
     if (n_grid < 1 || n_grid > 32) return AWQ_ERR_INVALID_ARG;
-    if (flags & ~(AWQ_SCALE_FP32 | AWQ_DUO_SCALING)) return AWQ_ERR_INVALID_ARG;
+    if (flags & ~(AWQ_SCALE_FP32 | AWQ_DUO_SCALING | AWQ_ASYMMETRIC)) return AWQ_ERR_INVALID_ARG;
     const bool duo = (flags & AWQ_DUO_SCALING) != 0;
     if (duo && d_in > kDuoMaxDin) return AWQ_ERR_UNSUPPORTED;
     if (d_in < group_size || d_in % group_size || d_in > (int64_t(1) << 24))
@@ -154,7 +154,9 @@ awq_status awq_quantize_pack(const void* W, int64_t d_out, int64_t d_in, const f
                              int32_t* qweight, void* scales, int32_t* qzeros, void* stream) {
     if (!W || !qweight || !scales || !qzeros) return AWQ_ERR_INVALID_ARG;
     if (!valid_group(group_size)) return AWQ_ERR_UNSUPPORTED;
-    if (zero_point != 7 && zero_point != 8) return AWQ_ERR_INVALID_ARG;
+    if (zero_point != 7 && zero_point != 8 && zero_point != AWQ_ZERO_POINT_ASYM)
+        return AWQ_ERR_INVALID_ARG;
+    if (zero_point == AWQ_ZERO_POINT_ASYM && clip_idx) return AWQ_ERR_UNSUPPORTED;
     if (d_out < 8 || d_out % 8 || d_out > (int64_t(1) << 31)) return AWQ_ERR_INVALID_ARG;
     if (d_in < group_size || d_in % group_size || d_in > (int64_t(1) << 24))
         return AWQ_ERR_INVALID_ARG;

@@ -136,6 +136,19 @@ __device__ __forceinline__ float div7_rn(float m) {
 // smaller m a value below 2^-25, which rounds to the same fp16 value (zero).
 // Used where only the fp16 rounding of the quotient matters; an infinite m
 // gives NaN.
+// RN(m / 15) for finite m >= 0 (the asymmetric grid's scale): two residual
+// corrections of m * RN(1/15); tiny m, where a residual could underflow,
+// takes the IEEE division.  Checked against __fdiv_rn for every
+// non-negative finite fp32 value.
+__device__ __forceinline__ float div15_rn(float m) {
+    if (m < 0x1p-100f) return __fdiv_rn(m, 15.0f);
+    const float c = 0.0666666701f;           // RN(1/15) = 0x3D888889
+    float q = __fmul_rn(m, c);
+    float r = __fmaf_rn(-q, 15.0f, m);
+    q = __fmaf_rn(r, c, q);
+    r = __fmaf_rn(-q, 15.0f, m);
+    return __fmaf_rn(r, c, q);
+}
 __device__ __forceinline__ float div7_rn_for_fp16(float m) {
     const float c = 0.142857149f;            // RN(1/7)
     const float q0 = __fmul_rn(m, c);

@@ -51,10 +51,15 @@ __device__ __forceinline__ constexpr int nibble_of_row(int r8) {
     return (r8 >> 1) + 4 * (r8 & 1);
 }
 
-// NaN-propagating maximum of three values (a NaN anywhere gives NaN)
+// NaN-propagating maximum / minimum of three values (a NaN anywhere gives NaN)
 __device__ __forceinline__ float max3_nan(float a, float b, float c) {
     float d;
     asm("max.NaN.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+__device__ __forceinline__ float min3_nan(float a, float b, float c) {
+    float d;
+    asm("min.NaN.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
     return d;
 }
 
@@ -63,16 +68,19 @@ __device__ __forceinline__ float max3_nan(float a, float b, float c) {
 // different banks.
 __device__ __forceinline__ int sabs_slot(int j) { return j + 4 * (j >> 6); }
 
-template <int G, bool kFast>
+// kAsym: codes rint(quotient) + zero of the row, clamped to 0..15; the
+// rows' zero points enter through word_init (one per word).
+template <int G, bool kFast, bool kAsym>
 __device__ __forceinline__ void pack_columns(const uint4* tile, const float2* qr_tile,
-                                             const int* bad_tile, int jp, int cq, int kk,
-                                             float2 s2, uint32_t word_init,
+                                             const int* bad_tile, const int* zero_tile,
+                                             int jp, int cq, int kk, float2 s2,
+                                             const uint32_t word_init[4],
                                              uint32_t words[2][4]) {
     const float2 magic2 = make_float2(kRoundMagic, kRoundMagic);
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-        words[0][q] = word_init;
-        words[1][q] = word_init;
+        words[0][q] = word_init[q];
+        words[1][q] = word_init[q];
     }
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
@@ -92,7 +100,13 @@ __device__ __forceinline__ void pack_columns(const uint4* tile, const float2* qr
         res = __ffma2_rn(q, nb2, a);
         q = __ffma2_rn(res, y2, q);
         float2 t = __fadd2_rn(q, magic2);
-        if (!kFast) {
+        if (kAsym) {
+            const float z = (float)zero_tile[row_slot(kk, r)];
+            const float lo = kRoundMagic - z, hi = kRoundMagic + 15.f - z;
+            t.x = fminf(fmaxf(t.x, lo), hi);
+            t.y = fminf(fmaxf(t.y, lo), hi);
+            if (bad_tile[row_slot(kk, r)]) t = magic2;   // code = zero point (8)
+        } else if (!kFast) {
             t.x = fminf(fmaxf(t.x, kRoundMagic - 7.f), kRoundMagic + 7.f);
             t.y = fminf(fmaxf(t.y, kRoundMagic - 7.f), kRoundMagic + 7.f);
             if (bad_tile[row_slot(kk, r)]) t = magic2;   // code = zero point
@@ -103,7 +117,7 @@ __device__ __forceinline__ void pack_columns(const uint4* tile, const float2* qr
     }
 }
 
-template <int G>
+template <int G, bool kAsym>
 __global__ void __launch_bounds__(kPackThreads, 5)
 pack_kernel(const uint4* __restrict__ W, int64_t d_out, int64_t d_in,
             const float* __restrict__ s, const uint8_t* __restrict__ clip_idx, int zero_point,
@@ -117,6 +131,9 @@ pack_kernel(const uint4* __restrict__ W, int64_t d_out, int64_t d_in,
     float2* qr_tile = reinterpret_cast<float2*>(sabs_tile + kPackCols + 8);  // [KG][kRowStride]
     int* bad_tile = reinterpret_cast<int*>(qr_tile + KG * kRowStride);  // [KG][kRowStride]
     int* slow_blk = bad_tile + KG * kRowStride;                          // [KG][kBlocks32]
+    int* zero_tile = slow_blk + KG * kBlocks32;                          // [KG][kRowStride]
+    uint32_t* zw_tile = reinterpret_cast<uint32_t*>(zero_tile + KG * kRowStride);  // [KG][16]
+    float* ssgn_tile = reinterpret_cast<float*>(zw_tile + KG * (kPackRows / 8));   // s, padded
 
     // a programmatic dependent launch: W and s may come from the kernel before
     pdl_wait();
@@ -150,60 +167,120 @@ pack_kernel(const uint4* __restrict__ W, int64_t d_out, int64_t d_in,
         const float sv = gc < d_in ? (s ? s[gc] : 1.0f) : 1.0f;
         s_tile[tid] = sv;
         sabs_tile[sabs_slot(tid)] = fabsf(sv);
+        if (kAsym) ssgn_tile[sabs_slot(tid)] = sv;
     }
     if (tid < KG * kBlocks32) slow_blk[tid] = 0;
     pdl_launch_dependents();   // the tile is read; the next kernel may start launching
     __syncthreads();
 
     // ---- phase 2: group scale of every (row, group), two threads each.
-    // max |w s| = max |w| |s|: the sign bits are cleared before the fp16 ->
-    // fp32 conversion, so the products are non-negative and a three-input
-    // NaN-propagating maximum takes two of them per instruction.
-    for (int task = tid; task < 2 * KG * kPackRows; task += kPackThreads) {
-        const int half = task & 1;
-        const int r = (task >> 1) % kPackRows, kk = (task >> 1) / kPackRows;
-        float m = 0.f;
+    if (kAsym) {
+        // asymmetric grid: the signed max and min of w s (NaN-propagating)
+        for (int task = tid; task < 2 * KG * kPackRows; task += kPackThreads) {
+            const int half = task & 1;
+            const int r = (task >> 1) % kPackRows, kk = (task >> 1) / kPackRows;
+            float mx = __int_as_float(0xff800000), mn = __int_as_float(0x7f800000);
 #pragma unroll
-        for (int cc = 0; cc < G / 16; ++cc) {
-            const int c = kk * (G / 8) + half * (G / 16) + cc;
-            const uint4 v = tile[r * kPackChunks + (c ^ pack_swz(r))];
-            const uint32_t hw[4] = {v.x & 0x7fff7fffu, v.y & 0x7fff7fffu, v.z & 0x7fff7fffu,
-                                    v.w & 0x7fff7fffu};
-            const float4 sa = *reinterpret_cast<const float4*>(&sabs_tile[sabs_slot(8 * c)]);
-            const float4 sb = *reinterpret_cast<const float4*>(&sabs_tile[sabs_slot(8 * c + 4)]);
-            const float sv[8] = {sa.x, sa.y, sa.z, sa.w, sb.x, sb.y, sb.z, sb.w};
+            for (int cc = 0; cc < G / 16; ++cc) {
+                const int c = kk * (G / 8) + half * (G / 16) + cc;
+                const uint4 v = tile[r * kPackChunks + (c ^ pack_swz(r))];
+                const uint32_t hw[4] = {v.x, v.y, v.z, v.w};
+                const float4 sa = *reinterpret_cast<const float4*>(&ssgn_tile[sabs_slot(8 * c)]);
+                const float4 sb =
+                    *reinterpret_cast<const float4*>(&ssgn_tile[sabs_slot(8 * c + 4)]);
+                const float sv[8] = {sa.x, sa.y, sa.z, sa.w, sb.x, sb.y, sb.z, sb.w};
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const float2 w = __half22float2(*reinterpret_cast<const __half2*>(&hw[i]));
-                const float2 a = __fmul2_rn(w, make_float2(sv[2 * i], sv[2 * i + 1]));
-                m = max3_nan(m, a.x, a.y);
-            }
-        }
-        {
-            const float o = __shfl_xor_sync(0xffffffffu, m, 1);
-            m = max3_nan(m, o, o);
-        }
-        if (half == 0) {
-            const bool bad = !(m <= 3.402823466e38f);      // a NaN or an infinity
-            const int64_t gr = row0 + r, gk = col0 / G + kk;
-            // clipping shrinks the range to c * m, c = RN((20 - i) / 20); codes
-            // beyond it saturate, so the block takes the clamping path
-            bool clipped = false;
-            if (clip_idx && gr < d_out && gk * G < d_in) {
-                const int ci = min((int)clip_idx[gr * (d_in / G) + gk], kClipMaxIndex);
-                if (ci > 0) {
-                    m = __fmul_rn(m, __fdiv_rn((float)(kClipDen - ci), (float)kClipDen));
-                    clipped = true;
+                for (int i = 0; i < 4; ++i) {
+                    const float2 w = __half22float2(*reinterpret_cast<const __half2*>(&hw[i]));
+                    const float2 a = __fmul2_rn(w, make_float2(sv[2 * i], sv[2 * i + 1]));
+                    mx = max3_nan(mx, a.x, a.y);
+                    mn = min3_nan(mn, a.x, a.y);
                 }
             }
-            bool in_range;
-            const float qs = bad ? 1.0f : group_scale(m, false, &in_range);
-            qr_tile[row_slot(kk, r)] = make_float2(qs, (qs > 0.f) ? __frcp_rn(qs) : 0.f);
-            bad_tile[row_slot(kk, r)] = bad;
-            if (bad || clipped || !in_range) slow_blk[kk * kBlocks32 + r / 32] = 1;
-            if (gr < d_out && gk * G < d_in)
-                scales[gk * d_out + gr] = bad ? __ushort_as_half((unsigned short)0x7E00)
-                                              : __float2half_rn(qs);
+            {
+                const float ox = __shfl_xor_sync(0xffffffffu, mx, 1);
+                const float on = __shfl_xor_sync(0xffffffffu, mn, 1);
+                mx = max3_nan(mx, ox, ox);
+                mn = min3_nan(mn, on, on);
+            }
+            if (half == 0) {
+                const bool bad = !(mx <= 3.402823466e38f) || !(mn >= -3.402823466e38f);
+                float qs = 1.0f;
+                int z = 8;
+                if (!bad) {
+                    const float range = fmaxf(__fsub_rn(mx, mn), 1e-5f);
+                    qs = fminf(__half2float(__float2half_rn(div15_rn(range))), kHalfMax);
+                    z = (int)fminf(fmaxf(rintf(div_rn_rcp(-mn, qs, __frcp_rn(qs))), 0.f), 15.f);
+                }
+                qr_tile[row_slot(kk, r)] = make_float2(qs, __frcp_rn(qs));
+                bad_tile[row_slot(kk, r)] = bad;
+                zero_tile[row_slot(kk, r)] = z;
+                const int64_t gr = row0 + r, gk = col0 / G + kk;
+                if (gr < d_out && gk * G < d_in)
+                    scales[gk * d_out + gr] = bad ? __ushort_as_half((unsigned short)0x7E00)
+                                                  : __float2half_rn(qs);
+            }
+        }
+        __syncthreads();
+        // zero-point words of every 8-row block: nibble p holds row 8c + order[p]
+        for (int i = tid; i < KG * (kPackRows / 8); i += kPackThreads) {
+            const int kk = i / (kPackRows / 8), c8 = i % (kPackRows / 8);
+            uint32_t wv = 0;
+#pragma unroll
+            for (int i8 = 0; i8 < 8; ++i8)
+                wv |= (uint32_t)zero_tile[row_slot(kk, 8 * c8 + i8)] << (4 * nibble_of_row(i8));
+            zw_tile[kk * (kPackRows / 8) + c8] = wv;
+        }
+    } else {
+        // max |w s| = max |w| |s|: the sign bits are cleared before the fp16 ->
+        // fp32 conversion, so the products are non-negative and a three-input
+        // NaN-propagating maximum takes two of them per instruction.
+        for (int task = tid; task < 2 * KG * kPackRows; task += kPackThreads) {
+            const int half = task & 1;
+            const int r = (task >> 1) % kPackRows, kk = (task >> 1) / kPackRows;
+            float m = 0.f;
+#pragma unroll
+            for (int cc = 0; cc < G / 16; ++cc) {
+                const int c = kk * (G / 8) + half * (G / 16) + cc;
+                const uint4 v = tile[r * kPackChunks + (c ^ pack_swz(r))];
+                const uint32_t hw[4] = {v.x & 0x7fff7fffu, v.y & 0x7fff7fffu, v.z & 0x7fff7fffu,
+                                        v.w & 0x7fff7fffu};
+                const float4 sa = *reinterpret_cast<const float4*>(&sabs_tile[sabs_slot(8 * c)]);
+                const float4 sb = *reinterpret_cast<const float4*>(&sabs_tile[sabs_slot(8 * c + 4)]);
+                const float sv[8] = {sa.x, sa.y, sa.z, sa.w, sb.x, sb.y, sb.z, sb.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float2 w = __half22float2(*reinterpret_cast<const __half2*>(&hw[i]));
+                    const float2 a = __fmul2_rn(w, make_float2(sv[2 * i], sv[2 * i + 1]));
+                    m = max3_nan(m, a.x, a.y);
+                }
+            }
+            {
+                const float o = __shfl_xor_sync(0xffffffffu, m, 1);
+                m = max3_nan(m, o, o);
+            }
+            if (half == 0) {
+                const bool bad = !(m <= 3.402823466e38f);      // a NaN or an infinity
+                const int64_t gr = row0 + r, gk = col0 / G + kk;
+                // clipping shrinks the range to c * m, c = RN((20 - i) / 20); codes
+                // beyond it saturate, so the block takes the clamping path
+                bool clipped = false;
+                if (clip_idx && gr < d_out && gk * G < d_in) {
+                    const int ci = min((int)clip_idx[gr * (d_in / G) + gk], kClipMaxIndex);
+                    if (ci > 0) {
+                        m = __fmul_rn(m, __fdiv_rn((float)(kClipDen - ci), (float)kClipDen));
+                        clipped = true;
+                    }
+                }
+                bool in_range;
+                const float qs = bad ? 1.0f : group_scale(m, false, &in_range);
+                qr_tile[row_slot(kk, r)] = make_float2(qs, (qs > 0.f) ? __frcp_rn(qs) : 0.f);
+                bad_tile[row_slot(kk, r)] = bad;
+                if (bad || clipped || !in_range) slow_blk[kk * kBlocks32 + r / 32] = 1;
+                if (gr < d_out && gk * G < d_in)
+                    scales[gk * d_out + gr] = bad ? __ushort_as_half((unsigned short)0x7E00)
+                                                  : __float2half_rn(qs);
+            }
         }
     }
     __syncthreads();
@@ -211,18 +288,29 @@ pack_kernel(const uint4* __restrict__ W, int64_t d_out, int64_t d_in,
     // ---- phase 3: codes and packed words
     const int64_t C = d_out / 8;
     const int64_t c0 = row0 / 8;
-    const uint32_t bias = kRoundMagicBits - (uint32_t)zero_point;
-    const uint32_t word_init = 0u - bias * 0x11111111u;
     {
         const int cq = tid & 3;          // 4 output words = 32 rows
         const int jp = tid >> 2;         // 2 input columns
         const int kk = (2 * jp) / G;
         const float2 s2 = make_float2(s_tile[2 * jp], s_tile[2 * jp + 1]);
+        // each nibble starts at (zero point - bits of 1.5*2^23); adding the
+        // bits of the rounded quotient + 1.5*2^23 leaves the unsigned code
+        uint32_t word_init[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+            word_init[q] = kAsym ? zw_tile[kk * (kPackRows / 8) + 4 * cq + q] -
+                                       kRoundMagicBits * 0x11111111u
+                                 : 0u - (kRoundMagicBits - (uint32_t)zero_point) * 0x11111111u;
         uint32_t words[2][4];
-        if (slow_blk[kk * kBlocks32 + cq])
-            pack_columns<G, false>(tile, qr_tile, bad_tile, jp, cq, kk, s2, word_init, words);
+        if (kAsym)
+            pack_columns<G, false, true>(tile, qr_tile, bad_tile, zero_tile, jp, cq, kk, s2,
+                                         word_init, words);
+        else if (slow_blk[kk * kBlocks32 + cq])
+            pack_columns<G, false, false>(tile, qr_tile, bad_tile, zero_tile, jp, cq, kk, s2,
+                                          word_init, words);
         else
-            pack_columns<G, true>(tile, qr_tile, bad_tile, jp, cq, kk, s2, word_init, words);
+            pack_columns<G, true, false>(tile, qr_tile, bad_tile, zero_tile, jp, cq, kk, s2,
+                                         word_init, words);
         const int64_t cw = c0 + 4 * cq;
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
@@ -245,7 +333,8 @@ pack_kernel(const uint4* __restrict__ W, int64_t d_out, int64_t d_in,
     for (int i = tid; i < KG * (kPackRows / 8); i += kPackThreads) {
         const int kk = i / (kPackRows / 8), cwl = i % (kPackRows / 8);
         const int64_t gk = col0 / G + kk, cw = c0 + cwl;
-        if (gk * G < d_in && cw < C) qzeros[gk * C + cw] = (int32_t)zword;
+        if (gk * G < d_in && cw < C)
+            qzeros[gk * C + cw] = (int32_t)(kAsym ? zw_tile[i] : zword);
     }
 }
 
@@ -256,20 +345,25 @@ cudaError_t launch_pack_G(const void* W, int64_t d_out, int64_t d_in, const floa
     constexpr int KG = kPackCols / G;
     const size_t smem = (size_t)kPackRows * kPackCols * 2 + (2 * kPackCols + 8) * sizeof(float) +
                         (size_t)KG * kRowStride * (sizeof(float2) + sizeof(int)) +
-                        (size_t)KG * kBlocks32 * sizeof(int);
-    static int configured[64] = {};
+                        (size_t)KG * kBlocks32 * sizeof(int) +
+                        (size_t)KG * kRowStride * sizeof(int) +          // zero points
+                        (size_t)KG * (kPackRows / 8) * sizeof(uint32_t) +  // zero words
+                        (size_t)(kPackCols + 8) * sizeof(float);          // signed s, padded
+    const bool asym = zero_point == AWQ_ZERO_POINT_ASYM;
+    static int configured[64][2] = {};
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev < 0 || dev >= 64 || !configured[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(pack_kernel<G>,
+    if (dev < 0 || dev >= 64 || !configured[dev][asym]) {
+        cudaError_t e = cudaFuncSetAttribute(asym ? pack_kernel<G, true> : pack_kernel<G, false>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)smem);
         if (e != cudaSuccess) return e;
-        if (dev >= 0 && dev < 64) configured[dev] = 1;
+        if (dev >= 0 && dev < 64) configured[dev][asym] = 1;
     }
     dim3 grid((unsigned)((d_in + kPackCols - 1) / kPackCols),
               (unsigned)((d_out + kPackRows - 1) / kPackRows));
-    return launch_pdl(pack_kernel<G>, grid, dim3(kPackThreads), smem, stream,
+    return launch_pdl(asym ? pack_kernel<G, true> : pack_kernel<G, false>, grid,
+                      dim3(kPackThreads), smem, stream,
                       static_cast<const uint4*>(W), d_out, d_in, s, clip_idx, zero_point,
                       qweight, static_cast<__half*>(scales), qzeros);
 }

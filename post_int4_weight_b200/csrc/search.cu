@@ -258,7 +258,79 @@ __device__ __forceinline__ float2 rows_errors(const float2* ws0, const float2* w
     return __fadd2_rn(acc2[0], acc2[1]);
 }
 
+// ---- asymmetric grid (16 levels, per-group zero point)
+// Pass 1: ws = w * s and the lane's largest and smallest ws.
+__device__ __forceinline__ float2 row_products_minmax(const float2* w, const float4* s4,
+                                                      float2* ws) {
+    float mx = __int_as_float(0xff800000), mn = __int_as_float(0x7f800000);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        ws[2 * k] = __fmul2_rn(w[2 * k], f2(s4[k].x, s4[k].y));
+        ws[2 * k + 1] = __fmul2_rn(w[2 * k + 1], f2(s4[k].z, s4[k].w));
+        mx = fmaxf(fmaxf(mx, fmaxf(ws[2 * k].x, ws[2 * k].y)),
+                   fmaxf(ws[2 * k + 1].x, ws[2 * k + 1].y));
+        mn = fminf(fminf(mn, fminf(ws[2 * k].x, ws[2 * k].y)),
+                   fminf(ws[2 * k + 1].x, ws[2 * k + 1].y));
+    }
+    return f2(mx, mn);
+}
+
+// The row's scale fp16(max(max - min, 1e-5) / 15) (exact quotient), its
+// zero point clamp(rint(-min / q_scale), 0, 15) (exact quotient), the
+// rounding constant 1.5*2^23 + zero and an approximate reciprocal for the
+// codes.  A non-finite ws makes the row's error non-finite by itself.
 template <int L, bool kFp32>
+__device__ __forceinline__ void row_scale_asym(float2 mm, float* qs, float* rq, float* mz) {
+    float mx = mm.x, mn = mm.y;
+#pragma unroll
+    for (int o = 1; o < L; o <<= 1) {
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    }
+    const float range = fmaxf(__fsub_rn(mx, mn), 1e-5f);
+    float q = div15_rn(range);
+    if (!kFp32) q = fminf(__half2float(__float2half_rn(q)), kHalfMax);
+    const float z = fminf(fmaxf(rintf(div_rn_rcp(-mn, q, __frcp_rn(q))), 0.f), 15.f);
+    *qs = q;
+    *rq = rcp_approx(q);
+    *mz = kRoundMagic + z;
+}
+
+// Pass 2 on the asymmetric grid: codes clamp(rint(ws / q_scale) + zero, 0, 15)
+// by the rounding addition of 1.5*2^23 + zero, then the same weighted sum as
+// rows_errors.
+template <int L>
+__device__ __forceinline__ float2 rows_errors_asym(const float2* ws0, const float2* ws1,
+                                                   const float4* T2, int l, float qs0,
+                                                   float rq0, float mz0, float qs1, float rq1,
+                                                   float mz1) {
+    const float2 nqs0 = f2(-qs0, -qs0), nqs1 = f2(-qs1, -qs1);
+    const float2 rq02 = f2(rq0, rq0), mz02 = f2(mz0, mz0), nmz02 = f2(-mz0, -mz0);
+    constexpr float lo = kRoundMagic, hi = kRoundMagic + 15.f;
+    float2 acc2[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const float4 tv = T2[k * L + l];
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            const int i = 2 * k + j;
+            float2 t0 = __ffma2_rn(ws0[i], rq02, mz02);
+            t0 = f2(fminf(fmaxf(t0.x, lo), hi), fminf(fmaxf(t0.y, lo), hi));
+            float t1x = fminf(fmaxf(__fmaf_rn(ws1[i].x, rq1, mz1), lo), hi);
+            float t1y = fminf(fmaxf(__fmaf_rn(ws1[i].y, rq1, mz1), lo), hi);
+            const float2 q0 = __fadd2_rn(t0, nmz02);
+            const float2 q1 = f2(__fadd_rn(t1x, -mz1), __fadd_rn(t1y, -mz1));
+            const float2 d0 = __ffma2_rn(q0, nqs0, ws0[i]);
+            const float2 d1 = __ffma2_rn(q1, nqs1, ws1[i]);
+            float2 sq = __fmul2_rn(d0, d0);
+            sq = __ffma2_rn(d1, d1, sq);
+            acc2[j] = __ffma2_rn(j ? f2(tv.z, tv.w) : f2(tv.x, tv.y), sq, acc2[j]);
+        }
+    }
+    return __fadd2_rn(acc2[0], acc2[1]);
+}
+
+template <int L, bool kFp32, bool kAsym>
 __global__ void __launch_bounds__(kThreads, 1)
 search_kernel(const __grid_constant__ SearchParams p) {
     constexpr int G = 16 * L;                    // group size
@@ -405,13 +477,23 @@ search_kernel(const __grid_constant__ SearchParams p) {
 #pragma unroll
             for (int k = 0; k < 4; ++k) s4[k] = Sa[k * L + l];
             float2 ws[2][kElemsPerRow / 2];
+            float2 e;
+            if (kAsym) {
+                const float2 mm0 = row_products_minmax(w[0], s4, ws[0]);
+                const float2 mm1 = row_products_minmax(w[1], s4, ws[1]);
+                float qs0, rq0, mz0, qs1, rq1, mz1;
+                row_scale_asym<L, kFp32>(mm0, &qs0, &rq0, &mz0);
+                row_scale_asym<L, kFp32>(mm1, &qs1, &rq1, &mz1);
+                e = rows_errors_asym<L>(ws[0], ws[1], Ta, l, qs0, rq0, mz0, qs1, rq1, mz1);
+                acc[a * kThreads + tid] += e.x + e.y;
+                continue;
+            }
             const float m0 = row_products(w[0], s4, ws[0]);
             const float m1 = row_products(w[1], s4, ws[1]);
             float qs0, rq0, qs1, rq1;
             bool in0, in1;
             row_scale<L, kFp32>(m0, &qs0, &rq0, &in0);
             row_scale<L, kFp32>(m1, &qs1, &rq1, &in1);
-            float2 e;
             if (__all_sync(0xffffffffu, in0 & in1)) {
                 e = rows_errors<false, L>(ws[0], ws[1], Ta, l, qs0, rq0, qs1, rq1);
             } else {   // some row has an fp16-subnormal, overflowing, zero or NaN scale
@@ -572,28 +654,28 @@ size_t search_smem_bytes(int group_size, int n_grid) {
            (size_t)n_grid * kThreads * sizeof(float) + 2 * kStages * sizeof(uint64_t) + 16;
 }
 
-template <int L, bool kFp32>
+template <int L, bool kFp32, bool kAsym>
 cudaError_t launch_search_L(const SearchParams& p, int grid, size_t smem, cudaStream_t st) {
     static int configured_smem[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64 || configured_smem[dev] < (int)smem) {
-        cudaError_t e = cudaFuncSetAttribute(search_kernel<L, kFp32>,
+        cudaError_t e = cudaFuncSetAttribute(search_kernel<L, kFp32, kAsym>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)smem);
         if (e != cudaSuccess) return e;
         if (dev >= 0 && dev < 64) configured_smem[dev] = (int)smem;
     }
-    return launch_pdl(search_kernel<L, kFp32>, dim3(grid), dim3(kThreads), smem, st, p);
+    return launch_pdl(search_kernel<L, kFp32, kAsym>, dim3(grid), dim3(kThreads), smem, st, p);
 }
 
-template <bool kFp32>
+template <bool kFp32, bool kAsym>
 cudaError_t launch_search(int L, const SearchParams& p, int grid, size_t smem,
                           cudaStream_t st) {
     switch (L) {
-        case 2: return launch_search_L<2, kFp32>(p, grid, smem, st);
-        case 4: return launch_search_L<4, kFp32>(p, grid, smem, st);
-        case 8: return launch_search_L<8, kFp32>(p, grid, smem, st);
+        case 2: return launch_search_L<2, kFp32, kAsym>(p, grid, smem, st);
+        case 4: return launch_search_L<4, kFp32, kAsym>(p, grid, smem, st);
+        case 8: return launch_search_L<8, kFp32, kAsym>(p, grid, smem, st);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -692,9 +774,12 @@ awq_status launch_scale_search(int n_seg, const void* const* W, const int64_t* d
                                 stream, kTableTauSq);
     }
     if (note_cuda(te, "scale table launch") != cudaSuccess) return AWQ_ERR_CUDA;
-    const cudaError_t e = (flags & AWQ_SCALE_FP32)
-                              ? launch_search<true>(L, p, (int)grid, smem, stream)
-                              : launch_search<false>(L, p, (int)grid, smem, stream);
+    const bool fp32 = (flags & AWQ_SCALE_FP32) != 0, asym = (flags & AWQ_ASYMMETRIC) != 0;
+    const cudaError_t e =
+        fp32 ? (asym ? launch_search<true, true>(L, p, (int)grid, smem, stream)
+                     : launch_search<true, false>(L, p, (int)grid, smem, stream))
+             : (asym ? launch_search<false, true>(L, p, (int)grid, smem, stream)
+                     : launch_search<false, false>(L, p, (int)grid, smem, stream));
     if (e != cudaSuccess) return AWQ_ERR_CUDA;
     return AWQ_OK;
 }

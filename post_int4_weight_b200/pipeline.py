@@ -67,7 +67,8 @@ class GroupJob:
 
     def __init__(self, Ws: Sequence[torch.Tensor], X: torch.Tensor, group_size: int = 128,
                  n_grid: int = 20, output_mode: bool = False, zero_point: int = 8,
-                 n_clip: int = 0, scale_mode: str = "joint", duo: bool = False):
+                 n_clip: int = 0, scale_mode: str = "joint", duo: bool = False,
+                 asym: bool = False):
         if output_mode and len(Ws) != 1:
             raise ValueError("the output-space score takes one linear per call")
         if scale_mode not in ("joint", "geomean"):
@@ -77,11 +78,15 @@ class GroupJob:
         self.g = group_size
         self.n_grid = n_grid
         self.output_mode = output_mode
-        self.zero_point = zero_point
         self.n_clip = n_clip
-        self.flags = awq.DUO_SCALING if duo else awq.SCALE_FP16
-        if duo and output_mode:
-            raise ValueError("duo scaling is a weight-space search option")
+        self.flags = (awq.DUO_SCALING if duo else 0) | (awq.ASYMMETRIC if asym else 0)
+        if (duo or asym) and output_mode:
+            raise ValueError("duo scaling and the asymmetric grid are weight-space options")
+        if asym and n_clip > 0:
+            raise ValueError("the clip search is defined on the symmetric grid")
+        if asym:
+            zero_point = awq.ZERO_POINT_ASYM
+        self.zero_point = zero_point
         # geomean with one member is the joint search
         self.geomean = scale_mode == "geomean" and len(self.Ws) > 1
         dev = X.device
@@ -206,7 +211,8 @@ class LayerStreamer:
 
     def __init__(self, template, device, group_size: int = 128, n_grid: int = 20,
                  output_mode: bool = False, zero_point: int = 8, depth: int = 2,
-                 n_clip: int = 0, scale_mode: str = "joint", duo: bool = False):
+                 n_clip: int = 0, scale_mode: str = "joint", duo: bool = False,
+                 asym: bool = False):
         self.device = torch.device(device)
         self.depth = depth
         self.slots = []
@@ -216,7 +222,7 @@ class LayerStreamer:
                 dWs = [torch.empty(W.shape, dtype=torch.float16, device=self.device) for W in Ws]
                 dX = torch.empty(X.shape, dtype=torch.float16, device=self.device)
                 jobs.append(GroupJob(dWs, dX, group_size, n_grid, output_mode, zero_point,
-                                     n_clip, scale_mode, duo))
+                                     n_clip, scale_mode, duo, asym))
             self.slots.append(jobs)
         self.ws = Workspaces(self.slots[0], self.device)
         self.h2d = torch.cuda.Stream(self.device)

@@ -18,23 +18,38 @@ __global__ void check_div7(uint32_t lo, uint32_t hi, unsigned long long* bad,
     }
 }
 
+// every non-negative finite fp32 bit pattern in [lo, hi): m / 15
+__global__ void check_div15(uint32_t lo, uint32_t hi, unsigned long long* bad,
+                            uint32_t* first_bad) {
+    for (uint64_t i = lo + blockIdx.x * (uint64_t)blockDim.x + threadIdx.x; i < hi;
+         i += (uint64_t)gridDim.x * blockDim.x) {
+        const float m = __uint_as_float((uint32_t)i);
+        const float a = awq::div15_rn(m);
+        const float b = __fdiv_rn(m, 15.0f);
+        if (__float_as_uint(a) != __float_as_uint(b)) {
+            atomicAdd(bad, 1ull);
+            atomicMin(first_bad, (uint32_t)i);
+        }
+    }
+}
+
 // for every positive finite fp16 divisor b (blockIdx.x selects it), numerators
-// a near every half-integer multiple of b in [-8b, 8b] (+-8 ulps) and a
+// a near every half-integer multiple of b in [-16b, 16b] (+-8 ulps) and a
 // stride of other values
 __global__ void check_div_rcp(unsigned long long* bad, uint32_t* first_bad_b) {
     const uint32_t hb = blockIdx.x + 1;           // 0x0001 .. 0x7bff
     const float b = __half2float(__ushort_as_half((unsigned short)hb));
     const float y = __frcp_rn(b);
-    for (int t = threadIdx.x; t < 16 * 17 * 2 + 4096; t += blockDim.x) {
+    for (int t = threadIdx.x; t < 32 * 17 * 2 + 4096; t += blockDim.x) {
         float a;
-        if (t < 16 * 17 * 2) {
+        if (t < 32 * 17 * 2) {
             const int k = t / 34, d = (t % 34) / 2, sgn = t & 1;
-            const float base = __fmul_rn((float)(k - 8) + 0.5f, b);
+            const float base = __fmul_rn((float)(k - 16) + 0.5f, b);
             a = __uint_as_float(__float_as_uint(base) + (uint32_t)(d - 8));
             if (sgn) a = -a;
         } else {
-            const int u = t - 16 * 17 * 2;
-            a = __fmul_rn(b, ((float)u - 2048.0f) * (7.5f / 2048.0f) + 1e-3f * (float)(u & 7));
+            const int u = t - 32 * 17 * 2;
+            a = __fmul_rn(b, ((float)u - 2048.0f) * (15.5f / 2048.0f) + 1e-3f * (float)(u & 7));
         }
         if (!(fabsf(a) <= 3.0e38f)) continue;
         const float q = awq::div_rn_rcp(a, b, y);
@@ -66,19 +81,21 @@ __global__ void check_ddiv_rcp(unsigned long long* bad, uint32_t* first_bad_b) {
 extern "C" int run_checks(unsigned long long* out) {
     // out[0]: div7 mismatches, out[1]: first bad bits, out[2]: div_rcp
     // mismatches, out[3]: first bad fp16 divisor, out[4]: ddiv_rcp
-    // mismatches, out[5]: its first bad fp16 divisor
+    // mismatches, out[5]: its first bad fp16 divisor, out[6]: div15
+    // mismatches, out[7]: first bad bits
     unsigned long long* d_bad;
     uint32_t* d_first;
-    if (cudaMalloc(&d_bad, 3 * sizeof(unsigned long long)) != cudaSuccess) return 1;
-    if (cudaMalloc(&d_first, 3 * sizeof(uint32_t)) != cudaSuccess) return 1;
-    cudaMemset(d_bad, 0, 3 * sizeof(unsigned long long));
-    cudaMemset(d_first, 0xff, 3 * sizeof(uint32_t));
+    if (cudaMalloc(&d_bad, 4 * sizeof(unsigned long long)) != cudaSuccess) return 1;
+    if (cudaMalloc(&d_first, 4 * sizeof(uint32_t)) != cudaSuccess) return 1;
+    cudaMemset(d_bad, 0, 4 * sizeof(unsigned long long));
+    cudaMemset(d_first, 0xff, 4 * sizeof(uint32_t));
     check_div7<<<4096, 256>>>(0u, 0x7f800000u, d_bad, d_first);
     check_div_rcp<<<0x7bff, 256>>>(d_bad + 1, d_first + 1);
     check_ddiv_rcp<<<0x7bff, 256>>>(d_bad + 2, d_first + 2);
+    check_div15<<<4096, 256>>>(0u, 0x7f800000u, d_bad + 3, d_first + 3);
     if (cudaDeviceSynchronize() != cudaSuccess) return 2;
-    unsigned long long h_bad[3];
-    uint32_t h_first[3];
+    unsigned long long h_bad[4];
+    uint32_t h_first[4];
     cudaMemcpy(h_bad, d_bad, sizeof h_bad, cudaMemcpyDeviceToHost);
     cudaMemcpy(h_first, d_first, sizeof h_first, cudaMemcpyDeviceToHost);
     out[0] = h_bad[0];
@@ -87,6 +104,8 @@ extern "C" int run_checks(unsigned long long* out) {
     out[3] = h_first[1];
     out[4] = h_bad[2];
     out[5] = h_first[2];
+    out[6] = h_bad[3];
+    out[7] = h_first[3];
     cudaFree(d_bad);
     cudaFree(d_first);
     return 0;

@@ -82,7 +82,7 @@ def test_host_validation_without_a_gpu():
     assert search(n=9) == 1
     assert search(g=96) == 2
     assert search(n_grid=0) == 1 and search(n_grid=33) == 1
-    assert search(flags=4) == 1                      # an unknown flag bit
+    assert search(flags=8) == 1                      # an unknown flag bit
     assert search(flags=2, d_in=32768) == 2           # duo scaling: d_in <= 16384
     assert search(d_in=200) == 1
     assert search(W=(ctypes.c_void_p * 1)(odd)) == 3
@@ -99,6 +99,9 @@ def test_host_validation_without_a_gpu():
     assert L.awq_quantize_pack(fake, 64, 256, None, None, 128, 9, fake, fake, fake, None) == 1
     assert L.awq_quantize_pack(fake, 64, 256, None, None, 48, 8, fake, fake, fake, None) == 2
     assert L.awq_quantize_pack(fake, 64, 256, odd, None, 128, 8, fake, fake, fake, None) == 3
+    assert L.awq_quantize_pack(fake, 64, 256, None, None, 128, -2, fake, fake, fake, None) == 1
+    assert L.awq_quantize_pack(fake, 64, 256, None, fake, 128, -1, fake, fake, fake,
+                               None) == 2              # no clipping on the asymmetric grid
     # norm_group_scale
     ptrs1 = (ctypes.c_void_p * 1)(fake)
     ptrs_odd = (ctypes.c_void_p * 2)(fake, odd)
