@@ -7,8 +7,9 @@
 //   * a CTA owns 64 channels (8 chunks of 16 bytes) and one eighth of the
 //     tokens; the 8 CTAs of a thread-block cluster (1 x 8 x 1) cover all
 //     tokens of the same channels;
-//   * each thread walks its chunk down every 32nd row of its slice with eight
-//     16-byte loads in flight and adds |h| in fp64.  Every |fp16| is an
+//   * each thread walks its chunk down every 32nd row of its slice in
+//     batches of four 16-byte loads, the next batch issued before the
+//     current one is summed, and adds |h| in fp64.  Every |fp16| is an
 //     integer multiple of 2^-24 below 2^16, so a sum of up to 4096 of them is
 //     an integer multiple of 2^-24 below 2^28: exact in fp64.  Every 4096
 //     rows the fp64 sums are moved, exactly, into 64-bit integer counts of
@@ -35,7 +36,8 @@ namespace {
 constexpr int kCluster = 8;        // CTAs per cluster, splitting the tokens
 constexpr int kChunks = 8;         // 16-byte chunks per CTA (64 channels)
 constexpr int kRowLanes = 32;      // rows walked in parallel per CTA
-constexpr int kInFlight = 8;       // 16-byte loads in flight per thread
+constexpr int kBatch = 4;          // 16-byte loads per batch; the next batch is in flight
+                                   // while the current one is summed
 constexpr int kFlushRows = 4096;   // rows per thread between exact flushes
 
 // |h| as an fp64 value without the (slow-pipe) fp32 -> fp64 conversion: the
@@ -128,19 +130,37 @@ stats_kernel(const uint4* __restrict__ X, int64_t T, int64_t d_in, int64_t ld_ch
     const int sub = ry & 3;
     int64_t base = warp_row;
     int since_flush = 0;
-    for (; base + 3 + (kInFlight - 1) * kRowLanes < r1; base += kInFlight * kRowLanes) {
-        const int64_t r = base + sub;
-        uint4 v[kInFlight];
+    // software-pipelined batches: the loop's trip count depends only on the
+    // warp's first row (every lane of a warp runs it and the flush together)
+    uint4 cur[kBatch];
+    bool have = base + 3 + (kBatch - 1) * kRowLanes < r1;
+    if (have) {
 #pragma unroll
-        for (int k = 0; k < kInFlight; ++k)
-            v[k] = active ? __ldg(p + (r + k * kRowLanes) * ld_chunks) : make_uint4(0, 0, 0, 0);
+        for (int k = 0; k < kBatch; ++k)
+            cur[k] = active ? __ldg(p + (base + sub + k * kRowLanes) * ld_chunks)
+                            : make_uint4(0, 0, 0, 0);
+    }
+    while (have) {
+        const int64_t nb = base + kBatch * kRowLanes;
+        const bool have_next = nb + 3 + (kBatch - 1) * kRowLanes < r1;
+        uint4 nxt[kBatch];
+        if (have_next) {
 #pragma unroll
-        for (int k = 0; k < kInFlight; ++k) add_halves(v[k], acc, hmax);
-        since_flush += kInFlight;
+            for (int k = 0; k < kBatch; ++k)
+                nxt[k] = active ? __ldg(p + (nb + sub + k * kRowLanes) * ld_chunks)
+                                : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int k = 0; k < kBatch; ++k) add_halves(cur[k], acc, hmax);
+        since_flush += kBatch;
         if (since_flush >= kFlushRows) {
             flush(acc, hmax, cx, red, fred);
             since_flush = 0;
         }
+        base = nb;
+        have = have_next;
+#pragma unroll
+        for (int k = 0; k < kBatch; ++k) cur[k] = nxt[k];
     }
     for (int64_t r = base + sub; r < r1; r += kRowLanes)
         if (active) add_halves(__ldg(p + r * ld_chunks), acc, hmax);
