@@ -13,7 +13,8 @@
 //   wmean_partial_kernel   one CTA of 512 threads per SM, a contiguous range of
 //                          rows each; per row a block-wide max of |w|, then
 //                          every thread adds |w| / max for its own columns
-//                          into fp64 sums in shared memory (quotients
+//                          (at most 4 chunks of 8) into fp64 sums held in
+//                          registers (quotients
 //                          correctly rounded via ddiv_rn_rcp); the next row is
 //                          loaded while the current one is processed.  HBM
 //                          reads W once (2 B per weight).
@@ -64,12 +65,15 @@ __device__ __forceinline__ float chunk_absmax(const uint4 v) {
 
 __global__ void __launch_bounds__(kWmThreads, 1)
 wmean_partial_kernel(const __grid_constant__ WmParams p) {
-    extern __shared__ double acc[];                 // [d_in]
     __shared__ float red[2][kWmWarps];
     pdl_wait();   // W may come from the kernel before
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t chunks = p.d_in / 8;
-    for (int64_t j = tid; j < p.d_in; j += kWmThreads) acc[j] = 0.0;
+    double acc[kWmMaxChunks][8];                    // columns 8 * (tid + c * 512) + 0..7
+#pragma unroll
+    for (int c = 0; c < kWmMaxChunks; ++c)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[c][e] = 0.0;
     const int64_t r0 = p.rows * blockIdx.x / gridDim.x;
     const int64_t r1 = p.rows * (blockIdx.x + 1) / gridDim.x;
 
@@ -88,7 +92,6 @@ wmean_partial_kernel(const __grid_constant__ WmParams p) {
             cur[c] = ch < chunks ? __ldg(rp + ch) : z;
         }
     }
-    __syncthreads();   // acc cleared
     for (int64_t r = r0; r < r1; ++r) {
         if (r + 1 < r1) {   // the next row's loads are in flight while this one is summed
             const uint4* rp = row_ptr(r + 1);
@@ -121,8 +124,8 @@ wmean_partial_kernel(const __grid_constant__ WmParams p) {
                     for (int i = 0; i < 4; ++i) {
                         const double a0 = abs_half_to_double(w[i] & 0xffffu);
                         const double a1 = abs_half_to_double(w[i] >> 16);
-                        acc[8 * ch + 2 * i] += ddiv_rn_rcp(a0, mx, y);
-                        acc[8 * ch + 2 * i + 1] += ddiv_rn_rcp(a1, mx, y);
+                        acc[c][2 * i] += ddiv_rn_rcp(a0, mx, y);
+                        acc[c][2 * i + 1] += ddiv_rn_rcp(a1, mx, y);
                     }
                 }
             }
@@ -131,9 +134,16 @@ wmean_partial_kernel(const __grid_constant__ WmParams p) {
         for (int c = 0; c < kWmMaxChunks; ++c) cur[c] = nxt[c];
     }
     pdl_launch_dependents();
-    __syncthreads();
     double* out = p.partial + (int64_t)blockIdx.x * p.d_in;
-    for (int64_t j = tid; j < p.d_in; j += kWmThreads) out[j] = acc[j];
+#pragma unroll
+    for (int c = 0; c < kWmMaxChunks; ++c) {
+        const int64_t ch = tid + (int64_t)c * kWmThreads;
+        if (ch < chunks) {
+            double2* o2 = reinterpret_cast<double2*>(out + 8 * ch);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) o2[e] = make_double2(acc[c][2 * e], acc[c][2 * e + 1]);
+        }
+    }
 }
 
 __global__ void __launch_bounds__(256)
@@ -263,19 +273,7 @@ cudaError_t launch_duo_table(int n_seg, const void* const* W, const int64_t* d_o
     p.d_in = d_in;
     p.rows = rows;
     p.partial = partial;
-    const size_t smem = (size_t)d_in * sizeof(double);
-    static int configured[64] = {};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 0 || dev >= 64 || configured[dev] < (int)smem) {
-        cudaError_t e = cudaFuncSetAttribute(wmean_partial_kernel,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)smem);
-        if (e != cudaSuccess) return e;
-        if (dev >= 0 && dev < 64) configured[dev] = (int)smem;
-    }
-    cudaError_t e = launch_pdl(wmean_partial_kernel, dim3(grid), dim3(kWmThreads), smem, stream,
-                               p);
+    cudaError_t e = launch_pdl(wmean_partial_kernel, dim3(grid), dim3(kWmThreads), 0, stream, p);
     if (e != cudaSuccess) return e;
     const int fin_blocks = (int)std::min<int64_t>((d_in + 255) / 256, 4 * (int64_t)num_sms);
     e = launch_pdl(wmean_final_kernel, dim3(fin_blocks), dim3(256), 0, stream,
