@@ -61,7 +61,7 @@ FMA_OPS_PER_PAIR = 5
 # dram__bytes_read.sum + dram__bytes_write.sum of one launch of the dominant
 # kernel from the committed ncu captures (profiles/), for the kernels as they
 # stand; None where no capture of the current kernel exists.
-NCU_TRAFFIC = {"q_proj_4096x4096": 34249472,          # search_kernel<8,0>
+NCU_TRAFFIC = {"q_proj_4096x4096": 34248960,          # search_kernel<8,0,0>
                "down_proj_output_error": 3105129984}  # oe_gemm_kernel, per alpha
 FP32_LANES_PER_SM = 128
 DEFAULT_STEPS = {"single_linear_256x512": 1000, "q_proj_4096x4096": 1000,
