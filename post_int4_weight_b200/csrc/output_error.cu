@@ -30,7 +30,9 @@
 //                      (tcgen05.ld / st), so no accumulation chain inside the
 //                      tensor core is longer than 128 MMAs (its accumulation
 //                      does not round to nearest, and long chains drift
-//                      towards zero).  At the end of a tile each column is
+//                      towards zero).  The epilogue releases the accumulator
+//                      as soon as it has read it, so the next segment's MMAs
+//                      run while the running sum is updated.  At the end of a tile each column is
 //                      multiplied by 1/c_r (exact) and the squares summed.
 //                      X dW^T is never written out.
 // A final kernel sums the per-CTA partials of every grid point in a fixed
@@ -286,22 +288,28 @@ oe_gemm_kernel(const __grid_constant__ GemmParams p) {
                                 wait_or_abort(&tfull[0], seg & 1u, abort_flag, p.dev_err));
                 if (!ok) break;
                 tc_fence_after();
-#pragma unroll 1
+                // read the whole accumulator slice, then let the MMAs refill it
+                float a[kEpiCols];
+#pragma unroll
+                for (int c0 = 0; c0 < kEpiCols; c0 += 16) tmem_ld16(acc_addr + (uint32_t)c0, a + c0);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&tempty[0]);
+                // the running sum (columns the MMAs do not write) meanwhile
+#pragma unroll
                 for (int c0 = 0; c0 < kEpiCols; c0 += 16) {
                     float v[16];
-                    tmem_ld16(acc_addr + (uint32_t)c0, v);
                     if (sg > 0) {
-                        float r[16];
-                        tmem_ld16(run_addr + (uint32_t)c0, r);
+                        tmem_ld16(run_addr + (uint32_t)c0, v);
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) v[i] = __fadd_rn(v[i], r[i]);
+                        for (int i = 0; i < 16; ++i) v[i] = __fadd_rn(a[c0 + i], v[i]);
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) v[i] = a[c0 + i];
                     }
                     tmem_st16(run_addr + (uint32_t)c0, v);
                 }
                 tmem_wait_st();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&tempty[0]);
             }
             if (!ok) break;
             // the running sum holds this tile's slice of X dW^T
