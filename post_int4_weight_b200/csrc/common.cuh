@@ -136,6 +136,19 @@ __device__ __forceinline__ float div7_rn(float m) {
 // smaller m a value below 2^-25, which rounds to the same fp16 value (zero).
 // Used where only the fp16 rounding of the quotient matters; an infinite m
 // gives NaN.
+// The quotient a / b from y = RN(1 / b) with one residual correction, for
+// the rounding decision rint(a / b) only: it can differ from the IEEE
+// quotient by an ulp, which changes rint's result only within an ulp of a
+// half-integer; there it agrees with rint(__fdiv_rn(a, b)) for every fp16
+// divisor b and every a within 8 ulps of each half-integer multiple of b in
+// [-16 b, 16 b] (checked on the GPU).  Two-wide: the same operations as
+// __fmul2_rn / __ffma2_rn component by component.
+__device__ __forceinline__ float2 quot_rcp1_2(float2 a, float2 nb, float2 y) {
+    float2 q = __fmul2_rn(a, y);
+    const float2 r = __ffma2_rn(q, nb, a);
+    return __ffma2_rn(r, y, q);
+}
+
 // RN(m / 15) for finite m >= 0 (the asymmetric grid's scale): two residual
 // corrections of m * RN(1/15); tiny m, where a residual could underflow,
 // takes the IEEE division.  Checked against __fdiv_rn for every

@@ -18,8 +18,10 @@
 //   phase 2  two threads per (row, group): max |w*s| (NaN-propagating) ->
 //            q_scale, written to `scales`, and its correctly rounded
 //            reciprocal;
-//   phase 3  one thread per (2 columns, 32 rows): the IEEE quotient from the
-//            reciprocal with two residual corrections (div_rn_rcp), rounding
+//   phase 3  one thread per (2 columns, 32 rows): the quotient from the
+//            correctly rounded reciprocal with one residual correction,
+//            whose rounding decision is the IEEE quotient's (quot_rcp1_2,
+//            checked against __fdiv_rn around every half-integer), rounding
 //            by the 1.5*2^23 addition, nibble placement with one integer
 //            multiply-add per code, and one 16-byte store per column (four
 //            consecutive output words; four threads write 64 contiguous
@@ -93,12 +95,9 @@ __device__ __forceinline__ void pack_columns(const uint4* tile, const float2* qr
         const float2 a = __fmul2_rn(w, s2);
         const float2 nb2 = make_float2(-qs, -qs);
         const float2 y2 = make_float2(rq, rq);
-        // RN(a / qs): two residual corrections of a * RN(1/qs)
-        float2 q = __fmul2_rn(a, y2);
-        float2 res = __ffma2_rn(q, nb2, a);
-        q = __ffma2_rn(res, y2, q);
-        res = __ffma2_rn(q, nb2, a);
-        q = __ffma2_rn(res, y2, q);
+        // a / qs with one residual correction of a * RN(1/qs): its rounding
+        // decision is the IEEE quotient's (see quot_rcp1_2)
+        const float2 q = quot_rcp1_2(a, nb2, y2);
         float2 t = __fadd2_rn(q, magic2);
         if (kAsym) {
             const float z = (float)zero_tile[row_slot(kk, r)];

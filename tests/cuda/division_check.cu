@@ -78,24 +78,48 @@ __global__ void check_ddiv_rcp(unsigned long long* bad, uint32_t* first_bad_b) {
     }
 }
 
+// for every positive finite fp16 divisor b, numerators around every
+// half-integer multiple of b in [-16b, 16b] (+-8 ulps): the rounding decision
+// of the one-correction quotient (pack's codes) against rint(__fdiv_rn)
+__global__ void check_code_rcp1(unsigned long long* bad, uint32_t* first_bad_b) {
+    const uint32_t hb = blockIdx.x + 1;           // 0x0001 .. 0x7bff
+    const float b = __half2float(__ushort_as_half((unsigned short)hb));
+    const float y = __frcp_rn(b);
+    for (int t = threadIdx.x; t < 32 * 17 * 2; t += blockDim.x) {
+        const int k = t / 34, d = (t % 34) / 2, sgn = t & 1;
+        const float base = __fmul_rn((float)(k - 16) + 0.5f, b);
+        float a = __uint_as_float(__float_as_uint(base) + (uint32_t)(d - 8));
+        if (sgn) a = -a;
+        if (!(fabsf(a) <= 3.0e38f)) continue;
+        const float2 q = awq::quot_rcp1_2(make_float2(a, a), make_float2(-b, -b),
+                                          make_float2(y, y));
+        if (__float_as_uint(rintf(q.x)) != __float_as_uint(rintf(__fdiv_rn(a, b)))) {
+            atomicAdd(bad, 1ull);
+            atomicMin(first_bad_b, hb);
+        }
+    }
+}
+
 extern "C" int run_checks(unsigned long long* out) {
     // out[0]: div7 mismatches, out[1]: first bad bits, out[2]: div_rcp
     // mismatches, out[3]: first bad fp16 divisor, out[4]: ddiv_rcp
     // mismatches, out[5]: its first bad fp16 divisor, out[6]: div15
-    // mismatches, out[7]: first bad bits
+    // mismatches, out[7]: first bad bits, out[8]: one-correction code
+    // decision mismatches, out[9]: its first bad fp16 divisor
     unsigned long long* d_bad;
     uint32_t* d_first;
-    if (cudaMalloc(&d_bad, 4 * sizeof(unsigned long long)) != cudaSuccess) return 1;
-    if (cudaMalloc(&d_first, 4 * sizeof(uint32_t)) != cudaSuccess) return 1;
-    cudaMemset(d_bad, 0, 4 * sizeof(unsigned long long));
-    cudaMemset(d_first, 0xff, 4 * sizeof(uint32_t));
+    if (cudaMalloc(&d_bad, 5 * sizeof(unsigned long long)) != cudaSuccess) return 1;
+    if (cudaMalloc(&d_first, 5 * sizeof(uint32_t)) != cudaSuccess) return 1;
+    cudaMemset(d_bad, 0, 5 * sizeof(unsigned long long));
+    cudaMemset(d_first, 0xff, 5 * sizeof(uint32_t));
     check_div7<<<4096, 256>>>(0u, 0x7f800000u, d_bad, d_first);
     check_div_rcp<<<0x7bff, 256>>>(d_bad + 1, d_first + 1);
     check_ddiv_rcp<<<0x7bff, 256>>>(d_bad + 2, d_first + 2);
     check_div15<<<4096, 256>>>(0u, 0x7f800000u, d_bad + 3, d_first + 3);
+    check_code_rcp1<<<0x7bff, 256>>>(d_bad + 4, d_first + 4);
     if (cudaDeviceSynchronize() != cudaSuccess) return 2;
-    unsigned long long h_bad[4];
-    uint32_t h_first[4];
+    unsigned long long h_bad[5];
+    uint32_t h_first[5];
     cudaMemcpy(h_bad, d_bad, sizeof h_bad, cudaMemcpyDeviceToHost);
     cudaMemcpy(h_first, d_first, sizeof h_first, cudaMemcpyDeviceToHost);
     out[0] = h_bad[0];
@@ -106,6 +130,8 @@ extern "C" int run_checks(unsigned long long* out) {
     out[5] = h_first[2];
     out[6] = h_bad[3];
     out[7] = h_first[3];
+    out[8] = h_bad[4];
+    out[9] = h_first[4];
     cudaFree(d_bad);
     cudaFree(d_first);
     return 0;

@@ -29,9 +29,11 @@ def test_division_helpers_equal_ieee_division():
                         "-O3", "-std=c++17", "-Xcompiler", "-fPIC", "-shared", "-I" + inc,
                         src, "-o", so], check=True)
         lib = ctypes.CDLL(so)
-        out = (ctypes.c_ulonglong * 8)()
+        out = (ctypes.c_ulonglong * 10)()
         assert lib.run_checks(out) == 0
     assert out[0] == 0, f"div7_rn differs from IEEE for {out[0]} values, first bits {out[1]:#x}"
     assert out[2] == 0, f"div_rn_rcp differs for {out[2]} pairs, first fp16 divisor {out[3]:#x}"
     assert out[4] == 0, f"ddiv_rn_rcp differs for {out[4]} pairs, first fp16 divisor {out[5]:#x}"
     assert out[6] == 0, f"div15_rn differs from IEEE for {out[6]} values, first bits {out[7]:#x}"
+    assert out[8] == 0, (f"one-correction code decision differs for {out[8]} pairs, "
+                         f"first fp16 divisor {out[9]:#x}")
