@@ -362,6 +362,8 @@ def run_ours(a):
     e2e = {"value": _total_params(work, world, params) / (ms_e2e * 1e-3) / 1e9, "unit": UNIT,
            "ms_per_step": ms_e2e, "h2d_bytes_per_step": int(h2d_l * per_step_layers),
            "d2h_bytes_per_step": int(d2h_l * per_step_layers), "steps": e2e_units,
+           # the copies bound this number: host->device bytes over the step time
+           "h2d_GBps": h2d_l * per_step_layers / (ms_e2e * 1e-3) / 1e9,
            "pipeline": "pinned host -> 2-slot device ring; H2D, kernels and D2H on three "
                        "streams, overlapped across layers"}
 
