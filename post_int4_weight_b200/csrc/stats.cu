@@ -112,7 +112,9 @@ stats_kernel(const uint4* __restrict__ X, int64_t T, int64_t d_in, int64_t ld_ch
         red[tid] = 0;
         fred[tid] = 0;
     }
-    cluster.sync();   // every CTA's accumulators are cleared before remote adds
+    // every CTA's accumulators must be cleared before other CTAs add into
+    // them: arrive now, wait just before the remote adds (after the loads)
+    cluster.barrier_arrive();
 
     const int64_t chunk = (int64_t)blockIdx.x * kChunks + cx;
     const bool active = chunk * 8 < d_in;
@@ -167,6 +169,7 @@ stats_kernel(const uint4* __restrict__ X, int64_t T, int64_t d_in, int64_t ld_ch
     pdl_launch_dependents();   // X is read; the next kernel may start launching
     flush(acc, hmax, cx, red, fred);
     __syncthreads();
+    cluster.barrier_wait();
     if (rank != 0 && tid < kChunks * 8) {
         unsigned long long* red0 = cluster.map_shared_rank(red, 0);
         uint32_t* fred0 = cluster.map_shared_rank(fred, 0);
