@@ -104,3 +104,12 @@ def test_asym_nonfinite_reports_minus_one():
     err, best, s = awq.scale_search([W.cuda()], x, 128, 20, awq.ASYMMETRIC)
     torch.cuda.synchronize()
     assert int(best.cpu()[0]) == -1 and np.isnan(s.cpu().numpy()).all()
+
+
+def test_asym_duo_stack_layer_gate_up():
+    """The 36-layer stack's gate/up group (2 x 12288 rows, 2048 tokens) with
+    the asymmetric grid and duo scaling together."""
+    work = wl.WORKLOADS["qwen3_8b_stack36"]
+    grp, Ws, X = wl.group_inputs(work, 17)[2]
+    s = _search_both(Ws, X, 128, awq.ASYMMETRIC | awq.DUO_SCALING)
+    _pack_both(Ws[1], s, 128)

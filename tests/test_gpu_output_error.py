@@ -101,3 +101,15 @@ def test_output_error_fp32_scale_and_nonfinite():
     W[5, 9] = float("nan")
     err_g, best_g = _run(X, W, x, 128)
     assert best_g == -1 and np.isnan(err_g).all()
+
+
+@pytest.mark.parametrize("n_grid", [1, 32])
+def test_output_error_grid_sizes(n_grid):
+    W = wl.weight(64, 256, 31 + n_grid)
+    X = wl.activations(48, 256, 32 + n_grid)
+    x = oracle.act_stats(X.numpy())
+    err_g, best_g = _run(X, W, x, 64, n_grid)
+    err_o = oracle.output_error(X.numpy(), W.numpy(), x, 64, n_grid)
+    _check(err_g, best_g, err_o)
+    if n_grid == 1:
+        assert best_g == 0
