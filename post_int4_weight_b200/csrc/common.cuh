@@ -183,18 +183,27 @@ __device__ __forceinline__ float div_rn_rcp(float a, float b, float y) {
     return __fmaf_rn(r, y, q);
 }
 
-// RN(a / b) in fp64 for finite a >= 0 and b > 0 from y = RN(1 / b): the
-// product a*y is within about one ulp of the quotient, and each residual
-// a - q*b (exact in an FMA) corrects it (Markstein's construction); two
-// corrections give the correctly rounded quotient.  Used for |w| / max|w|
-// of fp16 values, checked against __ddiv_rn for every pair of non-negative
-// fp16 values.
+// RN(a / b) in fp64 from y = RN(1 / b): the product a*y is within about one
+// ulp of the quotient and the residual a - q*b is exact in an FMA, so one
+// correction q + r*y gives the correctly rounded quotient (Markstein's
+// construction).  Used for |w| / max|w| of fp16 values, where it is exact
+// for every pair of non-negative finite fp16 values with b > 0 (checked
+// against __ddiv_rn for all of them, also in the scaled form below).
 __device__ __forceinline__ double ddiv_rn_rcp(double a, double b, double y) {
-    double q = __dmul_rn(a, y);
-    double r = __fma_rn(-q, b, a);
-    q = __fma_rn(r, y, q);
-    r = __fma_rn(-q, b, a);
+    const double q = __dmul_rn(a, y);
+    const double r = __fma_rn(-q, b, a);
     return __fma_rn(r, y, q);
+}
+
+// A non-negative finite fp32 value as an fp64 scaled by 2^-896: the fp32
+// bits shifted right by 3 put its exponent field in the low bits of the fp64
+// exponent field, so the result is exactly v * 2^(127 - 1023) (a normal
+// fp64 for every nonzero fp32 value, and 0 for 0).  For quotients of fp16
+// values both operands take the same scale: the scaled reciprocal of a
+// divisor in [2^-24, 65504] stays normal and the residual of ddiv_rn_rcp
+// stays exact, so the scaled quotient is the same number.
+__device__ __forceinline__ double f32_scaled_f64(float v) {
+    return __hiloint2double((int)(__float_as_uint(v) >> 3), 0);
 }
 
 // Group scale from the group's largest |w * s| (round-to-nearest-even

@@ -53,7 +53,7 @@ cudaError_t launch_quantize_pack(const void* W, int64_t d_out, int64_t d_in,
 // ---- duo scaling (the scale table from x and the weights' row-normalised
 // mean); its workspace follows the search workspace
 constexpr int kDuoMaxSms = 160;        // weight-mean CTAs (one per SM, at most this many)
-constexpr int64_t kDuoMaxDin = 16384;  // the weight-mean pass keeps d_in fp64 sums in smem
+constexpr int64_t kDuoMaxDin = 16384;  // the weight-mean pass: at most 4 chunks of 8 per thread
 size_t duo_workspace(int64_t d_in, int num_sms, int n_grid);
 size_t duo_workspace_bound(int64_t d_in, int n_grid);
 cudaError_t launch_duo_table(int n_seg, const void* const* W, const int64_t* d_out, int64_t d_in,

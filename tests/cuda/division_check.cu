@@ -62,16 +62,24 @@ __global__ void check_div_rcp(unsigned long long* bad, uint32_t* first_bad_b) {
 }
 
 // every pair (a, b) of non-negative finite fp16 values with b > 0 (blockIdx.x
-// selects b): ddiv_rn_rcp against the IEEE fp64 quotient __ddiv_rn
+// selects b): ddiv_rn_rcp against the IEEE fp64 quotient __ddiv_rn, both on
+// the plain fp64 values and in the form the weight-mean kernel uses (both
+// operands scaled by 2^-896 through f32_scaled_f64, the reciprocal of the
+// scaled divisor)
 __global__ void check_ddiv_rcp(unsigned long long* bad, uint32_t* first_bad_b) {
     const uint32_t hb = blockIdx.x + 1;           // 0x0001 .. 0x7bff
-    const double b = (double)__half2float(__ushort_as_half((unsigned short)hb));
+    const float bf = __half2float(__ushort_as_half((unsigned short)hb));
+    const double b = (double)bf;
     const double y = __drcp_rn(b);
+    const double bs = awq::f32_scaled_f64(bf);
+    const double ys = __drcp_rn(bs);
     for (uint32_t ha = threadIdx.x; ha <= 0x7bffu; ha += blockDim.x) {
-        const double a = (double)__half2float(__ushort_as_half((unsigned short)ha));
-        const double q = awq::ddiv_rn_rcp(a, b, y);
-        const double r = __ddiv_rn(a, b);
-        if (__double_as_longlong(q) != __double_as_longlong(r)) {
+        const float af = __half2float(__ushort_as_half((unsigned short)ha));
+        const double r = __ddiv_rn((double)af, b);
+        const double q = awq::ddiv_rn_rcp((double)af, b, y);
+        const double qs = awq::ddiv_rn_rcp(awq::f32_scaled_f64(af), bs, ys);
+        if (__double_as_longlong(q) != __double_as_longlong(r) ||
+            __double_as_longlong(qs) != __double_as_longlong(r)) {
             atomicAdd(bad, 1ull);
             atomicMin(first_bad_b, hb);
         }

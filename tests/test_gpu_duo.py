@@ -1,7 +1,8 @@
 """Duo scaling (AWQ_DUO_SCALING) on the GPU against the CPU oracle.
 
 The weight mean is an fp64 sum whose order differs between the two sides
-(rows in order on the CPU; row blocks, then blocks in order on the GPU), so
+(rows in order on the CPU; row blocks, then the blocks' sums in a fixed
+order on the GPU), so
 an fp32 entry of the scale table may differ by one ulp when it lies within
 ~1e-16 of a rounding boundary; the chosen scale is compared bit for bit
 except for such entries, and the pack is compared bit for bit at the GPU's
@@ -46,7 +47,12 @@ def _duo_case(Ws, X, g=128, n_grid=20):
 
 
 @pytest.mark.parametrize("shape", [((256,), 512, 64), ((200, 72, 8), 1024, 96),
-                                   ((4096,), 4096, 256)])
+                                   ((4096,), 4096, 256),
+                                   # wider rows: 2, 3 and 4 chunks of 8 per thread of
+                                   # the weight-mean pass; 600 rows give its CTAs
+                                   # several batches, 40-64 rows leave most CTAs idle
+                                   ((600,), 8192, 32), ((48, 16), 12288, 32),
+                                   ((40,), 16384, 32)])
 def test_duo_search_parity(shape):
     d_outs, d_in, T = shape
     seed = sum(d_outs) + d_in
@@ -88,3 +94,32 @@ def test_duo_rejects_wide_inputs_and_small_workspace():
     small = awq.workspace(awq.OP_SCALE_SEARCH, "cuda", 1, 8, 1024, 128, 20)
     with pytest.raises(awq.AwqError):
         awq.scale_search([W2], x2, 128, 20, awq.DUO_SCALING, ws=small)
+
+
+def test_duo_subnormal_rows():
+    """Rows whose largest |w| is an fp16 subnormal, a row of subnormals and
+    zeros, and a row mixing subnormal and normal magnitudes."""
+    W = wl.weight(64, 256, 7)
+    W[5] = W[5] * 1e-3              # largest |w| below 2^-14
+    W[6] = W[6] * 1e-4              # deep subnormals, some rounded to 0
+    W[9, ::3] = W[9, ::3] * 1e-3    # mixed within one row
+    assert float(W[5].abs().max()) < 6.1035e-05
+    X = wl.activations(32, 256, 8)
+    _duo_case([W], X)
+
+
+def test_duo_nonfinite_weight_reports_minus_one():
+    """A NaN and an inf weight: the weighted errors are not finite on either
+    side, so both report index -1 and the GPU a NaN scale vector."""
+    W = wl.weight(64, 256, 9)
+    W[3, 17] = float("nan")
+    W[10, 40] = float("inf")
+    X = wl.activations(16, 256, 10)
+    x_g = awq.act_stats(X.cuda())
+    err, best, s = awq.scale_search([W.cuda()], x_g, 128, 20, awq.DUO_SCALING)
+    torch.cuda.synchronize()
+    x = oracle.act_stats(X.numpy())
+    err_o, best_o, _ = oracle.scale_search([W.numpy()], x, 128, 20, oracle.DUO)
+    assert best_o == -1 and int(best.cpu()[0]) == -1
+    assert np.all(np.isnan(s.cpu().numpy()))
+    assert np.array_equal(np.isfinite(err.cpu().numpy()), np.isfinite(err_o))
