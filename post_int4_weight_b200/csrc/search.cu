@@ -278,9 +278,15 @@ __device__ __forceinline__ float2 row_products_minmax(const float2* w, const flo
 // The row's scale fp16(max(max - min, 1e-5) / 15) (exact quotient), its
 // zero point clamp(rint(-min / q_scale), 0, 15) (exact quotient), the
 // rounding constant 1.5*2^23 + zero and an approximate reciprocal for the
-// codes.  A non-finite ws makes the row's error non-finite by itself.
+// codes.  *in_range: the codes of the row's smallest and largest ws, taken
+// by the same FMA as the codes pass, lie in 0..15; that FMA is monotonic in
+// ws, so then no code of the row needs the clamp.  A non-finite ws makes
+// the row's error non-finite by itself: its residual is NaN with or without
+// the clamp (an inf also makes in_range false; a NaN is skipped by the
+// row's min and max).
 template <int L, bool kFp32>
-__device__ __forceinline__ void row_scale_asym(float2 mm, float* qs, float* rq, float* mz) {
+__device__ __forceinline__ void row_scale_asym(float2 mm, float* qs, float* rq, float* mz,
+                                               bool* in_range) {
     float mx = mm.x, mn = mm.y;
 #pragma unroll
     for (int o = 1; o < L; o <<= 1) {
@@ -291,15 +297,18 @@ __device__ __forceinline__ void row_scale_asym(float2 mm, float* qs, float* rq, 
     float q = div15_rn(range);
     if (!kFp32) q = fminf(__half2float(__float2half_rn(q)), kHalfMax);
     const float z = fminf(fmaxf(rintf(div_rn_rcp(-mn, q, __frcp_rn(q))), 0.f), 15.f);
+    const float r = rcp_approx(q);
     *qs = q;
-    *rq = rcp_approx(q);
+    *rq = r;
     *mz = kRoundMagic + z;
+    *in_range = (__fmaf_rn(mn, r, kRoundMagic + z) >= kRoundMagic) &
+                (__fmaf_rn(mx, r, kRoundMagic + z) <= kRoundMagic + 15.f);
 }
 
 // Pass 2 on the asymmetric grid: codes clamp(rint(ws / q_scale) + zero, 0, 15)
-// by the rounding addition of 1.5*2^23 + zero, then the same weighted sum as
-// rows_errors.
-template <int L>
+// by the rounding addition of 1.5*2^23 + zero (the clamp only when some row
+// of the warp may leave 0..15), then the same weighted sum as rows_errors.
+template <bool kClamp, int L>
 __device__ __forceinline__ float2 rows_errors_asym(const float2* ws0, const float2* ws1,
                                                    const float4* T2, int l, float qs0,
                                                    float rq0, float mz0, float qs1, float rq1,
@@ -315,9 +324,13 @@ __device__ __forceinline__ float2 rows_errors_asym(const float2* ws0, const floa
         for (int j = 0; j < 2; ++j) {
             const int i = 2 * k + j;
             float2 t0 = __ffma2_rn(ws0[i], rq02, mz02);
-            t0 = f2(fminf(fmaxf(t0.x, lo), hi), fminf(fmaxf(t0.y, lo), hi));
-            float t1x = fminf(fmaxf(__fmaf_rn(ws1[i].x, rq1, mz1), lo), hi);
-            float t1y = fminf(fmaxf(__fmaf_rn(ws1[i].y, rq1, mz1), lo), hi);
+            float t1x = __fmaf_rn(ws1[i].x, rq1, mz1);
+            float t1y = __fmaf_rn(ws1[i].y, rq1, mz1);
+            if (kClamp) {
+                t0 = f2(fminf(fmaxf(t0.x, lo), hi), fminf(fmaxf(t0.y, lo), hi));
+                t1x = fminf(fmaxf(t1x, lo), hi);
+                t1y = fminf(fmaxf(t1y, lo), hi);
+            }
             const float2 q0 = __fadd2_rn(t0, nmz02);
             const float2 q1 = f2(__fadd_rn(t1x, -mz1), __fadd_rn(t1y, -mz1));
             const float2 d0 = __ffma2_rn(q0, nqs0, ws0[i]);
@@ -482,9 +495,15 @@ search_kernel(const __grid_constant__ SearchParams p) {
                 const float2 mm0 = row_products_minmax(w[0], s4, ws[0]);
                 const float2 mm1 = row_products_minmax(w[1], s4, ws[1]);
                 float qs0, rq0, mz0, qs1, rq1, mz1;
-                row_scale_asym<L, kFp32>(mm0, &qs0, &rq0, &mz0);
-                row_scale_asym<L, kFp32>(mm1, &qs1, &rq1, &mz1);
-                e = rows_errors_asym<L>(ws[0], ws[1], Ta, l, qs0, rq0, mz0, qs1, rq1, mz1);
+                bool in0, in1;
+                row_scale_asym<L, kFp32>(mm0, &qs0, &rq0, &mz0, &in0);
+                row_scale_asym<L, kFp32>(mm1, &qs1, &rq1, &mz1, &in1);
+                if (__all_sync(0xffffffffu, in0 & in1))
+                    e = rows_errors_asym<false, L>(ws[0], ws[1], Ta, l, qs0, rq0, mz0, qs1, rq1,
+                                                   mz1);
+                else   // a row whose extreme codes leave 0..15 (or an infinite ws)
+                    e = rows_errors_asym<true, L>(ws[0], ws[1], Ta, l, qs0, rq0, mz0, qs1, rq1,
+                                                  mz1);
                 acc[a * kThreads + tid] += e.x + e.y;
                 continue;
             }
@@ -577,6 +596,17 @@ table_kernel(const float* __restrict__ x, int64_t d_in, int n_grid, int64_t slic
         dev_words[0] = 0;
         dev_words[1] = 0;
     }
+    // The thread's first channel: its pow does not depend on the reduction
+    // below, so it is taken first and its latency overlaps the reduction's.
+    const double alpha = __ddiv_rn((double)a, (double)n_grid);
+    const int64_t j0 = (int64_t)sl * slice, j1 = min(d_in, j0 + slice);
+    const int64_t jf = j0 + threadIdx.x;
+    float xf = 1.f;
+    double pf = 1.0;
+    if (jf < j1) {
+        xf = x[jf];
+        pf = table_pow(xf, alpha);
+    }
     // x is 16-byte aligned and d_in % 32 == 0: 16-byte loads, eight in
     // flight per thread (max and min are order-independent)
     float mx = 0.f, mn = __int_as_float(0x7f800000);
@@ -613,12 +643,11 @@ table_kernel(const float* __restrict__ x, int64_t d_in, int n_grid, int64_t slic
         mx = fmaxf(mx, red_mx[k]);
         mn = fminf(mn, red_mn[k]);
     }
-    const double alpha = __ddiv_rn((double)a, (double)n_grid);
     const double norm = __dsqrt_rn(__dmul_rn(table_pow(mx, alpha), table_pow(mn, alpha)));
-    const int64_t j0 = (int64_t)sl * slice, j1 = min(d_in, j0 + slice);
-    for (int64_t j = j0 + threadIdx.x; j < j1; j += blockDim.x) {
-        const float xj = x[j];
-        const float s = __double2float_rn(__ddiv_rn(table_pow(xj, alpha), norm));
+    for (int64_t j = jf; j < j1; j += blockDim.x) {
+        const float xj = j == jf ? xf : x[j];
+        const double pj = j == jf ? pf : table_pow(xj, alpha);
+        const float s = __double2float_rn(__ddiv_rn(pj, norm));
         S[(int64_t)a * d_in + j] = s;
         float t;
         if (kind == kTableInverse) {
@@ -708,9 +737,10 @@ size_t scale_search_workspace(int64_t d_in, int group_size, int n_grid) {
 cudaError_t launch_scale_table(const float* x_mean, int64_t d_in, int n_grid, float* S,
                                float* T, int* dev_words, int num_sms, cudaStream_t stream,
                                TableKind kind) {
-    int64_t slices = (2 * (int64_t)num_sms + n_grid - 1) / n_grid;
-    slices = std::min<int64_t>(slices, (d_in + 63) / 64);
-    slices = std::max<int64_t>(1, std::min<int64_t>(slices, kMaxTableSlices));
+    (void)num_sms;
+    // one channel per thread where d_in allows (every CTA also reads all of x
+    // for the row's max and min, so the slice count stays bounded)
+    int64_t slices = std::max<int64_t>(1, std::min<int64_t>((d_in + 255) / 256, kMaxTableSlices));
     const int64_t slice = (d_in + slices - 1) / slices;
     slices = (d_in + slice - 1) / slice;
     const dim3 grid((unsigned)slices, (unsigned)n_grid);
