@@ -191,26 +191,37 @@ __device__ __forceinline__ float row_products(const float2* w, const float4* s4,
     return fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
 }
 
-// q_scale of a row from its largest |ws| (the lane-local maxima combined
-// over the row's L lanes), its approximate reciprocal, and whether every
-// |ws| / q_scale of the row is known to stay below 7.5 (then the code needs
-// no clamp and the reciprocal is finite).  Non-finite ws need no flag here:
-// they make the row's error non-finite on their own.
+// q_scale of each of a lane's two rows from its largest |ws| (the lane-local
+// maxima combined over the row's L lanes), its approximate reciprocal, and
+// whether every |ws| / q_scale of the row is known to stay below 7.5 (then
+// the code needs no clamp and the reciprocal is finite).  Non-finite ws need
+// no flag here: they make the row's error non-finite on their own.  Even
+// lanes finish row 0 and odd lanes row 1 (one exchange with the neighbour,
+// then the butterfly over the row's remaining lanes), each lane computes one
+// q_scale, and the pair shares the results; *in_range covers the row this
+// lane computed, and every row of the warp is computed by some lane.
 template <int L, bool kFp32>
-__device__ __forceinline__ void row_scale(float m, float* qs, float* rq, bool* in_range) {
+__device__ __forceinline__ void rows_scale(float m0, float m1, int lane, float* qs0, float* rq0,
+                                           float* qs1, float* rq1, bool* in_range) {
+    const bool odd = (lane & 1) != 0;
+    float m = fmaxf(odd ? m1 : m0, __shfl_xor_sync(0xffffffffu, odd ? m0 : m1, 1));
 #pragma unroll
-    for (int o = 1; o < L; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    for (int o = 2; o < L; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    float q;
     if (kFp32) {
-        const float q = div7_rn(m);
-        *qs = q;
+        q = div7_rn(m);
         *in_range = q >= kFloatMinNormal && q <= 3.402823466e38f;
     } else {
-        const float qsf = div7_rn_for_fp16(m);
-        const float q = __half2float(__float2half_rn(qsf));
-        *in_range = (q >= kHalfMinNormal) & (q <= kHalfMax);
-        *qs = fminf(q, kHalfMax);
+        const float h = __half2float(__float2half_rn(div7_rn_for_fp16(m)));
+        *in_range = (h >= kHalfMinNormal) & (h <= kHalfMax);
+        q = fminf(h, kHalfMax);
     }
-    *rq = rcp_approx(*qs);
+    const float r = rcp_approx(q);
+    const int even = lane & ~1;
+    *qs0 = __shfl_sync(0xffffffffu, q, even);
+    *qs1 = __shfl_sync(0xffffffffu, q, even | 1);
+    *rq0 = __shfl_sync(0xffffffffu, r, even);
+    *rq1 = __shfl_sync(0xffffffffu, r, even | 1);
 }
 
 // Pass 2 of a lane's two rows for one alpha: codes (no clamp when the whole
@@ -275,21 +286,26 @@ __device__ __forceinline__ float2 row_products_minmax(const float2* w, const flo
     return f2(mx, mn);
 }
 
-// The row's scale fp16(max(max - min, 1e-5) / 15) (exact quotient), its
-// zero point clamp(rint(-min / q_scale), 0, 15) (exact quotient), the
-// rounding constant 1.5*2^23 + zero and an approximate reciprocal for the
-// codes.  *in_range: the codes of the row's smallest and largest ws, taken
-// by the same FMA as the codes pass, lie in 0..15; that FMA is monotonic in
-// ws, so then no code of the row needs the clamp.  A non-finite ws makes
-// the row's error non-finite by itself: its residual is NaN with or without
-// the clamp (an inf also makes in_range false; a NaN is skipped by the
-// row's min and max).
+// For each of a lane's two rows: the scale fp16(max(max - min, 1e-5) / 15)
+// (exact quotient), the zero point clamp(rint(-min / q_scale), 0, 15) (exact
+// quotient), the rounding constant 1.5*2^23 + zero and an approximate
+// reciprocal for the codes, split between the lanes of each pair as in
+// rows_scale.  *in_range: the codes of the row's smallest and largest ws,
+// taken by the same FMA as the codes pass, lie in 0..15; that FMA is
+// monotonic in ws, so then no code of the row needs the clamp.  A non-finite
+// ws makes the row's error non-finite by itself: its residual is NaN with or
+// without the clamp (an inf also makes in_range false; a NaN is skipped by
+// the row's min and max).
 template <int L, bool kFp32>
-__device__ __forceinline__ void row_scale_asym(float2 mm, float* qs, float* rq, float* mz,
-                                               bool* in_range) {
-    float mx = mm.x, mn = mm.y;
+__device__ __forceinline__ void rows_scale_asym(float2 mm0, float2 mm1, int lane, float* qs0,
+                                                float* rq0, float* mz0, float* qs1, float* rq1,
+                                                float* mz1, bool* in_range) {
+    const bool odd = (lane & 1) != 0;
+    const float2 own = odd ? mm1 : mm0, other = odd ? mm0 : mm1;
+    float mx = fmaxf(own.x, __shfl_xor_sync(0xffffffffu, other.x, 1));
+    float mn = fminf(own.y, __shfl_xor_sync(0xffffffffu, other.y, 1));
 #pragma unroll
-    for (int o = 1; o < L; o <<= 1) {
+    for (int o = 2; o < L; o <<= 1) {
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
         mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
     }
@@ -298,11 +314,15 @@ __device__ __forceinline__ void row_scale_asym(float2 mm, float* qs, float* rq, 
     if (!kFp32) q = fminf(__half2float(__float2half_rn(q)), kHalfMax);
     const float z = fminf(fmaxf(rintf(div_rn_rcp(-mn, q, __frcp_rn(q))), 0.f), 15.f);
     const float r = rcp_approx(q);
-    *qs = q;
-    *rq = r;
-    *mz = kRoundMagic + z;
-    *in_range = (__fmaf_rn(mn, r, kRoundMagic + z) >= kRoundMagic) &
-                (__fmaf_rn(mx, r, kRoundMagic + z) <= kRoundMagic + 15.f);
+    const float mz = kRoundMagic + z;
+    *in_range = (__fmaf_rn(mn, r, mz) >= kRoundMagic) & (__fmaf_rn(mx, r, mz) <= kRoundMagic + 15.f);
+    const int even = lane & ~1;
+    *qs0 = __shfl_sync(0xffffffffu, q, even);
+    *qs1 = __shfl_sync(0xffffffffu, q, even | 1);
+    *rq0 = __shfl_sync(0xffffffffu, r, even);
+    *rq1 = __shfl_sync(0xffffffffu, r, even | 1);
+    *mz0 = __shfl_sync(0xffffffffu, mz, even);
+    *mz1 = __shfl_sync(0xffffffffu, mz, even | 1);
 }
 
 // Pass 2 on the asymmetric grid: codes clamp(rint(ws / q_scale) + zero, 0, 15)
@@ -495,10 +515,10 @@ search_kernel(const __grid_constant__ SearchParams p) {
                 const float2 mm0 = row_products_minmax(w[0], s4, ws[0]);
                 const float2 mm1 = row_products_minmax(w[1], s4, ws[1]);
                 float qs0, rq0, mz0, qs1, rq1, mz1;
-                bool in0, in1;
-                row_scale_asym<L, kFp32>(mm0, &qs0, &rq0, &mz0, &in0);
-                row_scale_asym<L, kFp32>(mm1, &qs1, &rq1, &mz1, &in1);
-                if (__all_sync(0xffffffffu, in0 & in1))
+                bool in;
+                rows_scale_asym<L, kFp32>(mm0, mm1, lane, &qs0, &rq0, &mz0, &qs1, &rq1, &mz1,
+                                          &in);
+                if (__all_sync(0xffffffffu, in))
                     e = rows_errors_asym<false, L>(ws[0], ws[1], Ta, l, qs0, rq0, mz0, qs1, rq1,
                                                    mz1);
                 else   // a row whose extreme codes leave 0..15 (or an infinite ws)
@@ -510,10 +530,9 @@ search_kernel(const __grid_constant__ SearchParams p) {
             const float m0 = row_products(w[0], s4, ws[0]);
             const float m1 = row_products(w[1], s4, ws[1]);
             float qs0, rq0, qs1, rq1;
-            bool in0, in1;
-            row_scale<L, kFp32>(m0, &qs0, &rq0, &in0);
-            row_scale<L, kFp32>(m1, &qs1, &rq1, &in1);
-            if (__all_sync(0xffffffffu, in0 & in1)) {
+            bool in;
+            rows_scale<L, kFp32>(m0, m1, lane, &qs0, &rq0, &qs1, &rq1, &in);
+            if (__all_sync(0xffffffffu, in)) {
                 e = rows_errors<false, L>(ws[0], ws[1], Ta, l, qs0, rq0, qs1, rq1);
             } else {   // some row has an fp16-subnormal, overflowing, zero or NaN scale
                 e = rows_errors<true, L>(ws[0], ws[1], Ta, l, qs0, rq0, qs1, rq1);
