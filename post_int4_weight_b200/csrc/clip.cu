@@ -83,13 +83,6 @@ __device__ __forceinline__ float lane_error(const float2* ws, const float2* t2, 
 }
 
 template <int L>
-__device__ __forceinline__ float row_sum(float v) {
-#pragma unroll
-    for (int o = 1; o < L; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    return v;
-}
-
-template <int L>
 __device__ __forceinline__ float row_max(float v) {
 #pragma unroll
     for (int o = 1; o < L; o <<= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
@@ -109,7 +102,7 @@ clip_kernel(const ClipParams p) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int l = lane % L, slot = lane / L;
     const int64_t ld = p.d_in / 8;
-    double tot0 = 0.0, tot1 = 0.0;          // this lane's rows (lanes with l == 0)
+    double tot0 = 0.0, tot1 = 0.0;   // rows this lane reports (l == 0: row 0, l == 1: row 1)
 
     const int64_t n_warps = (int64_t)gridDim.x * kClipWarps;
     for (int64_t t = (int64_t)blockIdx.x * kClipWarps + warp; t < p.n_tasks; t += n_warps) {
@@ -172,42 +165,39 @@ clip_kernel(const ClipParams p) {
         if (nan0) m0 = __int_as_float(0x7fc00000);
         if (nan1) m1 = __int_as_float(0x7fc00000);
 
-        float e00 = 0.f, e01 = 0.f, best0 = 0.f, best1 = 0.f;
-        int b0 = 0, b1 = 0;
+        // Each lane pair splits the two rows: even lanes finish row 0's group
+        // scale, error sum and best ratio, odd lanes row 1's.  The error sum
+        // is the same pairwise tree as a butterfly over the row's lanes.
+        const bool odd = (lane & 1) != 0;
+        const int even = lane & ~1;
+        const float m_own = odd ? m1 : m0;
+        float e_first = 0.f, best = 0.f;
+        int b_own = 0;
         for (int i = 0; i < p.n_clip; ++i) {
             const float c = __fdiv_rn((float)(kClipDen - i), (float)kClipDen);
             bool unused;
-            const float qs0 = group_scale(__fmul_rn(m0, c), p.fp32_scale != 0, &unused);
-            const float qs1 = group_scale(__fmul_rn(m1, c), p.fp32_scale != 0, &unused);
-            const float rq0 = qs0 > 0.f ? rcp_approx(qs0) : (qs0 == 0.f ? 0.f : qs0);
-            const float rq1 = qs1 > 0.f ? rcp_approx(qs1) : (qs1 == 0.f ? 0.f : qs1);
-            const float e0 = row_sum<L>(lane_error(ws0, t2, qs0, rq0));
-            const float e1 = row_sum<L>(lane_error(ws1, t2, qs1, rq1));
+            const float qs = group_scale(__fmul_rn(m_own, c), p.fp32_scale != 0, &unused);
+            const float rq = qs > 0.f ? rcp_approx(qs) : (qs == 0.f ? 0.f : qs);
+            const float qs0 = __shfl_sync(0xffffffffu, qs, even);
+            const float qs1 = __shfl_sync(0xffffffffu, qs, even | 1);
+            const float rq0 = __shfl_sync(0xffffffffu, rq, even);
+            const float rq1 = __shfl_sync(0xffffffffu, rq, even | 1);
+            const float ea = lane_error(ws0, t2, qs0, rq0);
+            const float eb = lane_error(ws1, t2, qs1, rq1);
+            float e = (odd ? eb : ea) + __shfl_xor_sync(0xffffffffu, odd ? ea : eb, 1);
+#pragma unroll
+            for (int o = 2; o < L; o <<= 1) e += __shfl_xor_sync(0xffffffffu, e, o);
             if (i == 0) {
-                e00 = best0 = e0;
-                e01 = best1 = e1;
-            } else {
-                if (e0 < best0) {
-                    best0 = e0;
-                    b0 = i;
-                }
-                if (e1 < best1) {
-                    best1 = e1;
-                    b1 = i;
-                }
+                e_first = best = e;
+            } else if (e < best) {
+                best = e;
+                b_own = i;
             }
         }
-        if (l == 0) {
-            if (v0) {
-                p.idx[r0 * p.groups + k] = (uint8_t)b0;
-                tot0 += (double)e00;
-                tot1 += (double)best0;
-            }
-            if (v1) {
-                p.idx[r1 * p.groups + k] = (uint8_t)b1;
-                tot0 += (double)e01;
-                tot1 += (double)best1;
-            }
+        if (l < 2 && (odd ? v1 : v0)) {   // l == 0 reports row 0, l == 1 row 1
+            p.idx[(odd ? r1 : r0) * p.groups + k] = (uint8_t)b_own;
+            tot0 += (double)e_first;
+            tot1 += (double)best;
         }
     }
     pdl_launch_dependents();
