@@ -67,6 +67,18 @@ def test_duo_search_parity(shape):
         assert np.array_equal(sc.cpu().numpy().view(np.uint16), sc_o.view(np.uint16))
 
 
+@pytest.mark.parametrize("n_grid", [1, 32])
+def test_duo_grid_sizes(n_grid):
+    """One grid point (r = 0: the candidate is 1 / (w_mean + 1e-4)) and the
+    largest grid, whose alphas the candidates kernel's warps take in four
+    rounds."""
+    W = wl.weight(96, 512, 41 + n_grid)
+    X = wl.activations(48, 512, 42 + n_grid)
+    s = _duo_case([W], X, 128, n_grid)
+    if n_grid == 1:
+        assert np.all(np.isfinite(s)) and np.all(s > 0)
+
+
 def test_duo_qwen3_gate_up_group():
     """The Qwen3-8B gate/up group (2 x 12288 rows x 4096) with duo scaling."""
     work = wl.WORKLOADS["qwen3_8b_stack36"]
