@@ -61,8 +61,11 @@ FMA_OPS_PER_PAIR = 5
 # dram__bytes_read.sum + dram__bytes_write.sum of one launch of the dominant
 # kernel from the committed ncu captures (profiles/), for the kernels as they
 # stand; None where no capture of the current kernel exists.
-NCU_TRAFFIC = {"q_proj_4096x4096": 34248960,          # search_kernel<8,0,0>
-               "down_proj_output_error": 3105129984}  # oe_gemm_kernel, per alpha
+# DRAM bytes (read + write) of one launch of the dominant kernel, from an ncu
+# capture of the current kernel: (workload, asymmetric grid) -> bytes.
+NCU_TRAFFIC = {("q_proj_4096x4096", False): 34254848,        # search_kernel<8,0,0>
+               ("q_proj_4096x4096", True): 34256384,         # search_kernel<8,0,1>
+               ("down_proj_output_error", False): 3105129984}  # oe_gemm_kernel, per alpha
 FP32_LANES_PER_SM = 128
 DEFAULT_STEPS = {"single_linear_256x512": 1000, "q_proj_4096x4096": 1000,
                  "qwen3_8b_block": 100, "down_proj_output_error": 10,
@@ -395,8 +398,8 @@ def run_ours(a):
                           "GEMM with fused square-sum + finalize)",
                 "achieved": achieved / 1e12, "peak": peak_t / 1e12, "unit": "TFLOP/s",
                 "frac": achieved / peak_t,
-                "traffic": (NCU_TRAFFIC[a.workload] * n_grid
-                            if a.workload in NCU_TRAFFIC else None),
+                "traffic": (NCU_TRAFFIC[(a.workload, False)] * n_grid
+                            if (a.workload, False) in NCU_TRAFFIC else None),
                 "traffic_basis": "DRAM bytes of the n_grid GEMM launches of one call "
                                  "(ncu, per launch x n_grid)",
                 "flops_per_step": flops, "executed_flops_per_step": 2 * flops,
@@ -415,7 +418,7 @@ def run_ours(a):
                 "kernel": "awq_scale_search (table kernel + fused search kernel with finalize)",
                 "achieved": achieved / 1e12, "peak": peak_ops / 1e12, "unit": "Top/s",
                 "frac": achieved / peak_ops,
-                "traffic": NCU_TRAFFIC.get(a.workload),
+                "traffic": NCU_TRAFFIC.get((a.workload, bool(a.asym))),
                 "ops_per_weight_alpha": ALG_OPS_PER_PAIR,
                 "executed_fma_pipe_ops_per_weight_alpha": FMA_OPS_PER_PAIR,
                 "executed_frac": executed / peak_ops,
