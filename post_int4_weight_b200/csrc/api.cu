@@ -107,6 +107,7 @@ awq_status awq_workspace_size(int op, int64_t T, int64_t d_out_total, int64_t d_
 
 awq_status awq_act_stats(const void* X, int64_t T, int64_t d_in, int64_t ld, float* x_mean,
                          void* ws, size_t ws_bytes, void* stream) {
+    const NvtxRange nvtx_range("awq_act_stats");
     if (!X || !x_mean) return AWQ_ERR_INVALID_ARG;
     if (T < 1 || T > (int64_t(1) << 23)) return AWQ_ERR_INVALID_ARG;
     if (d_in < 1 || d_in > (int64_t(1) << 24) || ld < d_in) return AWQ_ERR_INVALID_ARG;
@@ -125,6 +126,7 @@ awq_status awq_scale_search(int n_seg, const void* const* W, const int64_t* d_ou
                             int64_t d_in, const float* x_mean, int group_size, int n_grid,
                             int flags, double* err, int32_t* best_idx, float* s_best,
                             void* ws, size_t ws_bytes, void* stream) {
+    const NvtxRange nvtx_range("awq_scale_search");
     if (n_seg < 1 || n_seg > AWQ_MAX_SEGMENTS || !W || !d_out) return AWQ_ERR_INVALID_ARG;
     if (!x_mean || !err || !best_idx || !s_best) return AWQ_ERR_INVALID_ARG;
     if (!valid_group(group_size)) return AWQ_ERR_UNSUPPORTED;
@@ -152,6 +154,7 @@ awq_status awq_scale_search(int n_seg, const void* const* W, const int64_t* d_ou
 awq_status awq_quantize_pack(const void* W, int64_t d_out, int64_t d_in, const float* s,
                              const uint8_t* clip_idx, int group_size, int zero_point,
                              int32_t* qweight, void* scales, int32_t* qzeros, void* stream) {
+    const NvtxRange nvtx_range("awq_quantize_pack");
     if (!W || !qweight || !scales || !qzeros) return AWQ_ERR_INVALID_ARG;
     if (!valid_group(group_size)) return AWQ_ERR_UNSUPPORTED;
     if (zero_point != 7 && zero_point != 8 && zero_point != AWQ_ZERO_POINT_ASYM)
@@ -173,6 +176,7 @@ awq_status awq_quantize_pack(const void* W, int64_t d_out, int64_t d_in, const f
 
 awq_status awq_norm_group_scale(int n, const float* const* s, int64_t d_in, float* s_shared,
                                void* stream) {
+    const NvtxRange nvtx_range("awq_norm_group_scale");
     if (n < 1 || n > AWQ_MAX_SEGMENTS || !s || !s_shared) return AWQ_ERR_INVALID_ARG;
     if (d_in < 1 || d_in > (int64_t(1) << 24)) return AWQ_ERR_INVALID_ARG;
     for (int m = 0; m < n; ++m) {
@@ -193,6 +197,7 @@ awq_status awq_clip_search(const void* W, int64_t d_out, int64_t d_in, const flo
                            const float* s, int group_size, int n_clip, int flags,
                            uint8_t* clip_idx, double* err, void* ws, size_t ws_bytes,
                            void* stream) {
+    const NvtxRange nvtx_range("awq_clip_search");
     if (!W || !x_mean || !clip_idx || !err) return AWQ_ERR_INVALID_ARG;
     if (!valid_group(group_size)) return AWQ_ERR_UNSUPPORTED;
     if (n_clip < 1 || n_clip > AWQ_CLIP_MAX) return AWQ_ERR_INVALID_ARG;
@@ -215,6 +220,7 @@ awq_status awq_output_error(const void* X, int64_t T, const void* W, int64_t d_o
                             int64_t d_in, const float* x_mean, int group_size, int n_grid,
                             int flags, double* err, int32_t* best_idx, float* s_best,
                             void* ws, size_t ws_bytes, void* stream) {
+    const NvtxRange nvtx_range("awq_output_error");
     if (!X || !W || !x_mean || !err || !best_idx) return AWQ_ERR_INVALID_ARG;
     if (!valid_group(group_size)) return AWQ_ERR_UNSUPPORTED;
     if (n_grid < 1 || n_grid > 32) return AWQ_ERR_INVALID_ARG;

@@ -9,8 +9,20 @@
 #include <utility>
 
 #include "awq.h"
+#include <nvtx3/nvToolsExt.h>
 
 namespace awq {
+
+// A named NVTX range spanning one entry-point call, so that a timeline
+// profiler shows each call (and the kernels it enqueued) under its name.
+// Without a profiler attached a push or pop costs a pointer check.
+struct NvtxRange {
+    explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange&) = delete;
+    NvtxRange& operator=(const NvtxRange&) = delete;
+};
+
 
 constexpr size_t kWsAlign = 256;
 
