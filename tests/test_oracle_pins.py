@@ -538,6 +538,28 @@ def test_weight_mean_row_scaling_invariance():
     assert np.array_equal(oracle.weight_mean([W]), oracle.weight_mean([W2]))
 
 
+def test_weight_mean_nonfinite_weights():
+    """IEEE rules fix what a NaN or an infinity does: the row maximum skips a
+    NaN (|w| >= 0, so it acts as a 0 there) and the NaN's own quotient is
+    NaN; an infinite maximum makes every finite quotient of its row 0 and
+    its own quotient inf / inf = NaN."""
+    rng = np.random.default_rng(73)
+    W = (rng.standard_normal((16, 64)) * 0.02).astype(np.float16)
+    Wn = W.copy()
+    Wn[3, 5] = np.nan
+    Wz = W.copy()
+    Wz[3, 5] = 0
+    got, ref = oracle.weight_mean([Wn]), oracle.weight_mean([Wz])
+    assert np.isnan(got[5]) and np.array_equal(np.delete(got, 5), np.delete(ref, 5))
+    Wi = W.copy()
+    Wi[7, 9] = np.inf
+    Wr = np.delete(W, 7, axis=0)            # the inf row adds 0 to the finite channels
+    got = oracle.weight_mean([Wi])
+    ref = oracle.weight_mean([Wr]) * 15 / 16
+    assert np.isnan(got[9])
+    assert np.allclose(np.delete(got, 9), np.delete(ref, 9), rtol=1e-15, atol=0)
+
+
 def test_duo_table_r0_closed_form_and_constant_weights():
     x = np.array([0.5, 2.0, 8.0, 1e-6], np.float32)
     wm = np.array([1, 0.75, 0.375, 0.625])
