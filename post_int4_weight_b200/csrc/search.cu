@@ -457,13 +457,32 @@ search_kernel(const __grid_constant__ SearchParams p) {
         decode(u, &seg, &grp, &rb);
         if (grp != cur_grp) {   // uniform: every thread walks the same units
             __syncthreads();
-            const float* Sg = p.S + (int64_t)grp * G;
-            const float* Tg = p.tau2 + (int64_t)grp * G;
-            for (int i = tid; i < p.n_grid * G; i += kThreads) {
-                const int a = i / G, c = i % G;
-                const int slot = table_slot<L>(c);
-                tab[a * 2 * G + slot] = __ldcg(Sg + (int64_t)a * p.d_in + c);
-                tab[a * 2 * G + G + slot] = __ldcg(Tg + (int64_t)a * p.d_in + c);
+            // The group's S and tau2 columns, 16 bytes at a time (rows are
+            // 16-byte aligned: d_in % 32 == 0; table_slot keeps each run of
+            // four channels together), every load issued before any store.
+            constexpr int kC4 = G / 4;                                   // float4 per row
+            constexpr int kPer = (kMaxGrid * kC4 + kThreads - 1) / kThreads;
+            const float4* Sg = reinterpret_cast<const float4*>(p.S + (int64_t)grp * G);
+            const float4* Tg = reinterpret_cast<const float4*>(p.tau2 + (int64_t)grp * G);
+            const int64_t ld4 = p.d_in / 4;
+            const int n4 = p.n_grid * kC4;
+            float4 sv[kPer], tv[kPer];
+#pragma unroll
+            for (int k = 0; k < kPer; ++k) {
+                const int i = tid + k * kThreads;
+                if (i < n4) {
+                    sv[k] = __ldcg(Sg + (int64_t)(i / kC4) * ld4 + i % kC4);
+                    tv[k] = __ldcg(Tg + (int64_t)(i / kC4) * ld4 + i % kC4);
+                }
+            }
+#pragma unroll
+            for (int k = 0; k < kPer; ++k) {
+                const int i = tid + k * kThreads;
+                if (i < n4) {
+                    const int a = i / kC4, slot = table_slot<L>(4 * (i % kC4));
+                    *reinterpret_cast<float4*>(&tab[a * 2 * G + slot]) = sv[k];
+                    *reinterpret_cast<float4*>(&tab[a * 2 * G + G + slot]) = tv[k];
+                }
             }
             for (int i = tid; i < 2 * G; i += kThreads) tab[p.n_grid * 2 * G + i] = 0.f;
             cur_grp = grp;
