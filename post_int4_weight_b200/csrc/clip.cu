@@ -202,7 +202,8 @@ clip_kernel(const ClipParams p) {
     }
     pdl_launch_dependents();
 
-    // fixed-order reduction: warp tree, then warps in order, then CTAs in order
+    // fixed-order reduction: warp tree, then warps in order, then (last CTA)
+    // the CTAs' partials in a fixed order
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
         tot0 += __shfl_xor_sync(0xffffffffu, tot0, o);
@@ -225,11 +226,37 @@ clip_kernel(const ClipParams p) {
         last = (atomicAdd(p.counter, 1) == (int)gridDim.x - 1);
     }
     __syncthreads();
-    if (last && threadIdx.x < 2) {
+    if (last && warp == 0) {
         __threadfence();
-        double a = 0.0;
-        for (int c = 0; c < (int)gridDim.x; ++c) a += __ldcg(p.partial + 2 * c + threadIdx.x);
-        p.err[threadIdx.x] = a;
+        // lane k adds the CTAs k, k + 32, k + 64, ... in that order (every
+        // load of a batch in flight before its adds), then a fixed shuffle
+        // tree: the same order on every run
+        constexpr int kB = 8;
+        const int n = (int)gridDim.x;
+        double a = 0.0, b = 0.0;
+        for (int c0 = 0; c0 < n; c0 += 32 * kB) {
+            double va[kB], vb[kB];
+#pragma unroll
+            for (int k = 0; k < kB; ++k) {
+                const int c = c0 + lane + 32 * k;
+                va[k] = c < n ? __ldcg(p.partial + 2 * c) : 0.0;
+                vb[k] = c < n ? __ldcg(p.partial + 2 * c + 1) : 0.0;
+            }
+#pragma unroll
+            for (int k = 0; k < kB; ++k) {
+                a += va[k];
+                b += vb[k];
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            a += __shfl_xor_sync(0xffffffffu, a, o);
+            b += __shfl_xor_sync(0xffffffffu, b, o);
+        }
+        if (lane == 0) {
+            p.err[0] = a;
+            p.err[1] = b;
+        }
     }
 }
 
