@@ -189,9 +189,11 @@ awq_status awq_scale_search(int n_seg, const void *const *W,
  * The scratch is one static device array of AWQ_NOALLOC_SCRATCH_BYTES inside
  * the library; every GPU that uses the library keeps it until the process
  * exits.  Calls whose workspace need (awq_workspace_size with
- * AWQ_OP_SCALE_SEARCH) exceeds it return AWQ_ERR_WORKSPACE with nothing
+ * AWQ_OP_SCALE_SEARCH, or AWQ_OP_SCALE_SEARCH_DUO when flags hold
+ * AWQ_DUO_SCALING) exceeds it return AWQ_ERR_WORKSPACE with nothing
  * enqueued -- e.g. d_in = 16384 fits with n_grid <= 29, d_in = 12288 with
- * n_grid <= 32.  The first call on a device looks the array's address up
+ * n_grid <= 32; duo scaling needs d_in * 8 bytes per weight-mean CTA on top
+ * and so fits only small d_in (d_in <= 2048 at 20 grid points).  The first call on a device looks the array's address up
  * (cudaGetSymbolAddress, that device current) and caches it: make it before
  * any stream capture on that device.  All calls on a device share the array;
  * each call rewrites every scratch byte it reads, but calls that overlap on
