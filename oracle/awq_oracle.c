@@ -18,7 +18,10 @@
  *        scale and a 4-bit zero point per group and output channel) and
  *        "The scale search as code" (the worked example: values up to 0.5
  *        in magnitude give a step of about 1/15 and a worst rounding error
- *        of about 0.033); the formula is a reading listed in the design doc.
+ *        of about 0.033).  The pages give no formula; the reading here is the
+ *        min-max grid: range = max(max ws - min ws, 1e-5), q_scale =
+ *        fp16(range / 15), zero = clamp(rint(-min ws / q_scale), 0, 15),
+ *        q = clamp(rint(ws / q_scale) + zero, 0, 15) (orc_fake_quant_group_asym).
  *   Duo scaling: [P3] "The scale search as code" (with duo scaling the
  *        candidate is also divided by the mean normalised weight magnitude
  *        raised to 1 - r).
@@ -28,10 +31,12 @@
  *   Clip search: [P3] "The pipeline end to end", step 5 (an optional search
  *        of a clipping range per output channel that shrinks the
  *        quantisation range); [P5] "AWQ, Reproduced" (the paper also clips
- *        the weight range).  The pages give no formula; the reading used
- *        here is listed in the design doc.
+ *        the weight range).  The pages give no formula; the reading here:
+ *        ratios c_i = RN((20 - i) / 20), the group's largest |ws| scaled by
+ *        c_i before the fp16 scale is formed, the same weighted error, and
+ *        the first minimum per (row, group) (orc_clip_search).
  *
- * Precision (readings are listed in the design doc):
+ * Precision (readings of the pages where they leave it open):
  *   - every decision that produces an integer (a code, the group scale, the
  *     chosen grid index) is taken in fp32 with IEEE round-to-nearest-even,
  *     the group scale then rounded to fp16 (round-to-nearest-even);
