@@ -109,7 +109,7 @@ def test_act_stats_nonfinite_and_extremes():
 
 SEARCH_CASES = [
     # (name, [d_out per segment], d_in, T, g, n_grid, flags)
-    ("config1_256x512_g128", [256], 512, 64, 128, 20, 0),
+    ("single_linear_256x512_g128", [256], 512, 64, 128, 20, 0),
     ("g64", [256], 512, 64, 64, 20, 0),
     ("g32", [128], 256, 48, 32, 20, 0),
     ("ragged_rows_200", [200], 384, 32, 128, 20, 0),
