@@ -152,3 +152,24 @@ def test_pipeline_workspace_sizes_from_host_query():
     assert jc.launches == 1 + 2 + 2 + 2
     ws = pipeline.Workspaces([j, jo, jc], "cpu")
     assert ws.search.numel() == max(se, se_o)
+
+
+def test_duo_workspace_growth_and_noalloc_limit():
+    """The duo workspace adds, to the plain search's, one fp64 column-sum row
+    per weight-mean CTA, the fp64 candidates of every grid point and their
+    per-block extremes; it grows with d_in and n_grid.  The no-alloc entry's
+    4 MiB scratch holds the duo search up to d_in 2048 at 20 grid points
+    (the limit include/awq.h states) and not at 4096."""
+    def duo(d_in, n_grid):
+        return awq.workspace_size(awq.OP_SCALE_SEARCH_DUO, 1, 8, d_in, 128, n_grid)
+
+    def plain(d_in, n_grid):
+        return awq.workspace_size(awq.OP_SCALE_SEARCH, 1, 8, d_in, 128, n_grid)
+
+    for d_in in (512, 2048, 4096, 16384):
+        extra = duo(d_in, 20) - plain(d_in, 20)
+        assert extra >= 148 * d_in * 8 + 20 * d_in * 8
+        assert duo(d_in, 32) > duo(d_in, 20)
+    assert duo(2048, 20) <= 4 << 20 < duo(4096, 20)
+    with pytest.raises(awq.AwqError):
+        duo(16384 + 128, 20)                    # beyond the weight-mean pass's 16384
