@@ -9,7 +9,9 @@ import subprocess
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 SRC = os.path.join(HERE, "awq_oracle.c")
-LIB = os.path.join(HERE, "liborc.so")
+# AWQ_ORACLE_LIB: a separately built copy to load instead (the sanitizer
+# test builds one with -fsanitize=... and points the pins at it)
+LIB = os.environ.get("AWQ_ORACLE_LIB") or os.path.join(HERE, "liborc.so")
 
 
 def build(force: bool = False) -> str:
