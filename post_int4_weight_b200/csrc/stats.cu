@@ -14,8 +14,9 @@
 //     an integer multiple of 2^-24 below 2^28: exact in fp64.  Every 4096
 //     rows the fp64 sums are moved, exactly, into 64-bit integer counts of
 //     2^-24;
-//   * the integer sums are added across the warp's row lanes with shuffles,
-//     then meet in shared memory, then in CTA 0 of the cluster
+//   * the integer sums are added across the warp's row lanes with shuffles
+//     into the warp's own shared slots, the warps' slots are added in warp
+//     order, and the CTAs' sums meet in CTA 0 of the cluster
 //     through distributed shared memory atomics; integer addition makes the
 //     result independent of order.  CTA 0 writes x[j] = (sum * 2^-24) / T
 //     (fp64 division, rounded to fp32).
@@ -65,15 +66,24 @@ __device__ __forceinline__ void add_halves(const uint4& v, double* acc, uint32_t
 // Moves the exact fp64 partial sums into integer counts of 2^-24 (or flag
 // bits for a column that held a non-finite value: bit 0 infinity, bit 1
 // NaN, from the largest |h| bit patterns seen), adds them over the warp's
-// row lanes (lanes with the same chunk) and into the CTA's shared
-// accumulators, and clears them.  Called by every lane of a warp together.
+// row lanes (lanes with the same chunk) and into the warp's own shared
+// slots (lanes 0..7 own disjoint entries: no atomics), and clears them.
+// Called by every lane of a warp together.  A thread's sum covers at most
+// kFlushRows rows of values of at most 65504 (the main loop flushes once it
+// reaches kFlushRows; at most kBatch tail rows follow its last flush and
+// leave it at most kFlushRows), so sum * 2^24 is an integer below
+// 4096 * 65504 * 2^24 < 2^52 (plus the zeros' 2^-127 terms, far below 1/2):
+// adding 2^52 rounds it to that integer exactly and leaves it in the low 52
+// bits.
 __device__ __forceinline__ void flush(double* acc, const uint32_t* hmax, int cx,
-                                      unsigned long long* red, uint32_t* fred) {
+                                      unsigned long long* wred, uint32_t* wfred) {
     const int lane = threadIdx.x & 31;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
         const uint32_t hm = (hmax[i >> 1] >> (16 * (i & 1))) & 0xffffu;
-        unsigned long long u = __double2ull_rn(acc[i] * 0x1p24);
+        unsigned long long u =
+            (unsigned long long)__double_as_longlong(__fma_rn(acc[i], 0x1p24, 0x1p52)) -
+            0x4330000000000000ull;
         uint32_t f = 0;
         if (hm > 0x7c00u) {
             f = 2u;
@@ -88,8 +98,8 @@ __device__ __forceinline__ void flush(double* acc, const uint32_t* hmax, int cx,
             f |= __shfl_xor_sync(0xffffffffu, f, o);
         }
         if (lane < kChunks) {
-            if (u) atomicAdd(&red[cx * 8 + i], u);
-            if (f) atomicOr(&fred[cx * 8 + i], f);
+            wred[cx * 8 + i] += u;
+            wfred[cx * 8 + i] |= f;
         }
         acc[i] = 0.0;
     }
@@ -98,8 +108,11 @@ __device__ __forceinline__ void flush(double* acc, const uint32_t* hmax, int cx,
 __global__ void __cluster_dims__(1, kCluster, 1) __launch_bounds__(kChunks * kRowLanes, 4)
 stats_kernel(const uint4* __restrict__ X, int64_t T, int64_t d_in, int64_t ld_chunks,
              float* __restrict__ x_mean) {
+    constexpr int kWarps = kChunks * kRowLanes / 32;
     __shared__ unsigned long long red[kChunks * 8];
     __shared__ uint32_t fred[kChunks * 8];
+    __shared__ unsigned long long red_w[kWarps][kChunks * 8];   // per-warp sums
+    __shared__ uint32_t fred_w[kWarps][kChunks * 8];
     cg::cluster_group cluster = cg::this_cluster();
     const int rank = (int)cluster.block_rank();
 
@@ -111,6 +124,14 @@ stats_kernel(const uint4* __restrict__ X, int64_t T, int64_t d_in, int64_t ld_ch
     if (tid < kChunks * 8) {
         red[tid] = 0;
         fred[tid] = 0;
+    }
+    {   // each warp clears its own slots (only it writes them, in flush)
+        const int w = tid >> 5, l = tid & 31;
+        for (int i = l; i < kChunks * 8; i += 32) {
+            red_w[w][i] = 0;
+            fred_w[w][i] = 0;
+        }
+        __syncwarp();
     }
     // every CTA's accumulators must be cleared before other CTAs add into
     // them: arrive now, wait just before the remote adds (after the loads)
@@ -156,7 +177,7 @@ stats_kernel(const uint4* __restrict__ X, int64_t T, int64_t d_in, int64_t ld_ch
         for (int k = 0; k < kBatch; ++k) add_halves(cur[k], acc, hmax);
         since_flush += kBatch;
         if (since_flush >= kFlushRows) {
-            flush(acc, hmax, cx, red, fred);
+            flush(acc, hmax, cx, red_w[tid >> 5], fred_w[tid >> 5]);
             since_flush = 0;
         }
         base = nb;
@@ -167,7 +188,20 @@ stats_kernel(const uint4* __restrict__ X, int64_t T, int64_t d_in, int64_t ld_ch
     for (int64_t r = base + sub; r < r1; r += kRowLanes)
         if (active) add_halves(__ldg(p + r * ld_chunks), acc, hmax);
     pdl_launch_dependents();   // X is read; the next kernel may start launching
-    flush(acc, hmax, cx, red, fred);
+    flush(acc, hmax, cx, red_w[tid >> 5], fred_w[tid >> 5]);
+    __syncthreads();
+    if (tid < kChunks * 8) {   // the warps' sums, in warp order (integers: exact)
+        unsigned long long s = 0;
+        uint32_t f = 0;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) {
+            s += red_w[w][tid];
+            f |= fred_w[w][tid];
+        }
+        // other CTAs of the cluster may already be adding into rank 0's red
+        if (s) atomicAdd(&red[tid], s);
+        if (f) atomicOr(&fred[tid], f);
+    }
     __syncthreads();
     cluster.barrier_wait();
     if (rank != 0 && tid < kChunks * 8) {

@@ -81,9 +81,11 @@ def test_act_stats_bit_exact(T, d_in):
 
 
 def test_act_stats_long_token_slices():
-    """More than 4096 rows per thread: the exact fp64 partial sums are moved
-    into the integer accumulators mid-way (rows of 16 lanes x 8 CTAs)."""
-    X = wl.activations(600_011, 16, seed=77)
+    """More than 4096 rows per thread (32 row lanes x 8 CTAs of a cluster:
+    T > 8 * 32 * 4096): the exact fp64 partial sums are moved into the
+    integer accumulators mid-way, and a column of 65504 drives a thread's
+    count to the largest value the conversion allows (4096 x 65504 x 2^24)."""
+    X = wl.activations(1_310_731, 16, seed=77)
     X[:, 3] = 65504.0                      # the largest sums the format allows
     x = awq.act_stats(X.cuda())
     torch.cuda.synchronize()
