@@ -19,8 +19,8 @@ k/v 1024x4096, gate/up 12288x4096, down 4096x12288) that the pages quantise
 from __future__ import annotations
 
 import math
-from dataclasses import dataclass, field
-from typing import List, Tuple
+from dataclasses import dataclass
+from typing import Tuple
 
 import torch
 

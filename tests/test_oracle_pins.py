@@ -5,7 +5,6 @@ example printed on a page, a closed form, a special case that reduces to a
 textbook routine, an invariant, or brute force on tiny inputs.  No expected
 value here comes from the CUDA path.
 """
-import itertools
 import math
 
 import numpy as np
