@@ -1,0 +1,132 @@
+"""Property pins of the oracle over generated inputs (hypothesis).
+
+Each property follows from the definitions or from plain mathematics, not
+from the oracle's own formulas: a code is the nearest of the grid's levels
+(found by trying every level), the rounding error of an unclamped weight is
+at most half a step, the activation mean equals the exact rational mean
+(Python integers and fractions), negating or doubling the weights acts on
+the results as the definitions say, and the searched error never exceeds
+plain round-to-nearest.  The generators reach fp16 subnormals, zeros, exact
+half-step ties and the largest fp16 magnitudes.  Runs are derandomised, so
+every run checks the same examples.
+"""
+from fractions import Fraction
+
+import numpy as np
+import pytest
+from hypothesis import HealthCheck, given, settings
+from hypothesis import strategies as st
+from hypothesis.extra import numpy as hnp
+
+import oracle
+
+SETTINGS = settings(max_examples=80, deadline=None, derandomize=True,
+                    suppress_health_check=[HealthCheck.too_slow])
+
+f16 = st.floats(width=16, allow_nan=False, allow_infinity=False)
+# finite fp16 weights of moderate size (so that w * s stays far from overflow)
+f16_w = st.floats(min_value=-8.0, max_value=8.0, width=16, allow_nan=False)
+scale = st.floats(min_value=2.0 ** -6, max_value=2.0 ** 6, width=32, allow_nan=False)
+
+
+def _group(n):
+    return hnp.arrays(np.float16, n, elements=f16_w)
+
+
+def _scales(n):
+    return hnp.arrays(np.float32, n, elements=scale)
+
+
+def _nearest_level(v, qs, lo, hi, shift=0):
+    """The level q in lo..hi nearest to v / qs by trying every one (ties: the
+    even value of q - shift, as round-half-to-even of v / qs gives)."""
+    best, best_d = None, None
+    for q in range(lo, hi + 1):
+        d = abs(Fraction(float(v)) - (q - shift) * Fraction(float(qs)))
+        if best is None or d < best_d or (d == best_d and (q - shift) % 2 == 0):
+            best, best_d = q, d
+    return best
+
+
+@SETTINGS
+@given(st.sampled_from([8, 32, 128]).flatmap(lambda n: st.tuples(_group(n), _scales(n))),
+       st.booleans())
+def test_symmetric_codes_are_nearest_levels(ws_pair, fp32_scale):
+    w, s = ws_pair
+    flags = oracle.SCALE_FP32 if fp32_scale else 0
+    q, qs, bad = oracle.fake_quant_group(w, s, flags)
+    assert not bad
+    assert np.all((q >= -7) & (q <= 7))
+    prod = w.astype(np.float32) * s            # fp32 products (IEEE, one rounding)
+    if qs == 0.0:
+        assert np.all(q == 0) and np.all(prod == 0)
+        return
+    for v, c in zip(prod, q):
+        assert c == _nearest_level(v, qs, -7, 7)
+        if abs(Fraction(float(v))) <= Fraction(15, 2) * Fraction(qs):
+            assert abs(Fraction(float(v)) - c * Fraction(qs)) <= Fraction(qs) / 2
+
+
+@SETTINGS
+@given(st.sampled_from([8, 32]).flatmap(lambda n: st.tuples(_group(n), _scales(n))))
+def test_symmetric_sign_and_power_of_two_scaling(ws_pair):
+    """Negating w negates every code (ties go to even either way); doubling
+    w (exact in fp16 below 8 * 2) doubles the fp32 group scale exactly and
+    keeps the codes."""
+    w, s = ws_pair
+    q, qs, _ = oracle.fake_quant_group(w, s, oracle.SCALE_FP32)
+    qn, qsn, _ = oracle.fake_quant_group(-w, s, oracle.SCALE_FP32)
+    assert qsn == qs and np.array_equal(qn, -q)
+    q2, qs2, _ = oracle.fake_quant_group((w.astype(np.float32) * 2).astype(np.float16), s,
+                                         oracle.SCALE_FP32)
+    if qs > 2.0 ** -100:                     # far from the fp32 subnormal range
+        assert qs2 == 2 * qs and np.array_equal(q2, q)
+
+
+@SETTINGS
+@given(st.sampled_from([8, 32, 128]).flatmap(lambda n: st.tuples(_group(n), _scales(n))))
+def test_asymmetric_codes_are_nearest_shifted_levels(ws_pair):
+    w, s = ws_pair
+    q, qs, z = oracle.fake_quant_group_asym(w, s)
+    assert 0 <= z <= 15 and np.all(q <= 15)
+    prod = w.astype(np.float32) * s
+    for v, c in zip(prod, q):
+        assert c == _nearest_level(v, qs, 0, 15, shift=z)
+
+
+@SETTINGS
+@given(hnp.arrays(np.float16, st.tuples(st.integers(1, 40), st.sampled_from([8, 16])),
+                  elements=f16))
+def test_act_stats_is_the_exact_mean(X):
+    """mean_t |X[t, j]| exactly (every |fp16| is an integer multiple of
+    2^-24), rounded once to fp64 and then to fp32, for any token order."""
+    x = oracle.act_stats(X)
+    T = X.shape[0]
+    for j in range(X.shape[1]):
+        exact = sum(Fraction(abs(float(v))) for v in X[:, j]) / T
+        assert x[j] == np.float32(float(exact))
+    perm = np.random.default_rng(T).permutation(T)
+    assert np.array_equal(oracle.act_stats(X[perm]), x)
+
+
+@SETTINGS
+@given(st.integers(1, 4).flatmap(lambda r: hnp.arrays(
+           np.float16, (8 * r, 64), elements=f16_w)),
+       hnp.arrays(np.float32, 64, elements=st.floats(min_value=0.0, max_value=100.0,
+                                                      width=32)),
+       st.sampled_from([1, 5, 20]))
+def test_search_never_worse_than_round_to_nearest(W, x, n_grid):
+    """Grid point 0 is s = 1 (plain round-to-nearest); the chosen error is
+    the first minimum and never above it."""
+    err, best, s = oracle.scale_search([W], x, 32, n_grid)
+    assert np.all(np.isfinite(err))
+    assert best == int(np.argmin(err)) and err[best] <= err[0]
+    if n_grid == 1:
+        assert best == 0 and np.all(s == 1.0)
+
+
+@pytest.mark.parametrize("n", [1, 2, 3])
+def test_geomean_of_equal_members_is_the_member(n):
+    rng = np.random.default_rng(n)
+    s = (rng.random(64) * 10 + 1e-3).astype(np.float32)
+    assert np.array_equal(oracle.geomean_scales([s] * n), s)
