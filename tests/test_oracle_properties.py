@@ -130,3 +130,53 @@ def test_geomean_of_equal_members_is_the_member(n):
     rng = np.random.default_rng(n)
     s = (rng.random(64) * 10 + 1e-3).astype(np.float32)
     assert np.array_equal(oracle.geomean_scales([s] * n), s)
+
+
+@SETTINGS
+@given(st.integers(1, 3).flatmap(
+           lambda r: hnp.arrays(np.float16, (8 * r, 64), elements=f16_w)),
+       hnp.arrays(np.float32, 64, elements=scale), st.sampled_from([7, 8]))
+def test_pack_round_trip_and_dequant(W, s, zp):
+    """Unpacked codes minus the zero point, times the stored fp16 scale, give
+    exactly the group fake-quant's q * q_scale; qzeros holds the zero point
+    in every nibble."""
+    g = 32
+    qw, sc, qz = oracle.quantize_pack(W, s, g, zp)
+    u = oracle.unpack(qw, W.shape[0]).astype(np.int64)
+    assert np.all(qz == np.int32(np.uint32(zp * 0x11111111).view(np.int32)))
+    for r in range(W.shape[0]):
+        for k in range(W.shape[1] // g):
+            q, qs, _ = oracle.fake_quant_group(W[r, k * g:(k + 1) * g], s[k * g:(k + 1) * g])
+            assert np.array_equal(u[r, k * g:(k + 1) * g] - zp, q)
+            assert float(sc[k, r]) == qs
+
+
+@SETTINGS
+@given(st.sampled_from([8, 32]).flatmap(lambda n: st.tuples(_group(n), _scales(n))),
+       st.integers(0, 19))
+def test_clipped_codes_are_nearest_levels(ws_pair, i):
+    """With the range shrunk to c_i * max|ws|, every code is still the nearest
+    of the 15 levels of the clipped scale; ratio 0 is the plain quantiser."""
+    w, s = ws_pair
+    c = oracle.clip_ratio(i)
+    q, qs = oracle.fake_quant_group_clip(w, s, c)
+    prod = w.astype(np.float32) * s
+    assert np.all((q >= -7) & (q <= 7))
+    if qs > 0:
+        for v, code in zip(prod, q):
+            assert code == _nearest_level(v, qs, -7, 7)
+    if i == 0:
+        q0, qs0, _ = oracle.fake_quant_group(w, s)
+        assert qs == qs0 and np.array_equal(q, q0)
+
+
+@SETTINGS
+@given(st.integers(1, 6).flatmap(lambda r: hnp.arrays(np.float16, (r, 16), elements=f16_w)))
+def test_weight_mean_bounds(W):
+    """|w| / max|w| of a row lies in [0, 1], so the mean does too; a channel
+    holding every row's largest magnitude has mean exactly 1."""
+    wm = oracle.weight_mean([W])
+    assert np.all((wm >= 0) & (wm <= 1))
+    W2 = W.copy()
+    W2[:, 0] = np.float16(16.0)              # above every other |w| (all <= 8)
+    assert oracle.weight_mean([W2])[0] == 1.0
