@@ -180,3 +180,35 @@ def test_weight_mean_bounds(W):
     W2 = W.copy()
     W2[:, 0] = np.float16(16.0)              # above every other |w| (all <= 8)
     assert oracle.weight_mean([W2])[0] == 1.0
+
+
+pos_x = st.floats(min_value=0.0, max_value=1e4, width=32, allow_nan=False)
+
+
+@SETTINGS
+@given(hnp.arrays(np.float32, st.integers(2, 40), elements=pos_x), st.sampled_from([1, 7, 20]))
+def test_scale_table_rows(x, n_grid):
+    """Row 0 is exactly 1; every row is monotone in x (pow is, and one
+    rounding keeps the order), which is what lets the GPU take the row's
+    extremes from the extreme x; after the normalisation the row's largest
+    times its smallest entry is 1 up to the two fp32 roundings."""
+    S = oracle.scale_table(x, n_grid)
+    assert np.all(S[0] == 1.0)
+    order = np.argsort(x, kind="stable")
+    for i in range(n_grid):
+        row = S[i][order].astype(np.float64)
+        assert np.all(np.diff(row) >= 0)
+        assert abs(row.max() * row.min() - 1.0) <= 2.0 ** -22
+
+
+@SETTINGS
+@given(hnp.arrays(np.float32, 32, elements=pos_x),
+       hnp.arrays(np.float64, 32, elements=st.floats(min_value=0.0, max_value=1.0)),
+       st.sampled_from([1, 20]))
+def test_duo_table_normalisation(x, wm, n_grid):
+    """Every duo row is positive and normalised: largest times smallest entry
+    is 1 up to the two fp32 roundings."""
+    S = oracle.scale_table_duo(x, wm, n_grid).astype(np.float64)
+    assert np.all(S > 0)
+    for i in range(n_grid):
+        assert abs(S[i].max() * S[i].min() - 1.0) <= 2.0 ** -22
