@@ -212,3 +212,42 @@ def test_duo_table_normalisation(x, wm, n_grid):
     assert np.all(S > 0)
     for i in range(n_grid):
         assert abs(S[i].max() * S[i].min() - 1.0) <= 2.0 ** -22
+
+
+@settings(max_examples=25, deadline=None, derandomize=True,
+          suppress_health_check=[HealthCheck.too_slow])
+@given(st.integers(1, 12).flatmap(lambda T: hnp.arrays(np.float16, (T, 64), elements=f16_w)),
+       st.integers(1, 2).flatmap(lambda r: hnp.arrays(np.float16, (8 * r, 64), elements=f16_w)))
+def test_output_error_nonnegative_and_quadratic_in_x(X, W):
+    """||X (W - W_hat)^T||^2 is a sum of squares; with the same x (so the
+    same scale table and W_hat), doubling X (exact in fp16 here) scales every
+    product and partial sum by a power of two, so the error becomes exactly
+    four times larger.  (Recomputing x from 2X would not do: the clamp at
+    1e-4 and pow's rounding do not commute with the doubling.)"""
+    x = oracle.act_stats(X)
+    err = oracle.output_error(X, W, x, 32, 5)
+    assert np.all(err >= 0)
+    X2 = (X.astype(np.float32) * 2).astype(np.float16)
+    err2 = oracle.output_error(X2, W, x, 32, 5)
+    assert np.array_equal(err2, 4 * err)
+
+
+def _f32_neighbours(r):
+    r = np.float32(r)
+    return np.nextafter(r, np.float32(-np.inf)), np.nextafter(r, np.float32(np.inf))
+
+
+@SETTINGS
+@given(hnp.arrays(np.float32, 2, elements=st.floats(min_value=2.0 ** -20, max_value=2.0 ** 20,
+                                                     width=32)))
+def test_geomean_of_two_is_the_rounded_square_root(ab):
+    """For two members the shared scale is sqrt(a b) rounded once to fp32:
+    r is the fp32 value whose neighbours' midpoints bracket sqrt(a b),
+    decided exactly by comparing squares of rationals."""
+    a, b = ab
+    r = oracle.geomean_scales([np.array([a], np.float32), np.array([b], np.float32)])[0]
+    P = Fraction(float(a)) * Fraction(float(b))
+    lo, hi = _f32_neighbours(r)
+    m_lo = (Fraction(float(lo)) + Fraction(float(r))) / 2
+    m_hi = (Fraction(float(r)) + Fraction(float(hi))) / 2
+    assert m_lo * m_lo <= P <= m_hi * m_hi
