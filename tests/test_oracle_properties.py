@@ -251,3 +251,36 @@ def test_geomean_of_two_is_the_rounded_square_root(ab):
     m_lo = (Fraction(float(lo)) + Fraction(float(r))) / 2
     m_hi = (Fraction(float(r)) + Fraction(float(hi))) / 2
     assert m_lo * m_lo <= P <= m_hi * m_hi
+
+
+@SETTINGS
+@given(st.sampled_from([8, 32]).flatmap(lambda n: st.tuples(_group(n), _scales(n),
+                                                            st.integers(0, n - 1))),
+       st.sampled_from([np.nan, np.inf, -np.inf]))
+def test_nonfinite_weight_flags_the_group(wsk, bad_value):
+    w, s, k = wsk
+    w = w.copy()
+    w[k] = bad_value
+    assert oracle.fake_quant_group(w, s)[2]
+
+
+@SETTINGS
+@given(hnp.arrays(np.float16, st.tuples(st.integers(2, 30), st.just(8)), elements=f16_w),
+       st.data())
+def test_act_stats_nonfinite_columns(X, data):
+    """A column holding an infinity has mean inf, one holding a NaN has mean
+    NaN (NaN wins over inf), wherever they sit; other columns are unaffected."""
+    X = X.copy()
+    T = X.shape[0]
+    ti = data.draw(st.integers(0, T - 1))
+    tn = data.draw(st.integers(0, T - 1))
+    ref = oracle.act_stats(X)
+    X[ti, 2] = np.inf
+    X[ti, 5] = -np.inf
+    X[tn, 5] = np.nan if tn != ti else X[tn, 5]
+    X[tn, 6] = np.nan
+    x = oracle.act_stats(X)
+    assert x[2] == np.inf and np.isnan(x[6])
+    assert (np.isnan(x[5]) if tn != ti else x[5] == np.inf)
+    keep = [0, 1, 3, 4, 7]
+    assert np.array_equal(x[keep], ref[keep])
