@@ -28,7 +28,9 @@
  *     A launch failure returns AWQ_ERR_CUDA.  The library never aborts.
  *   - A device pointer must be 16-byte aligned (AWQ_ERR_ALIGNMENT otherwise).
  *   - Errors found on the device (non-finite inputs, a bounded wait that
- *     gave up) are reported in the outputs, as each entry point states.
+ *     gave up) are reported twice: in the outputs, as each entry point
+ *     states, and as sticky condition bits of the device (AWQ_FLAG_*), which
+ *     awq_last_device_flags() returns and clears.
  *   - Results are deterministic: the same inputs give the same bits.
  *   - The calls may run concurrently on different streams provided their
  *     workspaces do not overlap.
@@ -50,7 +52,8 @@ typedef enum awq_status {
     AWQ_ERR_ALIGNMENT = 3,     /* a pointer or leading dimension misaligned   */
     AWQ_ERR_WORKSPACE = 4,     /* workspace NULL or smaller than required      */
     AWQ_ERR_CUDA = 5,          /* a CUDA runtime call or launch failed         */
-    AWQ_ERR_NONFINITE = 6      /* reserved: non-finite data (see outputs)      */
+    AWQ_ERR_NONFINITE = 6,     /* non-finite data met on the device (flags)    */
+    AWQ_ERR_DEVICE_TIMEOUT = 7 /* a bounded device-side wait gave up (flags)   */
 } awq_status;
 
 /* Flags of awq_scale_search / awq_output_error / awq_clip_search. */
@@ -85,6 +88,40 @@ typedef enum awq_status {
 #define AWQ_CLIP_DEN 20
 #define AWQ_CLIP_MAX 20
 
+/* Condition bits raised on the device (awq_last_device_flags). */
+#define AWQ_FLAG_NONFINITE_X     0x1u  /* awq_act_stats: a column of X held a NaN or
+                                          an infinity (its x_mean is NaN or inf)  */
+#define AWQ_FLAG_NONFINITE_SCORE 0x2u  /* awq_scale_search / awq_output_error /
+                                          awq_clip_search: an error sum was not
+                                          finite (NaN or inf in W, x_mean or s);
+                                          best_idx is -1, err NaN or inf          */
+#define AWQ_FLAG_NONFINITE_GROUP 0x4u  /* awq_quantize_pack: a group held a NaN or
+                                          an infinity (it stored scale NaN)      */
+#define AWQ_FLAG_NONFINITE_SCALE 0x8u  /* awq_norm_group_scale: a member scale or
+                                          the shared scale was not finite        */
+#define AWQ_FLAG_WAIT_TIMEOUT    0x10u /* a bounded wait inside a kernel gave up
+                                          (best_idx -2; outputs invalid)         */
+
+/*
+ * Sticky device-side condition bits of the CURRENT device.  The kernels of
+ * every entry point raise AWQ_FLAG_* bits there (in addition to what their
+ * outputs show) when they meet non-finite data or give up a bounded wait;
+ * the bits accumulate over calls, streams and host threads until read with
+ * clear != 0.
+ *
+ *   flags   HOST output: the bits raised since the last clearing read
+ *   clear   nonzero: zero the bits after reading them
+ *
+ * Synchronises the current device first (cudaDeviceSynchronize), so every
+ * call enqueued before it is reflected.  Returns AWQ_ERR_DEVICE_TIMEOUT if
+ * AWQ_FLAG_WAIT_TIMEOUT is set, else AWQ_ERR_NONFINITE if any other bit is
+ * set, else AWQ_OK; AWQ_ERR_CUDA if the synchronisation or the read failed
+ * (e.g. an earlier kernel faulted), with awq_last_error() holding the text.
+ * Clearing while other host threads enqueue work on the device may drop bits
+ * raised by that work.
+ */
+awq_status awq_last_device_flags(uint32_t *flags, int clear);
+
 /* Human-readable name of a status code (static storage; never NULL). */
 const char *awq_status_string(int status);
 
@@ -117,7 +154,8 @@ awq_status awq_workspace_size(int op, int64_t T, int64_t d_out_total,
  *
  * The sum is exact (every |fp16| is an integer multiple of 2^-24), then
  * divided by T in fp64 and rounded to fp32.  A column holding a NaN gives
- * NaN, one holding an infinity (and no NaN) gives +inf.
+ * NaN, one holding an infinity (and no NaN) gives +inf; either raises
+ * AWQ_FLAG_NONFINITE_X.
  *
  *   X        fp16 [T, ld] device, 16-byte aligned; ld % 8 == 0, ld >= d_in
  *   T        tokens, 1 <= T <= 2^23
@@ -160,7 +198,8 @@ awq_status awq_act_stats(const void *X, int64_t T, int64_t d_in, int64_t ld,
  *   flags       AWQ_SCALE_FP16 or AWQ_SCALE_FP32
  *   err         fp64 [n_grid] device output
  *   best_idx    int32 [1] device output; -1 if any err is not finite (NaN or
- *               infinite input), -2 if a device-side wait gave up
+ *               infinite input; raises AWQ_FLAG_NONFINITE_SCORE), -2 if a
+ *               device-side wait gave up (raises AWQ_FLAG_WAIT_TIMEOUT)
  *   s_best      fp32 [d_in] device output (NaN when best_idx < 0)
  *   ws          workspace of awq_workspace_size(AWQ_OP_SCALE_SEARCH, ...)
  * Each term is evaluated in fp32 as (ws - q * q_scale)^2 * (x_mean/s_i)^2,
@@ -194,8 +233,10 @@ awq_status awq_scale_search(int n_seg, const void *const *W,
  * enqueued -- e.g. d_in = 16384 fits with n_grid <= 29, d_in = 12288 with
  * n_grid <= 32; duo scaling needs d_in * 8 bytes per weight-mean CTA on top
  * and so fits only small d_in (d_in <= 2048 at 20 grid points).  The first call on a device looks the array's address up
- * (cudaGetSymbolAddress, that device current) and caches it: make it before
- * any stream capture on that device.  All calls on a device share the array;
+ * (cudaGetSymbolAddress, that device current) and caches it for the life of
+ * the process: make it before any stream capture on that device, and do not
+ * use this entry point on a device after a cudaDeviceReset of it (the cached
+ * address belonged to the destroyed context).  All calls on a device share the array;
  * each call rewrites every scratch byte it reads, but calls that overlap on
  * the GPU (unordered streams) race on it.  Allocates nothing.
  */
@@ -240,7 +281,7 @@ awq_status awq_scale_search_noalloc(int n_seg, const void *const *W,
  *   scales      fp16 [d_in / group_size, d_out] device output
  *   qzeros      int32 [d_in / group_size, d_out / 8] device output
  * A group holding a non-finite value stores scale NaN (0x7E00) and code
- * zero_point for all its weights.
+ * zero_point for all its weights, and raises AWQ_FLAG_NONFINITE_GROUP.
  */
 awq_status awq_quantize_pack(const void *W, int64_t d_out, int64_t d_in,
                              const float *s, const uint8_t *clip_idx,
@@ -263,7 +304,10 @@ awq_status awq_quantize_pack(const void *W, int64_t d_out, int64_t d_in,
  *   s          HOST array of n DEVICE pointers, fp32 [d_in] each (each
  *              normally the s_best of a one-segment awq_scale_search)
  *   d_in       1..2^24 channels
- *   s_shared   fp32 [d_in] device output
+ *   s_shared   fp32 [d_in] device output (a channel whose member scales
+ *              hold a NaN, an infinity, or whose product leaves the fp64
+ *              range gets that non-finite value and raises
+ *              AWQ_FLAG_NONFINITE_SCALE)
  */
 awq_status awq_norm_group_scale(int n, const float *const *s, int64_t d_in,
                                 float *s_shared, void *stream);
@@ -297,7 +341,8 @@ awq_status awq_norm_group_scale(int n, const float *const *s, int64_t d_in,
  *   flags       AWQ_SCALE_FP16 or AWQ_SCALE_FP32
  *   clip_idx    uint8 [d_out, d_in / group_size] device output
  *   err         fp64 [2] device output (NaN if W holds a non-finite value;
- *               such a group keeps index 0)
+ *               such a group keeps index 0; a non-finite total raises
+ *               AWQ_FLAG_NONFINITE_SCORE)
  *   ws          workspace of awq_workspace_size(AWQ_OP_CLIP_SEARCH, ...),
  *               256-byte aligned
  */
@@ -334,7 +379,8 @@ awq_status awq_clip_search(const void *W, int64_t d_out, int64_t d_in,
  *   err         fp64 [n_grid] device output (NaN for every i if W holds a
  *               non-finite value)
  *   best_idx    int32 [1] device output (first minimum; -1 if non-finite,
- *               -2 if a bounded wait inside a kernel gave up)
+ *               raising AWQ_FLAG_NONFINITE_SCORE; -2 if a bounded wait
+ *               inside a kernel gave up, raising AWQ_FLAG_WAIT_TIMEOUT)
  *   s_best      fp32 [d_in] device output s_{best_idx} (NaN if best_idx < 0),
  *               or NULL when the caller does not want it
  *   ws          workspace of awq_workspace_size(AWQ_OP_OUTPUT_ERROR, ...),

@@ -28,6 +28,12 @@ ASYMMETRIC = 4
 ZERO_POINT_ASYM = -1
 CLIP_DEN = 20
 MAX_SEGMENTS = 8
+# sticky device-side condition bits (awq_last_device_flags)
+FLAG_NONFINITE_X = 0x1
+FLAG_NONFINITE_SCORE = 0x2
+FLAG_NONFINITE_GROUP = 0x4
+FLAG_NONFINITE_SCALE = 0x8
+FLAG_WAIT_TIMEOUT = 0x10
 
 LIB_PATH = _build.LIB
 
@@ -75,6 +81,8 @@ def lib() -> ctypes.CDLL:
         L.awq_clip_search.restype = i32
         L.awq_output_error.argtypes = [p, i64, p, i64, i64, p, i32, i32, i32, p, p, p, p, sz, p]
         L.awq_output_error.restype = i32
+        L.awq_last_device_flags.argtypes = [ctypes.POINTER(ctypes.c_uint32), i32]
+        L.awq_last_device_flags.restype = i32
         _lib = L
     return _lib
 
@@ -100,6 +108,18 @@ def _cuda(t: torch.Tensor, dtype, name: str) -> torch.Tensor:
 
 def _stream(device) -> int:
     return torch.cuda.current_stream(device).cuda_stream
+
+
+def last_device_flags(clear: bool = True) -> Tuple[int, int]:
+    """awq_last_device_flags on the current device: (status, AWQ_FLAG_* bits
+    raised since the last clearing read).  Synchronises the device.  Status 6
+    (AWQ_ERR_NONFINITE) and 7 (AWQ_ERR_DEVICE_TIMEOUT) are returned, not
+    raised; any other non-zero status raises AwqError."""
+    bits = ctypes.c_uint32(0)
+    st = lib().awq_last_device_flags(ctypes.byref(bits), 1 if clear else 0)
+    if st not in (0, 6, 7):
+        raise AwqError(st, "awq_last_device_flags")
+    return st, int(bits.value)
 
 
 def workspace_size(op: int, T: int, d_out_total: int, d_in: int, group_size: int,

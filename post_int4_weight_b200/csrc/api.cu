@@ -63,14 +63,36 @@ const char* awq_status_string(int status) {
         case AWQ_ERR_ALIGNMENT: return "AWQ_ERR_ALIGNMENT: pointer or stride misaligned";
         case AWQ_ERR_WORKSPACE: return "AWQ_ERR_WORKSPACE: workspace missing or too small";
         case AWQ_ERR_CUDA: return "AWQ_ERR_CUDA: CUDA runtime or launch failure";
-        case AWQ_ERR_NONFINITE: return "AWQ_ERR_NONFINITE: non-finite data";
+        case AWQ_ERR_NONFINITE: return "AWQ_ERR_NONFINITE: non-finite data met on the device";
+        case AWQ_ERR_DEVICE_TIMEOUT:
+            return "AWQ_ERR_DEVICE_TIMEOUT: a bounded device-side wait gave up";
         default: return "unknown awq_status";
     }
 }
 
-int awq_abi_version(void) { return 100; }
+int awq_abi_version(void) { return 101; }
 
 const char* awq_last_error(void) { return g_last_error; }
+
+awq_status awq_last_device_flags(uint32_t* flags, int clear) {
+    if (!flags) return AWQ_ERR_INVALID_ARG;
+    *flags = 0;
+    if (note_cuda(cudaDeviceSynchronize(), "awq_last_device_flags: cudaDeviceSynchronize") !=
+        cudaSuccess)
+        return AWQ_ERR_CUDA;
+    unsigned int bits = 0;
+    const bool c = clear != 0;
+    cudaError_t (*const units[])(unsigned int*, bool) = {
+        stats_unit_flags, search_unit_flags, pack_unit_flags, clip_unit_flags,
+        norm_group_unit_flags};
+    for (auto unit : units)
+        if (note_cuda(unit(&bits, c), "awq_last_device_flags: flag word") != cudaSuccess)
+            return AWQ_ERR_CUDA;
+    *flags = bits;
+    if (bits & AWQ_FLAG_WAIT_TIMEOUT) return AWQ_ERR_DEVICE_TIMEOUT;
+    if (bits) return AWQ_ERR_NONFINITE;
+    return AWQ_OK;
+}
 
 awq_status awq_workspace_size(int op, int64_t T, int64_t d_out_total, int64_t d_in,
                               int group_size, int n_grid, size_t* bytes) {

@@ -256,6 +256,7 @@ clip_kernel(const ClipParams p) {
         if (lane == 0) {
             p.err[0] = a;
             p.err[1] = b;
+            if (!isfinite(a) || !isfinite(b)) raise_device_flag(AWQ_FLAG_NONFINITE_SCORE);
         }
     }
 }
@@ -266,6 +267,10 @@ cudaError_t launch_clip_L(const ClipParams& p, int grid, cudaStream_t st) {
 }
 
 }  // namespace
+
+cudaError_t clip_unit_flags(unsigned int* bits, bool clear) {
+    return unit_device_flags(bits, clear);
+}
 
 size_t clip_search_workspace() {
     return align_up((size_t)kMaxClipCtas * 2 * sizeof(double), kWsAlign) + kWsAlign;

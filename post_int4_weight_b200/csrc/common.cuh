@@ -21,8 +21,44 @@ constexpr float kFloatMinNormal = 1.17549435e-38f;  // 2^-126
 // Host-visible error bits written into a workspace word by the kernels.
 constexpr int kDevErrWaitTimeout = 1;
 
-// Bound on any spin-wait: 2 seconds of %globaltimer.
+// Bound on any spin-wait of a pipeline: 2 seconds of %globaltimer.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
+// Bound on a drain wait: after a pipeline wait gave up, a CTA still waits for
+// its own copies (or MMAs) in flight before it exits, so that none of them
+// writes shared memory or TMEM that the CTA no longer owns.  Ten times the
+// pipeline's limit: a copy that has not landed by then means the memory
+// system is not making progress at all; the CTA then leaves with the timeout
+// bit set, and its outputs are reported invalid.
+constexpr uint64_t kDrainLimitNs = 20000000000ull;
+
+// ------------------------------------------------------ sticky device flags
+// Condition bits (AWQ_FLAG_* of awq.h) that kernels raise when they meet
+// non-finite data or give up a bounded wait.  Each .cu file is its own device
+// module (the library is built without relocatable device code), so each
+// gets its own copy of this word; awq_last_device_flags() reads and clears
+// every module's copy through the host accessor each file defines with
+// unit_device_flags().  A raise is one atomic OR, taken only on those rare
+// paths.
+static __device__ unsigned int g_unit_flags;
+
+__device__ __forceinline__ void raise_device_flag(unsigned int bits) {
+    atomicOr(&g_unit_flags, bits);
+}
+
+// Host side: ORs this module's word into *bits and, if `clear`, zeroes it.
+// Synchronous (cudaMemcpyFromSymbol / ToSymbol); the caller has synchronised
+// the device first.
+static inline cudaError_t unit_device_flags(unsigned int* bits, bool clear) {
+    unsigned int v = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(&v, g_unit_flags, sizeof v);
+    if (e != cudaSuccess) return e;
+    *bits |= v;
+    if (clear && v) {
+        const unsigned int zero = 0;
+        e = cudaMemcpyToSymbol(g_unit_flags, &zero, sizeof zero);
+    }
+    return e;
+}
 
 __device__ __forceinline__ uint64_t global_ns() {
     uint64_t t;
@@ -73,6 +109,16 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
     const uint64_t t0 = global_ns();
     while (!mbar_try_wait(bar, parity)) {
         if (global_ns() - t0 > kWaitLimitNs) return false;
+    }
+    return true;
+}
+
+// A drain wait: the same, with the longer kDrainLimitNs.
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (global_ns() - t0 > kDrainLimitNs) return false;
     }
     return true;
 }

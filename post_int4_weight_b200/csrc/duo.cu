@@ -270,7 +270,7 @@ wmean_partial_kernel(const __grid_constant__ WmParams p) {
     if (failed && tid == 0) {
         // batches b .. b + NB - 1 may still have copies in flight
         for (int64_t bb = b; bb < b + NB && bb < n_batches; ++bb)
-            (void)mbar_wait_bounded(&full[bb % NB], (uint32_t)(bb / NB) & 1u);
+            if (!mbar_wait_drain(&full[bb % NB], (uint32_t)(bb / NB) & 1u)) failed = true;
     }
     if (tid == 0) p.status[blockIdx.x] = failed ? kDevErrWaitTimeout : 0;
     pdl_launch_dependents();

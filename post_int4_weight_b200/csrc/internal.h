@@ -44,6 +44,14 @@ struct DeviceInfo {
 };
 cudaError_t query_device(DeviceInfo* info);
 
+// ---- sticky device flags: each device module's accessor (ORs its word into
+// *bits, zeroes it if `clear`; the caller has synchronised the device)
+cudaError_t stats_unit_flags(unsigned int* bits, bool clear);
+cudaError_t search_unit_flags(unsigned int* bits, bool clear);
+cudaError_t pack_unit_flags(unsigned int* bits, bool clear);
+cudaError_t clip_unit_flags(unsigned int* bits, bool clear);
+cudaError_t norm_group_unit_flags(unsigned int* bits, bool clear);
+
 // ---- activation statistics
 size_t act_stats_workspace(int64_t d_in);
 cudaError_t launch_act_stats(const void* X, int64_t T, int64_t d_in, int64_t ld,

@@ -25,17 +25,24 @@ geomean_kernel(const __grid_constant__ ScalePtrs p, int n, int64_t d_in, float* 
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; j < d_in; j += stride) {
         if (n == 1) {
-            out[j] = p.s[0][j];
+            const float v = p.s[0][j];
+            out[j] = v;
+            if (!isfinite(v)) raise_device_flag(AWQ_FLAG_NONFINITE_SCALE);
             continue;
         }
         double prod = 1.0;
         for (int m = 0; m < n; ++m) prod = __dmul_rn(prod, (double)p.s[m][j]);
         const double r = (n == 2) ? __dsqrt_rn(prod) : pow(prod, __drcp_rn((double)n));
         out[j] = __double2float_rn(r);
+        if (!isfinite(prod)) raise_device_flag(AWQ_FLAG_NONFINITE_SCALE);
     }
 }
 
 }  // namespace
+
+cudaError_t norm_group_unit_flags(unsigned int* bits, bool clear) {
+    return unit_device_flags(bits, clear);
+}
 
 cudaError_t launch_norm_group_scale(int n, const float* const* s, int64_t d_in, float* out,
                                     int num_sms, cudaStream_t stream) {

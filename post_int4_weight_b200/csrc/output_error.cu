@@ -225,7 +225,8 @@ oe_gemm_kernel(const __grid_constant__ GemmParams p) {
             }
             if (*abort_flag) {   // leave no TMA copy writing this CTA's shared memory
                 for (int s = 0; s < kStages; ++s)
-                    if (issued[s] > 0) (void)mbar_wait_bounded(&full[s], (issued[s] - 1) & 1u);
+                    if (issued[s] > 0 && !mbar_wait_drain(&full[s], (issued[s] - 1) & 1u))
+                        atomicOr(p.dev_err, kDevErrWaitTimeout);
             }
         }
     } else if (warp == 1) {
@@ -267,7 +268,7 @@ oe_gemm_kernel(const __grid_constant__ GemmParams p) {
             }
             if (*abort_flag) {   // no MMA may still write TMEM when it is freed
                 umma_commit(drain);
-                (void)mbar_wait_bounded(drain, 0);
+                if (!mbar_wait_drain(drain, 0)) atomicOr(p.dev_err, kDevErrWaitTimeout);
             }
         }
     } else {

@@ -214,6 +214,7 @@ pack_kernel(const uint4* __restrict__ W, int64_t d_out, int64_t d_in,
                 qr_tile[row_slot(kk, r)] = make_float2(qs, __frcp_rn(qs));
                 bad_tile[row_slot(kk, r)] = bad;
                 zero_tile[row_slot(kk, r)] = z;
+                if (bad) raise_device_flag(AWQ_FLAG_NONFINITE_GROUP);
                 const int64_t gr = row0 + r, gk = col0 / G + kk;
                 if (gr < d_out && gk * G < d_in)
                     scales[gk * d_out + gr] = bad ? __ushort_as_half((unsigned short)0x7E00)
@@ -275,6 +276,7 @@ pack_kernel(const uint4* __restrict__ W, int64_t d_out, int64_t d_in,
                 const float qs = bad ? 1.0f : group_scale(m, false, &in_range);
                 qr_tile[row_slot(kk, r)] = make_float2(qs, (qs > 0.f) ? __frcp_rn(qs) : 0.f);
                 bad_tile[row_slot(kk, r)] = bad;
+                if (bad) raise_device_flag(AWQ_FLAG_NONFINITE_GROUP);
                 if (bad || clipped || !in_range) slow_blk[kk * kBlocks32 + r / 32] = 1;
                 if (gr < d_out && gk * G < d_in)
                     scales[gk * d_out + gr] = bad ? __ushort_as_half((unsigned short)0x7E00)
@@ -368,6 +370,10 @@ cudaError_t launch_pack_G(const void* W, int64_t d_out, int64_t d_in, const floa
 }
 
 }  // namespace
+
+cudaError_t pack_unit_flags(unsigned int* bits, bool clear) {
+    return unit_device_flags(bits, clear);
+}
 
 cudaError_t launch_quantize_pack(const void* W, int64_t d_out, int64_t d_in, const float* s,
                                  const uint8_t* clip_idx, int group_size, int zero_point,

@@ -148,8 +148,14 @@ __device__ void finalize_cta(const double* partial, int n_parts, int n_grid,
             if (!isfinite(e_s[i])) finite = false;
             if (e_s[i] < e_s[b]) b = i;
         }
-        if (!finite) b = -1;
-        if (dev_err) b = -2;
+        if (!finite) {
+            b = -1;
+            raise_device_flag(AWQ_FLAG_NONFINITE_SCORE);
+        }
+        if (dev_err) {
+            b = -2;
+            raise_device_flag(AWQ_FLAG_WAIT_TIMEOUT);
+        }
         *best_s = b;
         *best_idx = b;
     }
@@ -576,10 +582,13 @@ search_kernel(const __grid_constant__ SearchParams p) {
     pdl_launch_dependents();
 
     // drain: never leave the CTA while a TMA copy may still write its smem.
-    // The n-th load into a stage completes that barrier's phase n.
+    // The n-th load into a stage completes that barrier's phase n.  On the
+    // normal path every load was consumed and these waits return at once; a
+    // drain that gives up (kDrainLimitNs) marks the result invalid.
     if (tid == 0) {
         for (int s = 0; s < kStages; ++s)
-            if (issued[s] > 0) (void)mbar_wait_bounded(&full[s], (uint32_t)(issued[s] - 1) & 1u);
+            if (issued[s] > 0 && !mbar_wait_drain(&full[s], (uint32_t)(issued[s] - 1) & 1u))
+                atomicOr(&p.dev_words[0], kDevErrWaitTimeout);
     }
     __syncthreads();
 
@@ -764,6 +773,10 @@ cudaError_t launch_search(int L, const SearchParams& p, int grid, size_t smem,
 }
 
 }  // namespace
+
+cudaError_t search_unit_flags(unsigned int* bits, bool clear) {
+    return unit_device_flags(bits, clear);
+}
 
 size_t scale_search_workspace(int64_t d_in, int group_size, int n_grid) {
     (void)group_size;

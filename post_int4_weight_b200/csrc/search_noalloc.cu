@@ -13,8 +13,11 @@
 //   * the array is a static device symbol, so every GPU on which this library
 //     is used holds kNoAllocScratchBytes of it until the process exits;
 //   * the first call on a device looks up the array's device address with
-//     cudaGetSymbolAddress (with that device current) and caches it; make that
-//     first call before any stream capture on that device;
+//     cudaGetSymbolAddress (with that device current) and caches it for the
+//     life of the process; make that first call before any stream capture on
+//     that device.  A cudaDeviceReset destroys the context the address
+//     belongs to, so the cached address is stale afterwards: do not call this
+//     entry point on a device after resetting it;
 //   * every call on a device shares the one array and it keeps the previous
 //     call's contents.  The kernels overwrite every scratch byte they read
 //     (scale tables, per-CTA partial sums) and clear the error word first, so
@@ -62,14 +65,19 @@ extern "C" awq_status awq_scale_search_noalloc(int n_seg, const void* const* W,
                                                int n_grid, int flags, double* err,
                                                int32_t* best_idx, float* s_best,
                                                void* stream) {
-    size_t need = 0;
-    const awq_status st =
-        awq_workspace_size(AWQ_OP_SCALE_SEARCH, 1, 8, d_in, group_size, n_grid, &need);
-    if (st != AWQ_OK) return st;
-    if (need > kNoAllocScratchBytes) return AWQ_ERR_WORKSPACE;
+    // Argument checks first, through the workspace entry point itself with no
+    // workspace: it validates every argument and then, finding no workspace,
+    // returns AWQ_ERR_WORKSPACE with nothing enqueued.  Any other code is an
+    // argument error, reported exactly as awq_scale_search reports it.
+    const awq_status pre = awq_scale_search(n_seg, W, d_out, d_in, x_mean, group_size,
+                                            n_grid, flags, err, best_idx, s_best, nullptr, 0,
+                                            stream);
+    if (pre != AWQ_ERR_WORKSPACE) return pre;
     void* scratch = nullptr;
     const awq_status s2 = scratch_on_current_device(&scratch);
     if (s2 != AWQ_OK) return s2;
+    // a size whose workspace need exceeds the array is rejected there with
+    // AWQ_ERR_WORKSPACE, again before anything is enqueued
     return awq_scale_search(n_seg, W, d_out, d_in, x_mean, group_size, n_grid, flags, err,
                             best_idx, s_best, scratch, kNoAllocScratchBytes, stream);
 }

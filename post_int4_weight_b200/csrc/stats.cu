@@ -218,8 +218,10 @@ stats_kernel(const uint4* __restrict__ X, int64_t T, int64_t d_in, int64_t ld_ch
             float v;
             if (f & 2u) {
                 v = __int_as_float(0x7fc00000);
+                raise_device_flag(AWQ_FLAG_NONFINITE_X);
             } else if (f & 1u) {
                 v = __int_as_float(0x7f800000);
+                raise_device_flag(AWQ_FLAG_NONFINITE_X);
             } else {
                 const double s = __ull2double_rn(red[tid]);
                 v = __double2float_rn(__ddiv_rn(s * 0x1p-24, (double)T));
@@ -230,6 +232,10 @@ stats_kernel(const uint4* __restrict__ X, int64_t T, int64_t d_in, int64_t ld_ch
 }
 
 }  // namespace
+
+cudaError_t stats_unit_flags(unsigned int* bits, bool clear) {
+    return unit_device_flags(bits, clear);
+}
 
 size_t act_stats_workspace(int64_t d_in) {
     (void)d_in;

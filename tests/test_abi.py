@@ -35,9 +35,28 @@ def test_library_exports_every_declared_symbol():
 
 def test_status_strings_and_version():
     assert awq.string(0) == "AWQ_OK"
-    for s in range(1, 7):
+    for s in range(1, 8):
         assert awq.string(s).startswith("AWQ_ERR_")
-    assert awq.lib().awq_abi_version() == 100
+    assert awq.string(6).startswith("AWQ_ERR_NONFINITE")
+    assert awq.string(7).startswith("AWQ_ERR_DEVICE_TIMEOUT")
+    assert awq.lib().awq_abi_version() == 101
+
+
+def test_device_flag_bits_in_header_and_binding():
+    """The AWQ_FLAG_* bits of the header are distinct powers of two and the
+    binding carries the same values; a NULL output is an argument error,
+    answered on the host."""
+    text = open(HEADER).read()
+    bits = {m.group(1): int(m.group(2), 16)
+            for m in re.finditer(r"#define\s+(AWQ_FLAG_\w+)\s+0x([0-9a-fA-F]+)u", text)}
+    assert set(bits) == {"AWQ_FLAG_NONFINITE_X", "AWQ_FLAG_NONFINITE_SCORE",
+                         "AWQ_FLAG_NONFINITE_GROUP", "AWQ_FLAG_NONFINITE_SCALE",
+                         "AWQ_FLAG_WAIT_TIMEOUT"}
+    vals = sorted(bits.values())
+    assert len(set(vals)) == len(vals) and all(v & (v - 1) == 0 for v in vals)
+    for name, v in bits.items():
+        assert getattr(awq, name[4:]) == v
+    assert awq.lib().awq_last_device_flags(None, 0) == 1   # AWQ_ERR_INVALID_ARG
 
 
 def test_workspace_sizes():
