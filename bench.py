@@ -54,10 +54,11 @@ UNIT = "Gparam/s"
 # q_scale, round, two clamps, multiply q*q_scale, divide by s, subtract,
 # multiply by x, square-accumulate.
 ALG_OPS_PER_PAIR = 11
-# FMA-pipe lane operations the search kernel actually executes per pair
-# (w*s, the rounding addition and its removal, the residual, the weighted
-# square-accumulate shared by a lane's two rows) -- reported beside it.
-FMA_OPS_PER_PAIR = 5
+# FMA-pipe lane operations the search kernel actually executes per pair:
+# w*s, the rounding addition and its removal, the residual, the square, and
+# half of the weighted accumulate that a lane's two rows share -- reported
+# beside it.
+FMA_OPS_PER_PAIR = 5.5
 # dram__bytes_read.sum + dram__bytes_write.sum of one launch of the dominant
 # kernel from the committed ncu captures (profiles/), for the kernels as they
 # stand; None where no capture of the current kernel exists.
@@ -113,7 +114,7 @@ def _peaks():
 # ----------------------------------------------------------------- clocks --
 
 class ClockSampler:
-    """Samples SM clock and clock-event reasons through NVML every 20 ms."""
+    """Samples SM clock and clock-event reasons through NVML every 2 ms."""
 
     REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
                0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
@@ -153,7 +154,7 @@ class ClockSampler:
                 self.reasons |= int(nv.nvmlDeviceGetCurrentClocksEventReasons(self._h))
             except Exception:
                 pass
-            time.sleep(0.02)
+            time.sleep(0.002)
 
     def __enter__(self):
         if self._h is not None:
@@ -172,6 +173,116 @@ class ClockSampler:
         names = [n for b, n in self.REASONS.items() if self.reasons & b and b != 0x1]
         return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
                 "reasons": names, "samples": len(self.samples)}
+
+
+def fp32_rate_probe(dev):
+    """Measured FP32 FMA rate of this GPU from the probe library
+    (libawq_probe.so): lane-ops per second for scalar FFMA, packed FFMA2 and
+    a half-and-half mix, best of 5 launches each, with the SM clock sampled
+    meanwhile.  None if the probe is unavailable."""
+    import ctypes
+    import torch
+    from post_int4_weight_b200 import build as b
+    try:
+        L = ctypes.CDLL(b.PROBE_LIB)
+    except OSError:
+        return None
+    fn = L.awq_probe_fp32_rate
+    fn.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_void_p,
+                   ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double)]
+    fn.restype = ctypes.c_int
+    n_sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    out = torch.empty(n_sms * 8 * 256, dtype=torch.float32, device=dev)
+    rates = {}
+    ck = ClockSampler(dev)
+    with ck:
+        for mode, name in ((0, "scalar_ffma"), (1, "packed_ffma2"), (2, "half_packed")):
+            ops, t = ctypes.c_double(0), ctypes.c_double(0)
+            if fn(mode, 32768, 5, out.data_ptr(), ctypes.byref(ops), ctypes.byref(t)) != 0:
+                return None
+            rates[name] = ops.value / (t.value * 1e-3)
+    summ = ck.summary()
+    mhz = summ["sm_mhz"] or summ["sm_max_mhz"]
+    best = max(rates.values())
+    return {"lane_op_per_s": rates, "best": best, "sm_mhz": mhz,
+            "samples": summ.get("samples", 0),
+            "lane_op_per_clk_per_sm": best / (n_sms * mhz * 1e6) if mhz else None}
+
+
+def launch_stream_times(jobs, wss, dev, stream, target_bytes=768 << 20, reps=20):
+    """Average launch duration of awq_act_stats and of awq_quantize_pack in a
+    steady stream: one CUDA graph of back-to-back calls, each on its own copy
+    of the inputs (copies rotate, more bytes than the 126 MB L2 in all, so
+    every call reads cold data), timed with CUDA events around the replay and
+    divided by the number of calls.  Returns {"stats": ms, "pack": ms,
+    "copies": n, "rot_bytes": bytes}."""
+    import torch
+    from post_int4_weight_b200 import awq
+    in_bytes = sum(j.X.numel() * 2 + sum(W.numel() * 2 for W in j.Ws) for j in jobs)
+    n = max(2, min(16, -(-target_bytes // max(in_bytes, 1))))
+    if n * in_bytes > (6 << 30):
+        return {}
+    Xs = [[j.X.clone() for j in jobs] for _ in range(n)]
+    Ws = [[[W.clone() for W in j.Ws] for j in jobs] for _ in range(n)]
+
+    def stats_all():
+        for c in range(n):
+            for j, X in zip(jobs, Xs[c]):
+                awq.act_stats(X, out=j.x, ws=wss.stats)
+
+    def pack_all():
+        for c in range(n):
+            for j, Wl in zip(jobs, Ws[c]):
+                for W, pk in zip(Wl, j.packs):
+                    awq.quantize_pack(W, j.s_best, j.g, j.zero_point, out=pk)
+
+    out = {"copies": n, "rot_bytes": n * in_bytes}
+    calls = {"stats": (stats_all, n * len(jobs)),
+             "pack": (pack_all, n * sum(len(j.Ws) for j in jobs))}
+    for name, (fn, n_calls) in calls.items():
+        fn()
+        torch.cuda.synchronize(dev)
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr):
+            fn()
+        ts = []
+        for _ in range(reps):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            gr.replay()
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            ts.append(e0.elapsed_time(e1))
+        out[name] = statistics.median(ts) / n_calls
+        del gr
+    del Xs, Ws
+    return out
+
+
+def h2d_bound_GBps(host_layer, dev, passes=5):
+    """Pinned host -> device copy rate of one layer's input buffers: one
+    cudaMemcpyAsync (torch non-blocking copy) per buffer, back to back on one
+    stream, best of `passes` passes."""
+    import torch
+    bufs = [t for Ws, X in host_layer for t in (*Ws, X)]
+    dst = [torch.empty_like(t, device=dev) for t in bufs]
+    nbytes = sum(t.numel() * t.element_size() for t in bufs)
+    st = torch.cuda.Stream(dev)
+    best = None
+    with torch.cuda.stream(st):
+        for _ in range(passes + 1):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(st)
+            for d, h in zip(dst, bufs):
+                d.copy_(h, non_blocking=True)
+            e1.record(st)
+            e1.synchronize()
+            t = e0.elapsed_time(e1)
+            best = t if best is None else min(best, t)
+    del dst
+    return nbytes / (best * 1e-3) / 1e9
 
 
 # ---------------------------------------------------------------- our arm --
@@ -296,7 +407,8 @@ def run_ours(a):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
-    with ClockSampler(dev) as clk:
+    clk = ClockSampler(dev)
+    with clk:
         for k in range(a.steps):
             do_flush()
             evs[k][0].record(stream)
@@ -308,25 +420,30 @@ def run_ours(a):
     t_step = [e0.elapsed_time(e1) for e0, e1 in evs]
     ms = pipeline.max_over_ranks(sum(t_step) / len(t_step), dev)
 
-    # per-call breakdown (separately timed passes, L2 flushed before each)
-    n_br = max(3, min(200, a.steps))
+    # per-call breakdown (separately timed passes, L2 flushed before each);
+    # about 0.2 s of passes, 3 to 200 of them; the clock sampler keeps
+    # running over them (their kernels are the step's)
+    n_br = max(3, min(200, int(200.0 / max(ms, 1e-3))))
     names = ["stats", "search"] + (["clip"] if a.clip > 0 else []) + ["pack"]
     br = {k: [] for k in names}
-    for _ in range(n_br):
-        do_flush()
-        ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
-        ev[0].record(stream)
-        for i, k in enumerate(names):
-            run[k]()
-            ev[i + 1].record(stream)
-        torch.cuda.synchronize(dev)
-        for i, k in enumerate(names):
-            br[k].append(ev[i].elapsed_time(ev[i + 1]))
+    clk_br = ClockSampler(dev)
+    with clk_br:
+        for _ in range(n_br):
+            do_flush()
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
+            ev[0].record(stream)
+            for i, k in enumerate(names):
+                run[k]()
+                ev[i + 1].record(stream)
+            torch.cuda.synchronize(dev)
+            for i, k in enumerate(names):
+                br[k].append(ev[i].elapsed_time(ev[i + 1]))
     ms_stats = sum(br["stats"]) / n_br
     ms_search = sum(br["search"]) / n_br
     ms_pack = sum(br["pack"]) / n_br
     ms_clip = sum(br["clip"]) / n_br if a.clip > 0 else None
     del graphs
+    stream_ms = launch_stream_times(jobs, wss, dev, stream) if work.layers == 1 else {}
 
     # --- end to end: the same work streamed from pinned host memory
     template = layer_inputs[0]
@@ -334,7 +451,7 @@ def run_ours(a):
                                       n_clip=a.clip, scale_mode=a.scale_mode, duo=a.duo,
                                       asym=a.asym)
     if work.layers == 1:
-        n_e2e = max(5, min(50, a.steps // 20))
+        n_e2e = max(20, min(50, a.steps // 20))
         host_layers = [host_layer] * n_e2e
         out_one = streamer.host_outputs()
         host_out = [out_one] * n_e2e
@@ -361,12 +478,17 @@ def run_ours(a):
     torch.cuda.synchronize(dev)
     ms_e2e = pipeline.max_over_ranks(e0.elapsed_time(e1) / e2e_units, dev)
     h2d_l, d2h_l = streamer.bytes_per_layer()
+    h2d_bound = h2d_bound_GBps(host_layers[0], dev)
     per_step_layers = len(host_layers) // e2e_units
     e2e = {"value": _total_params(work, world, params) / (ms_e2e * 1e-3) / 1e9, "unit": UNIT,
            "ms_per_step": ms_e2e, "h2d_bytes_per_step": int(h2d_l * per_step_layers),
            "d2h_bytes_per_step": int(d2h_l * per_step_layers), "steps": e2e_units,
            # the copies bound this number: host->device bytes over the step time
            "h2d_GBps": h2d_l * per_step_layers / (ms_e2e * 1e-3) / 1e9,
+           "h2d_bound_GBps": h2d_bound,
+           "h2d_frac": (h2d_l * per_step_layers / (ms_e2e * 1e-3) / 1e9) / h2d_bound,
+           "h2d_bound_basis": "the same pinned host buffers copied to the device with one "
+                              "cudaMemcpyAsync each, back to back, best of 5 passes",
            "pipeline": "pinned host -> 2-slot device ring; H2D, kernels and D2H on three "
                        "streams, overlapped across layers"}
 
@@ -377,17 +499,34 @@ def run_ours(a):
 
     peaks, peak_src = _peaks()
     clocks = clk.summary()
+    clocks_br = clk_br.summary()
+    clocks["breakdown_sm_mhz"] = clocks_br["sm_mhz"]
+    clocks["breakdown_samples"] = clocks_br.get("samples", 0)
+    clocks["breakdown_reasons"] = clocks_br["reasons"]
     n_sms = torch.cuda.get_device_properties(dev).multi_processor_count
-    clk_mhz = clocks["sm_mhz"] or peaks.get("sm_max_mhz", 1965.0)
+    # the per-call times (ms_search and the others) come from the breakdown
+    # passes: their peaks use the clock sampled over those passes
+    clk_mhz = (clocks_br["sm_mhz"] or clocks["sm_mhz"] or peaks.get("sm_max_mhz", 1965.0))
     hbm = peaks["hbm_gbs"]
     bytes_stats = sum(j.X.numel() * 2 for j in jobs)
     bytes_pack = sum(W.numel() * 2 for j in jobs for W in j.Ws) + \
         sum(t.numel() * t.element_size() for j in jobs for pk in j.packs for t in pk)
+    def hbm_entry(name, nbytes, ms_single):
+        # per-launch time of a stream of back-to-back calls where measured,
+        # else the single-call replay (which carries the graph launch)
+        ms_l = stream_ms.get(name, ms_single)
+        return {"ms": ms_l, "GB/s": nbytes / (ms_l * 1e-3) / 1e9,
+                "hbm_frac": nbytes / (ms_l * 1e-3) / 1e9 / hbm,
+                "ms_single_call": ms_single,
+                "basis": ("average launch of a CUDA graph of back-to-back calls on "
+                          f"{stream_ms.get('copies')} rotating input copies "
+                          f"({stream_ms.get('rot_bytes', 0) / 1e6:.0f} MB in all, > L2); "
+                          "ms_single_call: one call per graph replay, with the graph "
+                          "launch" if name in stream_ms else
+                          "one call per graph replay (graph launch included)")}
     kernels = {
-        "act_stats": {"ms": ms_stats, "GB/s": bytes_stats / (ms_stats * 1e-3) / 1e9,
-                      "hbm_frac": bytes_stats / (ms_stats * 1e-3) / 1e9 / hbm},
-        "quantize_pack": {"ms": ms_pack, "GB/s": bytes_pack / (ms_pack * 1e-3) / 1e9,
-                          "hbm_frac": bytes_pack / (ms_pack * 1e-3) / 1e9 / hbm},
+        "act_stats": hbm_entry("stats", bytes_stats, ms_stats),
+        "quantize_pack": hbm_entry("pack", bytes_pack, ms_pack),
         "hbm_peak_GBs": hbm, "peak_source": peak_src}
     if work.output_mode:
         flops = sum(2.0 * j.X.shape[0] * W.numel() * n_grid for j in jobs for W in j.Ws)
@@ -423,8 +562,20 @@ def run_ours(a):
                 "executed_fma_pipe_ops_per_weight_alpha": FMA_OPS_PER_PAIR,
                 "executed_frac": executed / peak_ops,
                 "peak_basis": f"{n_sms} SMs x {FP32_LANES_PER_SM} FP32 lanes x "
-                              f"{clk_mhz:.0f} MHz (median SM clock sampled in the timed "
-                              f"region)"}
+                              f"{clk_mhz:.0f} MHz (median SM clock sampled over the "
+                              f"per-call passes that time the search)"}
+        probe = fp32_rate_probe(dev)
+        if probe and probe["lane_op_per_clk_per_sm"]:
+            peak_meas = probe["lane_op_per_clk_per_sm"] * n_sms * clk_mhz * 1e6
+            roof["peak_measured"] = peak_meas / 1e12
+            roof["frac_measured"] = achieved / peak_meas
+            roof["executed_frac_measured"] = executed / peak_meas
+            roof["measured_probe"] = {
+                "lane_op_per_clk_per_sm": probe["lane_op_per_clk_per_sm"],
+                "Tlane_op_per_s": {k: v / 1e12 for k, v in probe["lane_op_per_s"].items()},
+                "probe_sm_mhz": probe["sm_mhz"], "probe_clock_samples": probe["samples"],
+                "basis": "FP32 FMA stream (libawq_probe.so, best of scalar / packed / mixed), "
+                         "per SM per clock, scaled to the search passes' clock"}
         if a.clip > 0:
             clip_ops = params * a.clip * ALG_OPS_PER_PAIR
             kernels["clip_search"] = {"ms": ms_clip, "n_clip": a.clip,

@@ -3,7 +3,9 @@
     python -m post_int4_weight_b200.build [--verbose-ptxas]
 
 Each csrc/*.cu is compiled with nvcc for sm_100a only and linked into one
-shared library in the package directory, next to this file.  No fast-math:
+shared library in the package directory, next to this file.  The FP32 rate
+probe (probe/fp32_rate.cu, not part of the library or its C ABI) is built
+into its own small libawq_probe.so for bench.py.  No fast-math:
 the kernels rely on IEEE round-to-nearest-even fp32 division, square root and
 conversions where the method's integer decisions are taken.
 """
@@ -20,6 +22,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libawq_b200.so")
+PROBE_SRC = os.path.join(PKG, "probe", "fp32_rate.cu")
+PROBE_LIB = os.path.join(PKG, "libawq_probe.so")
 BUILD_DIR = os.path.join(PKG, "_build")
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
@@ -39,10 +43,11 @@ def _deps():
 
 
 def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+    if not os.path.exists(LIB) or not os.path.exists(PROBE_LIB):
         return False
     t = os.path.getmtime(LIB)
-    return all(os.path.getmtime(p) <= t for p in _deps())
+    return (all(os.path.getmtime(p) <= t for p in _deps())
+            and os.path.getmtime(PROBE_SRC) <= os.path.getmtime(PROBE_LIB))
 
 
 def build(force: bool = False, verbose_ptxas: bool = False, jobs: int = 8) -> str:
@@ -64,6 +69,10 @@ def build(force: bool = False, verbose_ptxas: bool = False, jobs: int = 8) -> st
     tmp = LIB + ".tmp"
     subprocess.run([NVCC, *ARCH, "-shared", "-o", tmp, *objs], check=True)
     os.replace(tmp, LIB)
+    tmp = PROBE_LIB + ".tmp"
+    subprocess.run([NVCC, *ARCH, "-O3", "-std=c++17", "-Xcompiler", "-fPIC", "-shared",
+                    PROBE_SRC, "-o", tmp], check=True)
+    os.replace(tmp, PROBE_LIB)
     return LIB
 
 

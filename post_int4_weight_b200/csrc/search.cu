@@ -28,11 +28,13 @@
 // range of units: two co-resident CTAs drift apart under the scheduler's
 // age priority and the later one ends alone on its SM.
 //
-// Register-level formulation of one (weight, alpha) pair: 5 FMA-pipe ops and
-// one max.  Packed fp32x2 instructions (sm_100) run on the FMA pipe's heavy
-// half only and scalar ones on either half, so the work is split between the
-// two kinds to keep both halves busy while issuing few instructions.  Each lane holds the
-// same 16 channels of two rows r0, r1:
+// Register-level formulation of one (weight, alpha) pair: 5.5 FMA-pipe lane
+// operations and one max, every FMA-pipe operation a packed fp32x2
+// instruction (sm_100): a packed instruction does two lane operations in one
+// issue slot, and a measured FMA stream reaches the same lane-op rate packed
+// or scalar, so packing leaves issue slots for the maxima, shuffles and
+// shared-memory reads.  Each lane holds the same 16 channels of two rows
+// r0, r1:
 //   ws = w * s                         (exact fp32 product, as the method)
 //   m  = max(m, |ws|)                  (then shuffled across the L lanes)
 //   t  = ws * (1/q_scale) + 1.5*2^23   (rounds to the nearest code, ties even)
@@ -40,7 +42,9 @@
 //   d  = ws - q * q_scale              (= (w - w_hat) * s)
 //   acc += tau2 * (d_r0^2 + d_r1^2),   tau2 = (x / s)^2
 // so that ((w - w_hat) * x)^2 = d^2 * tau2 is summed without forming each
-// product d * tau.  q_scale itself is computed exactly as the method states
+// product d * tau.  The error pass of one alpha is fused with the products
+// and row maxima of the next (rows_errors_next), so the two kinds of work
+// interleave in one instruction stream.  q_scale itself is computed exactly as the method states
 // (IEEE fp32 quotient by 7, fp16 round-to-nearest-even).  The code decision
 // uses the reciprocal of q_scale instead of the IEEE quotient; the two differ
 // only when ws/q_scale lies within an ulp of a half-integer, where either
@@ -230,51 +234,6 @@ __device__ __forceinline__ void rows_scale(float m0, float m1, int lane, float* 
     *rq1 = __shfl_sync(0xffffffffu, r, even | 1);
 }
 
-// Pass 2 of a lane's two rows for one alpha: codes (no clamp when the whole
-// warp's rows are known to stay in range), residuals d = ws - q * q_scale,
-// and sum over the lane's channels of tau2 * (d_r0^2 + d_r1^2).  With kClamp
-// a row whose q_scale is zero or NaN uses a zero reciprocal (all codes 0,
-// d = ws) and its NaN/inf propagates into the sum by itself.
-template <bool kClamp, int L>
-__device__ __forceinline__ float2 rows_errors(const float2* ws0, const float2* ws1,
-                                              const float4* T2, int l, float qs0, float rq0,
-                                              float qs1, float rq1) {
-    if (kClamp && !(qs0 > 0.f)) rq0 = 0.f;
-    if (kClamp && !(qs1 > 0.f)) rq1 = 0.f;
-    const float2 nqs0 = f2(-qs0, -qs0), nqs1 = f2(-qs1, -qs1);
-    const float2 rq02 = f2(rq0, rq0);
-    const float2 magic2 = f2(kRoundMagic, kRoundMagic), nmagic2 = f2(-kRoundMagic, -kRoundMagic);
-    float2 acc2[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        const float4 tv = T2[k * L + l];
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-            const int i = 2 * k + j;
-            // row 0 rounds with packed instructions (the FMA pipe's heavy
-            // half), row 1 with scalar ones (either half): this balance
-            // issued fastest
-            float2 t0 = __ffma2_rn(ws0[i], rq02, magic2);
-            float t1x = __fmaf_rn(ws1[i].x, rq1, kRoundMagic);
-            float t1y = __fmaf_rn(ws1[i].y, rq1, kRoundMagic);
-            if (kClamp) {
-                t0 = f2(fminf(fmaxf(t0.x, kRoundMagic - 7.f), kRoundMagic + 7.f),
-                        fminf(fmaxf(t0.y, kRoundMagic - 7.f), kRoundMagic + 7.f));
-                t1x = fminf(fmaxf(t1x, kRoundMagic - 7.f), kRoundMagic + 7.f);
-                t1y = fminf(fmaxf(t1y, kRoundMagic - 7.f), kRoundMagic + 7.f);
-            }
-            const float2 q0 = __fadd2_rn(t0, nmagic2);
-            const float2 q1 = f2(__fadd_rn(t1x, -kRoundMagic), __fadd_rn(t1y, -kRoundMagic));
-            const float2 d0 = __ffma2_rn(q0, nqs0, ws0[i]);
-            const float2 d1 = __ffma2_rn(q1, nqs1, ws1[i]);
-            float2 sq = __fmul2_rn(d0, d0);
-            sq = __ffma2_rn(d1, d1, sq);
-            acc2[j] = __ffma2_rn(j ? f2(tv.z, tv.w) : f2(tv.x, tv.y), sq, acc2[j]);
-        }
-    }
-    return __fadd2_rn(acc2[0], acc2[1]);
-}
-
 // ---- asymmetric grid (16 levels, per-group zero point)
 // Pass 1: ws = w * s and the lane's largest and smallest ws.
 __device__ __forceinline__ float2 row_products_minmax(const float2* w, const float4* s4,
@@ -331,21 +290,86 @@ __device__ __forceinline__ void rows_scale_asym(float2 mm0, float2 mm1, int lane
     *mz1 = __shfl_sync(0xffffffffu, mz, even | 1);
 }
 
-// Pass 2 on the asymmetric grid: codes clamp(rint(ws / q_scale) + zero, 0, 15)
-// by the rounding addition of 1.5*2^23 + zero (the clamp only when some row
-// of the warp may leave 0..15), then the same weighted sum as rows_errors.
-template <bool kClamp, int L>
-__device__ __forceinline__ float2 rows_errors_asym(const float2* ws0, const float2* ws1,
-                                                   const float4* T2, int l, float qs0,
-                                                   float rq0, float mz0, float qs1, float rq1,
-                                                   float mz1) {
+// The error pass of one alpha fused with the products pass of the next one
+// (software pipelining within the warp, in place): for every element pair
+// the terms of this alpha are taken from ws (as in rows_errors), then ws is
+// overwritten with w * s_next and the running row maxima |ws| (symmetric)
+// or max / min (asymmetric) of the next alpha are updated.  The next
+// alpha's group-scale chain (shuffles, division, reciprocal) therefore runs
+// after a loop that mixes FMA-pipe and ALU work, instead of the ALU-only max
+// tree and the FMA-only error loop running as separate phases in every
+// warp at once.  kNext = false for the last alpha (no next products).
+template <bool kClamp, bool kNext, int L>
+__device__ __forceinline__ float2 rows_errors_next(float2* ws0, float2* ws1, const float2* w0,
+                                                   const float2* w1, const float4* T2,
+                                                   const float4* Sn, int l, float qs0, float rq0,
+                                                   float qs1, float rq1, float* m0, float* m1) {
+    if (kClamp && !(qs0 > 0.f)) rq0 = 0.f;
+    if (kClamp && !(qs1 > 0.f)) rq1 = 0.f;
+    const float2 nqs0 = f2(-qs0, -qs0), nqs1 = f2(-qs1, -qs1);
+    const float2 rq02 = f2(rq0, rq0), rq12 = f2(rq1, rq1);
+    const float2 magic2 = f2(kRoundMagic, kRoundMagic), nmagic2 = f2(-kRoundMagic, -kRoundMagic);
+    float2 acc2[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
+    float mx0[2] = {0.f, 0.f}, mx1[2] = {0.f, 0.f};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const float4 tv = T2[k * L + l];
+        float4 sv;
+        if (kNext) sv = Sn[k * L + l];
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            const int i = 2 * k + j;
+            float2 t0 = __ffma2_rn(ws0[i], rq02, magic2);
+            float2 t1 = __ffma2_rn(ws1[i], rq12, magic2);
+            if (kClamp) {
+                t0 = f2(fminf(fmaxf(t0.x, kRoundMagic - 7.f), kRoundMagic + 7.f),
+                        fminf(fmaxf(t0.y, kRoundMagic - 7.f), kRoundMagic + 7.f));
+                t1 = f2(fminf(fmaxf(t1.x, kRoundMagic - 7.f), kRoundMagic + 7.f),
+                        fminf(fmaxf(t1.y, kRoundMagic - 7.f), kRoundMagic + 7.f));
+            }
+            const float2 q0 = __fadd2_rn(t0, nmagic2);
+            const float2 q1 = __fadd2_rn(t1, nmagic2);
+            const float2 d0 = __ffma2_rn(q0, nqs0, ws0[i]);
+            const float2 d1 = __ffma2_rn(q1, nqs1, ws1[i]);
+            float2 sq = __fmul2_rn(d0, d0);
+            sq = __ffma2_rn(d1, d1, sq);
+            acc2[j] = __ffma2_rn(j ? f2(tv.z, tv.w) : f2(tv.x, tv.y), sq, acc2[j]);
+            if (kNext) {
+                const float2 s2 = j ? f2(sv.z, sv.w) : f2(sv.x, sv.y);
+                ws0[i] = __fmul2_rn(w0[i], s2);
+                ws1[i] = __fmul2_rn(w1[i], s2);
+                mx0[j] = fmaxf(mx0[j], fmaxf(fabsf(ws0[i].x), fabsf(ws0[i].y)));
+                mx1[j] = fmaxf(mx1[j], fmaxf(fabsf(ws1[i].x), fabsf(ws1[i].y)));
+            }
+        }
+    }
+    if (kNext) {
+        *m0 = fmaxf(mx0[0], mx0[1]);
+        *m1 = fmaxf(mx1[0], mx1[1]);
+    }
+    return __fadd2_rn(acc2[0], acc2[1]);
+}
+
+// The asymmetric counterpart: rows_errors_asym for this alpha, then the
+// next alpha's products and their running max and min per row.
+template <bool kClamp, bool kNext, int L>
+__device__ __forceinline__ float2 rows_errors_asym_next(float2* ws0, float2* ws1,
+                                                        const float2* w0, const float2* w1,
+                                                        const float4* T2, const float4* Sn,
+                                                        int l, float qs0, float rq0, float mz0,
+                                                        float qs1, float rq1, float mz1,
+                                                        float2* mm0, float2* mm1) {
     const float2 nqs0 = f2(-qs0, -qs0), nqs1 = f2(-qs1, -qs1);
     const float2 rq02 = f2(rq0, rq0), mz02 = f2(mz0, mz0), nmz02 = f2(-mz0, -mz0);
     constexpr float lo = kRoundMagic, hi = kRoundMagic + 15.f;
     float2 acc2[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
+    float mx0 = __int_as_float(0xff800000), mn0 = __int_as_float(0x7f800000);
+    float mx1 = mx0, mn1 = mn0;
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
         const float4 tv = T2[k * L + l];
+        float4 sv;
+        if (kNext) sv = Sn[k * L + l];
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
             const int i = 2 * k + j;
@@ -364,7 +388,20 @@ __device__ __forceinline__ float2 rows_errors_asym(const float2* ws0, const floa
             float2 sq = __fmul2_rn(d0, d0);
             sq = __ffma2_rn(d1, d1, sq);
             acc2[j] = __ffma2_rn(j ? f2(tv.z, tv.w) : f2(tv.x, tv.y), sq, acc2[j]);
+            if (kNext) {
+                const float2 s2 = j ? f2(sv.z, sv.w) : f2(sv.x, sv.y);
+                ws0[i] = __fmul2_rn(w0[i], s2);
+                ws1[i] = __fmul2_rn(w1[i], s2);
+                mx0 = fmaxf(mx0, fmaxf(ws0[i].x, ws0[i].y));
+                mn0 = fminf(mn0, fminf(ws0[i].x, ws0[i].y));
+                mx1 = fmaxf(mx1, fmaxf(ws1[i].x, ws1[i].y));
+                mn1 = fminf(mn1, fminf(ws1[i].x, ws1[i].y));
+            }
         }
+    }
+    if (kNext) {
+        *mm0 = f2(mx0, mn0);
+        *mm1 = f2(mx1, mn1);
     }
     return __fadd2_rn(acc2[0], acc2[1]);
 }
@@ -528,41 +565,74 @@ search_kernel(const __grid_constant__ SearchParams p) {
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[stage]);
 
-        for (int a = 0; a < p.n_grid; ++a) {
-            const float4* Sa = reinterpret_cast<const float4*>(tab + a * 2 * G);
-            const float4* Ta = reinterpret_cast<const float4*>(tab + a * 2 * G + G);
+        // alpha 0's products and row extremes; then each alpha's group-scale
+        // chain, and its error pass fused with the next alpha's products
+        float2 ws[2][kElemsPerRow / 2];
+        {
+            const float4* S0 = reinterpret_cast<const float4*>(tab);
             float4 s4[4];
 #pragma unroll
-            for (int k = 0; k < 4; ++k) s4[k] = Sa[k * L + l];
-            float2 ws[2][kElemsPerRow / 2];
-            float2 e;
+            for (int k = 0; k < 4; ++k) s4[k] = S0[k * L + l];
             if (kAsym) {
-                const float2 mm0 = row_products_minmax(w[0], s4, ws[0]);
-                const float2 mm1 = row_products_minmax(w[1], s4, ws[1]);
-                float qs0, rq0, mz0, qs1, rq1, mz1;
-                bool in;
-                rows_scale_asym<L, kFp32>(mm0, mm1, lane, &qs0, &rq0, &mz0, &qs1, &rq1, &mz1,
-                                          &in);
-                if (__all_sync(0xffffffffu, in))
-                    e = rows_errors_asym<false, L>(ws[0], ws[1], Ta, l, qs0, rq0, mz0, qs1, rq1,
-                                                   mz1);
-                else   // a row whose extreme codes leave 0..15 (or an infinite ws)
-                    e = rows_errors_asym<true, L>(ws[0], ws[1], Ta, l, qs0, rq0, mz0, qs1, rq1,
-                                                  mz1);
-                acc[a * kThreads + tid] += e.x + e.y;
-                continue;
+                float2 mm0 = row_products_minmax(w[0], s4, ws[0]);
+                float2 mm1 = row_products_minmax(w[1], s4, ws[1]);
+                for (int a = 0; a < p.n_grid; ++a) {
+                    const float4* Ta = reinterpret_cast<const float4*>(tab + a * 2 * G + G);
+                    const float4* Sn = reinterpret_cast<const float4*>(tab + (a + 1) * 2 * G);
+                    float qs0, rq0, mz0, qs1, rq1, mz1;
+                    bool in;
+                    rows_scale_asym<L, kFp32>(mm0, mm1, lane, &qs0, &rq0, &mz0, &qs1, &rq1,
+                                              &mz1, &in);
+                    const bool all_in = __all_sync(0xffffffffu, in);
+                    float2 e;
+                    if (a + 1 < p.n_grid) {
+                        e = all_in ? rows_errors_asym_next<false, true, L>(
+                                         ws[0], ws[1], w[0], w[1], Ta, Sn, l, qs0, rq0, mz0,
+                                         qs1, rq1, mz1, &mm0, &mm1)
+                                   : rows_errors_asym_next<true, true, L>(
+                                         ws[0], ws[1], w[0], w[1], Ta, Sn, l, qs0, rq0, mz0,
+                                         qs1, rq1, mz1, &mm0, &mm1);
+                    } else {
+                        e = all_in ? rows_errors_asym_next<false, false, L>(
+                                         ws[0], ws[1], w[0], w[1], Ta, Sn, l, qs0, rq0, mz0,
+                                         qs1, rq1, mz1, &mm0, &mm1)
+                                   : rows_errors_asym_next<true, false, L>(
+                                         ws[0], ws[1], w[0], w[1], Ta, Sn, l, qs0, rq0, mz0,
+                                         qs1, rq1, mz1, &mm0, &mm1);
+                    }
+                    acc[a * kThreads + tid] += e.x + e.y;
+                }
+            } else {
+                float m0 = row_products(w[0], s4, ws[0]);
+                float m1 = row_products(w[1], s4, ws[1]);
+                for (int a = 0; a < p.n_grid; ++a) {
+                    const float4* Ta = reinterpret_cast<const float4*>(tab + a * 2 * G + G);
+                    const float4* Sn = reinterpret_cast<const float4*>(tab + (a + 1) * 2 * G);
+                    float qs0, rq0, qs1, rq1;
+                    bool in;
+                    rows_scale<L, kFp32>(m0, m1, lane, &qs0, &rq0, &qs1, &rq1, &in);
+                    const bool all_in = __all_sync(0xffffffffu, in);
+                    float2 e;
+                    // some row has an fp16-subnormal, overflowing, zero or NaN
+                    // scale: the clamping variant
+                    if (a + 1 < p.n_grid) {
+                        e = all_in ? rows_errors_next<false, true, L>(ws[0], ws[1], w[0], w[1],
+                                                                      Ta, Sn, l, qs0, rq0, qs1,
+                                                                      rq1, &m0, &m1)
+                                   : rows_errors_next<true, true, L>(ws[0], ws[1], w[0], w[1],
+                                                                     Ta, Sn, l, qs0, rq0, qs1,
+                                                                     rq1, &m0, &m1);
+                    } else {
+                        e = all_in ? rows_errors_next<false, false, L>(ws[0], ws[1], w[0], w[1],
+                                                                       Ta, Sn, l, qs0, rq0, qs1,
+                                                                       rq1, &m0, &m1)
+                                   : rows_errors_next<true, false, L>(ws[0], ws[1], w[0], w[1],
+                                                                      Ta, Sn, l, qs0, rq0, qs1,
+                                                                      rq1, &m0, &m1);
+                    }
+                    acc[a * kThreads + tid] += e.x + e.y;
+                }
             }
-            const float m0 = row_products(w[0], s4, ws[0]);
-            const float m1 = row_products(w[1], s4, ws[1]);
-            float qs0, rq0, qs1, rq1;
-            bool in;
-            rows_scale<L, kFp32>(m0, m1, lane, &qs0, &rq0, &qs1, &rq1, &in);
-            if (__all_sync(0xffffffffu, in)) {
-                e = rows_errors<false, L>(ws[0], ws[1], Ta, l, qs0, rq0, qs1, rq1);
-            } else {   // some row has an fp16-subnormal, overflowing, zero or NaN scale
-                e = rows_errors<true, L>(ws[0], ws[1], Ta, l, qs0, rq0, qs1, rq1);
-            }
-            acc[a * kThreads + tid] += e.x + e.y;
         }
         // every 8 units the per-thread fp32 partials move into the warp's fp64
         // accumulators (fixed order), bounding fp32 accumulation to 8 units

@@ -91,6 +91,20 @@ def test_output_error_down_proj_config_sampled_and_additive():
     np.testing.assert_allclose(err_full, err_a + err_b, rtol=1e-6, atol=0)
 
 
+def test_output_error_down_proj_row_slice_all_tokens():
+    """Realistic dense X at the full config: 128 rows of the 4096 x 12288
+    down_proj scored over all 8192 heavy-tailed tokens and all 12288
+    channels, every grid point against the fp64 oracle on the same slice
+    (x from the full X, as the method takes it)."""
+    work = wl.WORKLOADS["down_proj_output_error"]
+    (grp, Ws, X), = wl.group_inputs(work)
+    W = Ws[0][:128].contiguous()
+    x = oracle.act_stats(X.numpy())
+    err_g, best_g = _run(X, W, x, 128)
+    err_o = oracle.output_error(X.numpy(), W.numpy(), x, 128, 20)
+    _check(err_g, best_g, err_o)
+
+
 def test_output_error_fp32_scale_and_nonfinite():
     W = wl.weight(64, 256, 77)
     X = wl.activations(32, 256, 78)
