@@ -360,7 +360,8 @@ awq_status awq_clip_search(const void *W, int64_t d_out, int64_t d_in,
  *
  *   err[i] = || X (W - W_hat_i)^T ||_F^2,   W_hat_i = Q(W * s_i) / s_i
  *
- * with s_i and Q exactly as in awq_scale_search.  The contraction runs on
+ * with s_i and Q exactly as in awq_scale_search (symmetric, or the
+ * asymmetric grid with AWQ_ASYMMETRIC).  The contraction runs on
  * the tensor cores with fp16 operands and fp32 accumulation.  W - W_hat_i
  * is formed exactly in fp32, scaled per row by a power of two, and split
  * into two fp16 parts hi + lo (lo = the rounding error of hi), so that the
@@ -375,7 +376,10 @@ awq_status awq_clip_search(const void *W, int64_t d_out, int64_t d_in,
  *   W           fp16 [d_out, d_in] device; d_out % 8 == 0
  *   x_mean      fp32 [d_in] device (defines s_i)
  *   group_size  32, 64 or 128;  d_in multiple of group_size and of 64
- *   n_grid      1..32;  flags as in awq_scale_search
+ *   n_grid      1..32
+ *   flags       AWQ_SCALE_FP16 or AWQ_SCALE_FP32, optionally | AWQ_ASYMMETRIC
+ *               (W_hat from the asymmetric grid of awq_scale_search; pack the
+ *               chosen scale with AWQ_ZERO_POINT_ASYM)
  *   err         fp64 [n_grid] device output (NaN for every i if W holds a
  *               non-finite value)
  *   best_idx    int32 [1] device output (first minimum; -1 if non-finite,

@@ -614,8 +614,10 @@ void orc_unpack(const int32_t *qweight, int64_t d_out, int64_t d_in,
  * compared with the full-precision output; [P4] section 2: the output error
  * is X (W - W_hat)):
  *     err[i] = || X (W - W_hat_i)^T ||_F^2
- * with W_hat_i = Q(W * s_i) / s_i from the same group fake-quantisation, in
- * fp64.  X is fp16 [T, d_in] row-major, W fp16 [d_out, d_in].
+ * with W_hat_i = Q(W * s_i) / s_i from the same group fake-quantisation
+ * (the asymmetric grid of orc_fake_quant_group_asym with ORC_ASYM in flags:
+ * W_hat = (q - zero) q_scale / s), in fp64.  X is fp16 [T, d_in] row-major,
+ * W fp16 [d_out, d_in].
  */
 void orc_output_error(const uint16_t *X, int64_t T, const uint16_t *W,
                       int64_t d_out, int64_t d_in, const float *x, int64_t g,
@@ -636,14 +638,21 @@ void orc_output_error(const uint16_t *X, int64_t T, const uint16_t *W,
         for (int64_t r = 0; r < d_out; ++r) {
             float w[g];
             int8_t q[g];
+            uint8_t u[g];
             bad_row[r] = 0;
             for (int64_t k = 0; k < d_in / g; ++k) {
                 for (int64_t j = 0; j < g; ++j) w[j] = h2f(W[r * d_in + k * g + j]);
                 float qs;
-                if (orc_fake_quant_group(w, s + k * g, g, flags, q, &qs)) bad_row[r] = 1;
-                for (int64_t j = 0; j < g; ++j)
+                int z = 0;
+                int bad = (flags & ORC_ASYM)
+                              ? orc_fake_quant_group_asym(w, s + k * g, g, flags, u, &qs, &z)
+                              : orc_fake_quant_group(w, s + k * g, g, flags, q, &qs);
+                if (bad) bad_row[r] = 1;
+                for (int64_t j = 0; j < g; ++j) {
+                    double level = (flags & ORC_ASYM) ? (double)((int)u[j] - z) : (double)q[j];
                     dW[r * d_in + k * g + j] =
-                        (double)w[j] - (double)q[j] * (double)qs / (double)s[k * g + j];
+                        (double)w[j] - level * (double)qs / (double)s[k * g + j];
+                }
             }
         }
         /* ||X dW^T||^2: one partial per token, summed in token order */

@@ -246,7 +246,7 @@ awq_status awq_output_error(const void* X, int64_t T, const void* W, int64_t d_o
     if (!X || !W || !x_mean || !err || !best_idx) return AWQ_ERR_INVALID_ARG;
     if (!valid_group(group_size)) return AWQ_ERR_UNSUPPORTED;
     if (n_grid < 1 || n_grid > 32) return AWQ_ERR_INVALID_ARG;
-    if (flags != AWQ_SCALE_FP16 && flags != AWQ_SCALE_FP32) return AWQ_ERR_INVALID_ARG;
+    if (flags & ~(AWQ_SCALE_FP32 | AWQ_ASYMMETRIC)) return AWQ_ERR_INVALID_ARG;
     if (T < 1 || T > (int64_t(1) << 24)) return AWQ_ERR_INVALID_ARG;
     if (d_out < 8 || d_out % 8 || d_out > (int64_t(1) << 24)) return AWQ_ERR_INVALID_ARG;
     if (d_in < group_size || d_in % group_size || d_in % 64 || d_in > (int64_t(1) << 20))

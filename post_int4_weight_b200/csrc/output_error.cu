@@ -18,11 +18,19 @@
 //                      of the product is [dW_hi | dW_lo] against [X | X], so
 //                      the tensor cores see dW to ~22 bits, not 11;
 //   oe_gemm_kernel     persistent, one CTA per SM, 18 warps: warp 0 issues
-//                      TMA loads (128B-swizzled 128x64 tiles of X and 256x64
-//                      tiles of dW) into a 4-stage mbarrier ring; one thread
-//                      of warp 1 issues tcgen05.mma (kind::f16, M=128, N=256,
-//                      K=16, fp32 accumulation in TMEM) and commits each stage
-//                      back to the producer.  TMEM holds the MMA accumulator
+//                      TMA loads into a 5-stage mbarrier ring; a stage holds
+//                      one 128x32 tile of X and the matching 256x32 tiles of
+//                      dW hi and dW lo (64-byte swizzle), so every X tile
+//                      feeds both halves and X crosses DRAM once per tile;
+//                      one thread of warp 1 issues tcgen05.mma (kind::f16,
+//                      M=128, N=256, K=16, fp32 accumulation in TMEM), four
+//                      per stage (two K slices x hi, lo), and commits each
+//                      stage back to the producer.  Output tiles go in
+//                      groups of 8 row blocks of dW: all token blocks sweep
+//                      one group before the next starts, the group's dW
+//                      tiles (100 MB at 4096 x 12288) are read with an L2
+//                      evict-last policy and X with evict-first, so dW
+//                      crosses DRAM once per grid point and X once per group.  TMEM holds the MMA accumulator
 //                      (columns 0-255) and a running sum (256-511).  Every 32
 //                      K-blocks (2048 of K) warps 2-17 (four per TMEM lane
 //                      quadrant, 64 columns each) drain the accumulator into
@@ -48,17 +56,18 @@ namespace {
 // ----------------------------------------------------------- tile shape
 constexpr int kBM = 128;                    // tokens per tile (TMEM lanes)
 constexpr int kBN = 256;                    // output rows per tile (TMEM columns)
-constexpr int kBK = 64;                     // 64 fp16 = 128 bytes: one swizzle row
+constexpr int kBK = 32;                     // 32 fp16 = 64 bytes: one swizzle row
 constexpr int kUmmaK = 16;                  // K of one kind::f16 MMA
-constexpr int kStages = 4;
-constexpr int kABytes = kBM * kBK * 2;      // 16 KB
-constexpr int kBBytes = kBN * kBK * 2;      // 32 KB
-constexpr int kStageBytes = kABytes + kBBytes;
+constexpr int kStages = 5;
+constexpr int kABytes = kBM * kBK * 2;      // 8 KB of X
+constexpr int kBBytes = kBN * kBK * 2;      // 16 KB of dW hi (and as much of dW lo)
+constexpr int kStageBytes = kABytes + 2 * kBBytes;   // 40 KB
+constexpr int kGroupN = 8;                  // dW row blocks per raster group
 constexpr int kTmemCols = 2 * kBN;          // accumulator + running sum
 constexpr int kEpiWarps = 16;               // four per TMEM lane quadrant
 constexpr int kEpiCols = kBN / (kEpiWarps / 4);   // accumulator columns per epilogue warp
 constexpr int kGemmThreads = 32 * (2 + kEpiWarps);   // producer, MMA, epilogue
-constexpr int kSegBlocks = 32;              // K-blocks accumulated per drain
+constexpr int kSegBlocks = 32;              // K-blocks (x 4 MMAs) accumulated per drain
 constexpr int kMaxOeCtas = 1024;
 constexpr int kMaxGridOe = 32;
 
@@ -68,17 +77,31 @@ constexpr uint32_t kIdesc = (1u << 4) | ((uint32_t)(kBN >> 3) << 17) |
                             ((uint32_t)(kBM >> 4) << 24);
 
 // Shared-memory matrix descriptor of a K-major tile written by TMA with the
-// 128-byte swizzle: start address >> 4 (bits 0-13), leading byte offset
-// (unused for this layout; 1), stride byte offset = 1024 bytes between
-// 8-row groups (bits 32-45), descriptor version 1 (bits 46-47), layout
-// 128B-swizzle = 2 (bits 61-63).
+// 64-byte swizzle (rows of 64 bytes, 16-byte chunks XOR-permuted within each
+// 4-chunk row by the row's bits): start address >> 4 (bits 0-13), leading
+// byte offset (unused for this layout; 1), stride byte offset = 512 bytes
+// between 8-row groups (bits 32-45), descriptor version 1 (bits 46-47),
+// layout 64B-swizzle = 4 (bits 61-63).  The second K=16 slice of a row
+// starts 32 bytes further (the swizzle is applied to the final address).
 __device__ __forceinline__ uint64_t smem_desc(uint32_t addr) {
     uint64_t d = (uint64_t)((addr >> 4) & 0x3FFFu);
     d |= (uint64_t)1u << 16;
-    d |= (uint64_t)(1024u >> 4) << 32;
+    d |= (uint64_t)(512u >> 4) << 32;
     d |= (uint64_t)1u << 46;
-    d |= (uint64_t)2u << 61;
+    d |= (uint64_t)4u << 61;
     return d;
+}
+
+// Output tile t of the raster: groups of kGroupN dW row blocks; within a
+// group the token block advances slowest, so the CTAs working at one time
+// share the group's dW tiles and each X tile.
+__device__ __forceinline__ void tile_mn(int t, int m_blocks, int n_blocks, int* m, int* n) {
+    const int per_group = kGroupN * m_blocks;
+    const int g = t / per_group;
+    const int local = t - g * per_group;
+    const int ng = min(kGroupN, n_blocks - g * kGroupN);
+    *m = local / ng;
+    *n = g * kGroupN + local % ng;
 }
 
 __device__ __forceinline__ void umma_f16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
@@ -138,9 +161,10 @@ __device__ __forceinline__ void tmem_wait_st() {
 }
 
 struct GemmParams {
-    CUtensorMap tmA;        // X  fp16 [T, d_in], box {64, 128}, 128B swizzle
-    CUtensorMap tmB;        // dW fp16 [d_out, 2 d_in] (hi | lo), box {64, 256}, 128B swizzle
-    int32_t m_blocks, n_blocks, k_blocks;   // k_blocks of X (dW has twice as many)
+    CUtensorMap tmA;        // X  fp16 [T, d_in], box {32, 128}, 64B swizzle
+    CUtensorMap tmB;        // dW fp16 [d_out, 2 d_in] (hi | lo), box {32, 256}, 64B swizzle
+    int32_t m_blocks, n_blocks, k_blocks;   // k_blocks of X (and of each dW half)
+    int32_t d_in;
     int32_t alpha, n_grid;
     int64_t d_out;
     const float* inv_c;     // [d_out] 1 / c_r of this grid point
@@ -207,19 +231,23 @@ oe_gemm_kernel(const __grid_constant__ GemmParams p) {
     if (warp == 0) {
         // ---------------------------------------------------- TMA producer
         if (lane == 0) {
+            const uint64_t pol_x = l2_policy_evict_first(), pol_dw = l2_policy_evict_last();
             uint32_t it = 0;
             uint32_t issued[kStages] = {};
             for (int t = blockIdx.x; t < n_tiles && !*abort_flag; t += gridDim.x) {
-                const int n_blk = t / p.m_blocks, m_blk = t % p.m_blocks;
-                for (int kb = 0; kb < 2 * p.k_blocks; ++kb, ++it) {
+                int m_blk, n_blk;
+                tile_mn(t, p.m_blocks, p.n_blocks, &m_blk, &n_blk);
+                for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
                     const int s = it % kStages;
                     const uint32_t use = it / kStages;
                     if (use > 0 && !wait_or_abort(&empty[s], (use - 1) & 1u, abort_flag, p.dev_err))
                         break;
                     unsigned char* a = stages + s * kStageBytes;
                     mbar_arrive_expect_tx(&full[s], kStageBytes);
-                    tma_load_2d(a, &p.tmA, (kb % p.k_blocks) * kBK, m_blk * kBM, &full[s]);
-                    tma_load_2d(a + kABytes, &p.tmB, kb * kBK, n_blk * kBN, &full[s]);
+                    tma_load_2d_hint(a, &p.tmA, kb * kBK, m_blk * kBM, &full[s], pol_x);
+                    tma_load_2d_hint(a + kABytes, &p.tmB, kb * kBK, n_blk * kBN, &full[s], pol_dw);
+                    tma_load_2d_hint(a + kABytes + kBBytes, &p.tmB, p.d_in + kb * kBK, n_blk * kBN,
+                                     &full[s], pol_dw);
                     ++issued[s];
                 }
             }
@@ -233,7 +261,7 @@ oe_gemm_kernel(const __grid_constant__ GemmParams p) {
         // ---------------------------------------------------- MMA issuer
         if (lane == 0) {
             uint32_t it = 0, seg = 0;
-            const int kb_total = 2 * p.k_blocks;
+            const int kb_total = p.k_blocks;
             for (int t = blockIdx.x; t < n_tiles && !*abort_flag; t += gridDim.x) {
                 bool ok = true;
                 for (int kb0 = 0; kb0 < kb_total && ok; kb0 += kSegBlocks, ++seg) {
@@ -254,11 +282,15 @@ oe_gemm_kernel(const __grid_constant__ GemmParams p) {
                         }
                         tc_fence_after();
                         const uint32_t a = smem_addr(stages + s * kStageBytes);
+                        const uint32_t bh = a + kABytes, bl = bh + kBBytes;
 #pragma unroll
                         for (int k = 0; k < kBK / kUmmaK; ++k) {
+                            // X times dW hi, then the same X times dW lo
                             umma_f16(tmem_base, smem_desc(a + k * kUmmaK * 2),
-                                     smem_desc(a + kABytes + k * kUmmaK * 2),
+                                     smem_desc(bh + k * kUmmaK * 2),
                                      (kb > kb0 || k > 0) ? 1u : 0u);
+                            umma_f16(tmem_base, smem_desc(a + k * kUmmaK * 2),
+                                     smem_desc(bl + k * kUmmaK * 2), 1u);
                         }
                         umma_commit(&empty[s]);   // stage free once these MMAs are done
                     }
@@ -275,7 +307,7 @@ oe_gemm_kernel(const __grid_constant__ GemmParams p) {
         // ---------------------------------------------------- epilogue
         const int q = warp & 3;                 // TMEM lane quadrant of this warp
         const int h = (warp - 2) / 4;           // which kEpiCols-wide slice of the columns
-        const int kb_total = 2 * p.k_blocks;
+        const int kb_total = p.k_blocks;
         const int segs = (kb_total + kSegBlocks - 1) / kSegBlocks;
         const uint32_t lane_base = (uint32_t)(q * 32) << 16;
         const uint32_t acc_addr = tmem_base + lane_base + (uint32_t)(h * kEpiCols);
@@ -314,7 +346,9 @@ oe_gemm_kernel(const __grid_constant__ GemmParams p) {
             }
             if (!ok) break;
             // the running sum holds this tile's slice of X dW^T
-            const int64_t n0 = (int64_t)(t / p.m_blocks) * kBN + h * kEpiCols;
+            int m_blk, n_blk;
+            tile_mn(t, p.m_blocks, p.n_blocks, &m_blk, &n_blk);
+            const int64_t n0 = (int64_t)n_blk * kBN + h * kEpiCols;
             float s0 = 0.f, s1 = 0.f;
 #pragma unroll 1
             for (int c0 = 0; c0 < kEpiCols; c0 += 16) {
@@ -357,8 +391,20 @@ __device__ __forceinline__ float seg_max(float v) {
     for (int o = 1; o < G / 8; o <<= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
     return v;
 }
-
 template <int G>
+__device__ __forceinline__ float seg_min(float v) {
+#pragma unroll
+    for (int o = 1; o < G / 8; o <<= 1) v = fminf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+// kAsym: the asymmetric grid (AWQ_ASYMMETRIC), as the search and the pack
+// take it: range = max(max ws - min ws, 1e-5), q_scale = fp16(range / 15),
+// zero = clamp(rint(-min ws / q_scale), 0, 15), q = clamp(rint(ws / q_scale)
+// + zero, 0, 15) with exact quotients, and W - W_hat = (ws - (q - zero)
+// q_scale) / s.  |ws - (q - zero) q_scale| <= 3 max |ws| as in the symmetric
+// grid, so the row bound of pass 1 holds for both.
+template <int G, bool kAsym>
 __global__ void __launch_bounds__(256)
 dw_builder_kernel(const uint4* __restrict__ W, int64_t d_out, int64_t d_in,
                   const float* __restrict__ S, const float* __restrict__ inv_s,
@@ -426,10 +472,28 @@ dw_builder_kernel(const uint4* __restrict__ W, int64_t d_out, int64_t d_in,
             ws[2 * i + 1] = __fmul_rn(w.y, sv[2 * i + 1]);
             m = fmaxf(m, fmaxf(fabsf(ws[2 * i]), fabsf(ws[2 * i + 1])));
         }
-        m = seg_max<G>(m);
-        bool in_range;
-        const float qs = group_scale(m, fp32_scale != 0, &in_range);
-        const float rq = (qs > 0.f) ? __frcp_rn(qs) : 0.f;
+        float qs, rq, zf = 0.f;
+        if (kAsym) {
+            float mx = ws[0], mn = ws[0];
+#pragma unroll
+            for (int i = 1; i < 8; ++i) {
+                mx = fmaxf(mx, ws[i]);
+                mn = fminf(mn, ws[i]);
+            }
+            mx = seg_max<G>(mx);
+            mn = seg_min<G>(mn);
+            const float range = fmaxf(__fsub_rn(mx, mn), 1e-5f);
+            qs = div15_rn(range);
+            if (!fp32_scale) qs = fminf(__half2float(__float2half_rn(qs)), kHalfMax);
+            rq = __frcp_rn(qs);
+            zf = fminf(fmaxf(rintf(div_rn_rcp(-mn, qs, rq)), 0.f), 15.f);
+            // a NaN or infinite ws makes its own d, and so the error, non-finite
+        } else {
+            m = seg_max<G>(m);
+            bool in_range;
+            qs = group_scale(m, fp32_scale != 0, &in_range);
+            rq = (qs > 0.f) ? __frcp_rn(qs) : 0.f;
+        }
         uint32_t out[4], out_lo[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -437,10 +501,17 @@ dw_builder_kernel(const uint4* __restrict__ W, int64_t d_out, int64_t d_in,
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 const float a = ws[2 * i + h];
-                const float y = (qs > 0.f) ? div_rn_rcp(a, qs, rq) : 0.f;
-                float t = __fadd_rn(y, kRoundMagic);
-                t = fminf(fmaxf(t, kRoundMagic - 7.f), kRoundMagic + 7.f);
-                const float q = __fadd_rn(t, -kRoundMagic);
+                float q;
+                if (kAsym) {
+                    float t = __fadd_rn(__fadd_rn(div_rn_rcp(a, qs, rq), kRoundMagic), zf);
+                    t = fminf(fmaxf(t, kRoundMagic), kRoundMagic + 15.f);
+                    q = __fsub_rn(__fadd_rn(t, -kRoundMagic), zf);   // level q - zero
+                } else {
+                    const float y = (qs > 0.f) ? div_rn_rcp(a, qs, rq) : 0.f;
+                    float t = __fadd_rn(y, kRoundMagic);
+                    t = fminf(fmaxf(t, kRoundMagic - 7.f), kRoundMagic + 7.f);
+                    q = __fadd_rn(t, -kRoundMagic);
+                }
                 const float d = __fmaf_rn(-q, qs, a);          // (w - w_hat) * s
                 d2[h] = __fmul_rn(__fmul_rn(d, iv[2 * i + h]), c);
             }
@@ -492,7 +563,9 @@ cudaError_t launch_builder(const void* W, int64_t d_out, int64_t d_in, const flo
                            const float* inv_s, int flags, __half* dW, float* inv_c,
                            cudaStream_t st) {
     const dim3 grid((unsigned)((d_out + 7) / 8));
-    return launch_pdl(dw_builder_kernel<G>, grid, dim3(256), 0, st,
+    return launch_pdl((flags & AWQ_ASYMMETRIC) ? dw_builder_kernel<G, true>
+                                               : dw_builder_kernel<G, false>,
+                      grid, dim3(256), 0, st,
                       static_cast<const uint4*>(W), d_out, d_in, S, inv_s,
                       (int)((flags & AWQ_SCALE_FP32) != 0), dW, inv_c);
 }
@@ -527,7 +600,7 @@ awq_status launch_output_error(const void* X, int64_t T, const void* W, int64_t 
         const cuuint32_t es[2] = {1, 1};
         if (encode(&p.tmA, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(X), gdim,
                    gstride, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return AWQ_ERR_CUDA;
     }
@@ -537,7 +610,7 @@ awq_status launch_output_error(const void* X, int64_t T, const void* W, int64_t 
         const cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)kBN};
         const cuuint32_t es[2] = {1, 1};
         if (encode(&p.tmB, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, w.dW, gdim, gstride, box, es,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return AWQ_ERR_CUDA;
@@ -545,6 +618,7 @@ awq_status launch_output_error(const void* X, int64_t T, const void* W, int64_t 
     p.m_blocks = (int32_t)((T + kBM - 1) / kBM);
     p.n_blocks = (int32_t)((d_out + kBN - 1) / kBN);
     p.k_blocks = (int32_t)(d_in / kBK);
+    p.d_in = (int32_t)d_in;
     p.n_grid = n_grid;
     p.d_out = d_out;
     p.inv_c = w.inv_c;

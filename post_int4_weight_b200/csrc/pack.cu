@@ -90,6 +90,50 @@ __device__ __forceinline__ int s_slot(int j) { return j + 4 * (j >> 6); }
 // Byte offset of 16-byte chunk c (0..7) of row r in a 128-byte-swizzled box.
 __device__ __forceinline__ int swz(int r, int c) { return r * 128 + ((c ^ (r & 7)) << 4); }
 
+// Codes of one lane's 4 columns over the warp's 16 rows, packed into two
+// words per column.  kSlow: clamp the codes (and store the zero point for a
+// non-finite group); taken per lane outside the row loop, so the loop itself
+// has no branch.
+template <bool kSlow, bool kAsym>
+__device__ __forceinline__ void pack_rows(const unsigned char* box, int chunk, float2 s01,
+                                          float2 s23, const float2* qr_row, const int* bad_row,
+                                          const int* zero_row, uint32_t words[4][2]) {
+    const float2 magic2 = make_float2(kRoundMagic, kRoundMagic);
+#pragma unroll
+    for (int i = 0; i < kRowsPerWarp; ++i) {
+        // row rb + i: (rb + i) & 7 == i & 7, so the swizzle is a constant
+        const uint2 v = *reinterpret_cast<const uint2*>(box + i * 128 + ((chunk ^ (i & 7)) << 4));
+        const float2 qr = qr_row[i];           // (q_scale, 1 / q_scale)
+        const float2 nb2 = make_float2(-qr.x, -qr.x), y2 = make_float2(qr.y, qr.y);
+        const float2 w01 = __half22float2(*reinterpret_cast<const __half2*>(&v.x));
+        const float2 w23 = __half22float2(*reinterpret_cast<const __half2*>(&v.y));
+        // w s / q_scale with one residual correction of w s * RN(1 / q_scale):
+        // its rounding decision is the IEEE quotient's (see quot_rcp1_2)
+        float2 t01 = __fadd2_rn(quot_rcp1_2(__fmul2_rn(w01, s01), nb2, y2), magic2);
+        float2 t23 = __fadd2_rn(quot_rcp1_2(__fmul2_rn(w23, s23), nb2, y2), magic2);
+        if (kSlow) {
+            float lo = kRoundMagic - 7.f, hi = kRoundMagic + 7.f;
+            if (kAsym) {
+                const float z = (float)zero_row[i];
+                lo = kRoundMagic - z;
+                hi = kRoundMagic + 15.f - z;
+            }
+            t01 = make_float2(fminf(fmaxf(t01.x, lo), hi), fminf(fmaxf(t01.y, lo), hi));
+            t23 = make_float2(fminf(fmaxf(t23.x, lo), hi), fminf(fmaxf(t23.y, lo), hi));
+            if (bad_row[i]) {   // code = zero point
+                t01 = magic2;
+                t23 = magic2;
+            }
+        }
+        const uint32_t shift = 1u << (4 * nibble_of_row(i & 7));
+        const int hw = i >> 3;
+        words[0][hw] += __float_as_uint(t01.x) * shift;
+        words[1][hw] += __float_as_uint(t01.y) * shift;
+        words[2][hw] += __float_as_uint(t23.x) * shift;
+        words[3][hw] += __float_as_uint(t23.y) * shift;
+    }
+}
+
 template <int G, bool kAsym>
 __global__ void __launch_bounds__(kPackThreads, kPackCtasPerSm)
 pack_kernel(const __grid_constant__ PackParams p) {
@@ -270,7 +314,6 @@ pack_kernel(const __grid_constant__ PackParams p) {
         const float2* qr_row = qr_tile + kk * kRowStride + rb;
         const int* bad_row = bad_tile + kk * kRowStride + rb;
         const int* zero_row = zero_tile + kk * kRowStride + rb;
-        const float2 magic2 = make_float2(kRoundMagic, kRoundMagic);
         // each nibble starts at (zero point - bits of 1.5*2^23); adding the
         // bits of the rounded quotient + 1.5*2^23 leaves the unsigned code
         uint32_t words[4][2];
@@ -282,41 +325,10 @@ pack_kernel(const __grid_constant__ PackParams p) {
 #pragma unroll
             for (int e = 0; e < 4; ++e) words[e][hw] = init;
         }
-        const bool slow = kAsym || slow_blk[kk * kBlocks + warp] != 0;
-#pragma unroll
-        for (int i = 0; i < kRowsPerWarp; ++i) {
-            // row rb + i: (rb + i) & 7 == i & 7, so the swizzle is a constant
-            const uint2 v = *reinterpret_cast<const uint2*>(box + i * 128 +
-                                                            ((chunk ^ (i & 7)) << 4));
-            const float2 qr = qr_row[i];           // (q_scale, 1 / q_scale)
-            const float2 nb2 = make_float2(-qr.x, -qr.x), y2 = make_float2(qr.y, qr.y);
-            const float2 w01 = __half22float2(*reinterpret_cast<const __half2*>(&v.x));
-            const float2 w23 = __half22float2(*reinterpret_cast<const __half2*>(&v.y));
-            // w s / q_scale with one residual correction of w s * RN(1 / q_scale):
-            // its rounding decision is the IEEE quotient's (see quot_rcp1_2)
-            float2 t01 = __fadd2_rn(quot_rcp1_2(__fmul2_rn(w01, s01), nb2, y2), magic2);
-            float2 t23 = __fadd2_rn(quot_rcp1_2(__fmul2_rn(w23, s23), nb2, y2), magic2);
-            if (slow) {
-                float lo = kRoundMagic - 7.f, hi = kRoundMagic + 7.f;
-                if (kAsym) {
-                    const float z = (float)zero_row[i];
-                    lo = kRoundMagic - z;
-                    hi = kRoundMagic + 15.f - z;
-                }
-                t01 = make_float2(fminf(fmaxf(t01.x, lo), hi), fminf(fmaxf(t01.y, lo), hi));
-                t23 = make_float2(fminf(fmaxf(t23.x, lo), hi), fminf(fmaxf(t23.y, lo), hi));
-                if (bad_row[i]) {   // code = zero point
-                    t01 = magic2;
-                    t23 = magic2;
-                }
-            }
-            const uint32_t shift = 1u << (4 * nibble_of_row(i & 7));
-            const int hw = i >> 3;
-            words[0][hw] += __float_as_uint(t01.x) * shift;
-            words[1][hw] += __float_as_uint(t01.y) * shift;
-            words[2][hw] += __float_as_uint(t23.x) * shift;
-            words[3][hw] += __float_as_uint(t23.y) * shift;
-        }
+        if (kAsym || slow_blk[kk * kBlocks + warp] != 0)
+            pack_rows<true, kAsym>(box, chunk, s01, s23, qr_row, bad_row, zero_row, words);
+        else
+            pack_rows<false, kAsym>(box, chunk, s01, s23, qr_row, bad_row, zero_row, words);
         const int64_t cw = row0 / 8 + rb / 8;      // first output word of the warp
         if (cw < C) {   // d_out % 8 == 0: each word is wholly inside or outside
             const bool two = cw + 1 < C;

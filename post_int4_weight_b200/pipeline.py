@@ -158,7 +158,8 @@ class GroupJob:
             return
         out = (self.err, self.best, self.s_best)
         if self.output_mode:
-            awq.output_error(self.X, self.Ws[0], self.x, self.g, self.n_grid, out=out, ws=ws)
+            awq.output_error(self.X, self.Ws[0], self.x, self.g, self.n_grid,
+                             self.flags & awq.ASYMMETRIC, out=out, ws=ws)
         else:
             awq.scale_search(self.Ws, self.x, self.g, self.n_grid, self.flags, out=out, ws=ws)
 

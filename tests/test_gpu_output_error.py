@@ -117,6 +117,24 @@ def test_output_error_fp32_scale_and_nonfinite():
     assert best_g == -1 and np.isnan(err_g).all()
 
 
+@pytest.mark.parametrize("T,d_out,d_in,g", [(64, 256, 512, 128), (100, 264, 640, 64),
+                                            (256, 512, 1024, 32)])
+def test_output_error_asym(T, d_out, d_in, g):
+    """The asymmetric grid (AWQ_ASYMMETRIC) in output space against the fp64
+    oracle; s_best is the plain scale-table row (the grid does not change the
+    candidates)."""
+    seed = 3 * T + d_out + d_in + g
+    W = wl.weight(d_out, d_in, seed + 1)
+    X = wl.activations(T, d_in, seed)
+    x = oracle.act_stats(X.numpy())
+    err_g, best_g = _run(X, W, x, g, 20, awq.ASYMMETRIC)
+    err_o = oracle.output_error(X.numpy(), W.numpy(), x, g, 20, oracle.ASYM)
+    _check(err_g, best_g, err_o)
+    W[3, 17] = float("nan")
+    err_g, best_g = _run(X, W, x, g, 20, awq.ASYMMETRIC)
+    assert best_g == -1 and not np.isfinite(err_g).any()
+
+
 @pytest.mark.parametrize("n_grid", [1, 32])
 def test_output_error_grid_sizes(n_grid):
     W = wl.weight(64, 256, 31 + n_grid)

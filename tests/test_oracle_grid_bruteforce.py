@@ -223,3 +223,47 @@ def test_worked_example_grid(fp32_scale):
     else:
         np.testing.assert_allclose(plateau, dropped, rtol=1e-3)
     assert err[13] < dropped / 1.4            # alpha = 0.65 still keeps a code
+
+
+# ------------------------------------------------------------ output space --
+# "AWQ architecture, in depth", section "The scale search as code" (the
+# group's output after fake quantisation against the full-precision output);
+# "Weight-Only Quantization: GPTQ and AWQ", section 2 (the output error is
+# X (W - W_hat)).  err[i] = ||X (W - W_hat_i)^T||_F^2, recomputed here as a
+# plain fp64 matrix product from the brute-force W_hat_i above.
+
+@pytest.mark.parametrize("asym", [False, True], ids=["sym", "asym"])
+@pytest.mark.parametrize("fp32_scale", [False, True], ids=["fp16scale", "fp32scale"])
+def test_output_error_grid_bruteforce(asym, fp32_scale):
+    rng = np.random.default_rng(77)
+    T, d_out, d_in, g, n_grid = 12, 8, 96, 32, 20
+    W = (rng.standard_normal((d_out, d_in)) * 0.02).astype(np.float16)
+    X = (rng.standard_normal((T, d_in)) * np.exp(rng.standard_normal(d_in))).astype(np.float16)
+    x = np.abs(X.astype(np.float64)).mean(axis=0).astype(F32)
+    S = _table_plain(x, n_grid)
+    Xd = X.astype(np.float64)
+    ref = []
+    for s in S:
+        w = W.astype(F32)
+        what = np.concatenate(
+            [_group_dequant(w[:, k * g:(k + 1) * g], np.broadcast_to(s[k * g:(k + 1) * g], (d_out, g)),
+                            asym, fp32_scale) for k in range(d_in // g)], axis=1)
+        y = Xd @ (W.astype(np.float64) - what).T
+        ref.append(float((y * y).sum()))
+    flags = (oracle.ASYM if asym else 0) | (oracle.SCALE_FP32 if fp32_scale else 0)
+    err = oracle.output_error(X, W, x, g, n_grid, flags)
+    np.testing.assert_allclose(err, ref, rtol=1e-12, atol=0)
+
+
+def test_output_error_asym_diagonal_x_is_weight_space():
+    """X = diag(c): the asymmetric output-space score equals the asymmetric
+    weight-space score with x = c."""
+    rng = np.random.default_rng(43)
+    d_out, d_in, g = 16, 64, 32
+    W = (rng.standard_normal((d_out, d_in)) * 0.02).astype(np.float16)
+    c = np.exp(rng.standard_normal(d_in)).astype(np.float16)
+    X = np.diag(c.astype(np.float32)).astype(np.float16)
+    x = c.astype(F32)
+    eo = oracle.output_error(X, W, x, g, 20, oracle.ASYM)
+    ew, _, _ = oracle.scale_search([W], x, g, 20, oracle.ASYM)
+    np.testing.assert_allclose(eo, ew, rtol=1e-12)
