@@ -52,6 +52,7 @@ def _load():
         lib.orc_clip_group_error.argtypes = [p, p, p, i64, i32, ctypes.c_float]
         lib.orc_clip_group_error.restype = f64
         lib.orc_clip_search.argtypes = [p, i64, i64, p, p, i64, i32, i32, p, p]
+        lib.orc_clip_search_output.argtypes = [p, i64, p, i64, i64, p, i64, i32, i32, p, p]
         lib.orc_unpack.argtypes = [p, i64, i64, p]
         lib.orc_output_error.argtypes = [p, i64, p, i64, i64, p, i64, i32, i32, p]
         _lib = lib
@@ -223,6 +224,24 @@ def clip_search(W, x, s=None, group_size: int = 128, n_clip: int = 10, flags: in
     _load().orc_clip_search(_ptr(W), d_out, d_in, _ptr(x),
                             None if s_arr is None else _ptr(s_arr), group_size, n_clip,
                             flags, _ptr(idx), _ptr(err))
+    return idx, err
+
+
+def clip_search_output(X, W, s=None, group_size: int = 128, n_clip: int = 10,
+                       flags: int = 0):
+    """Output-space clip search: per (row, group) the ratio index minimising
+    sum_t (X[t, group] . (w - w_hat_clip))^2 (uint8 [d_out, d_in/g]) and the
+    totals (no clipping, chosen ratios) of those per-group errors."""
+    X, W = _f16(X), _f16(W)
+    T, d_in = X.shape
+    d_out = W.shape[0]
+    G = d_in // group_size
+    idx = np.empty((d_out, G), np.uint8)
+    err = np.empty(2, np.float64)
+    s_arr = None if s is None else _f32(s)
+    _load().orc_clip_search_output(_ptr(X), T, _ptr(W), d_out, d_in,
+                                   None if s_arr is None else _ptr(s_arr), group_size,
+                                   n_clip, flags, _ptr(idx), _ptr(err))
     return idx, err
 
 

@@ -467,6 +467,79 @@ void orc_clip_search(const uint16_t *W, int64_t d_out, int64_t d_in, const float
     free(row1);
 }
 
+/* Output-space clip search at a fixed scale s ([P3] "The pipeline end to
+ * end", step 5, with the candidates scored on the output as in [P3] "The
+ * scale search as code", restricted to one group so that every (row, group)
+ * choice is independent): for every row r, group k and ratio index i <
+ * n_clip,
+ *     e[r,k,i] = sum_t ( sum_{j in k} X[t,j] (W[r,j] - W_hat_i[r,j]) )^2
+ * with W_hat_i the clipped fake-quantisation of orc_fake_quant_group_clip,
+ * in fp64; clip_idx[r * G + k] = the first i with the smallest e.  err[0] is
+ * the sum over rows and groups of e[., ., 0] (no clipping), err[1] of the
+ * chosen e; summed per row, then over rows in order.  s == NULL: s = 1.  A
+ * non-finite group keeps index 0 and makes the totals NaN. */
+void orc_clip_search_output(const uint16_t *X, int64_t T, const uint16_t *W, int64_t d_out,
+                            int64_t d_in, const float *s, int64_t g, int n_clip, int flags,
+                            uint8_t *clip_idx, double *err)
+{
+    int64_t G = d_in / g;
+    double *Xd = (double *)malloc((size_t)T * (size_t)d_in * sizeof(double));
+    double *row0 = (double *)malloc((size_t)d_out * sizeof(double));
+    double *row1 = (double *)malloc((size_t)d_out * sizeof(double));
+    for (int64_t t = 0; t < T * d_in; ++t) Xd[t] = (double)h2f(X[t]);
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < d_out; ++r) {
+        float w[g], ones[g];
+        int8_t q[g];
+        double dw[g];
+        for (int64_t j = 0; j < g; ++j) ones[j] = 1.0f;
+        double a0 = 0.0, a1 = 0.0;
+        for (int64_t k = 0; k < G; ++k) {
+            for (int64_t j = 0; j < g; ++j) w[j] = h2f(W[r * d_in + k * g + j]);
+            const float *sk = s ? s + k * g : ones;
+            double best = 0.0, e0 = 0.0;
+            int b = 0, bad = 0;
+            for (int i = 0; i < n_clip; ++i) {
+                float qs;
+                if (orc_fake_quant_group_clip(w, sk, g, flags, orc_clip_ratio(i), q, &qs)) {
+                    bad = 1;
+                    break;
+                }
+                for (int64_t j = 0; j < g; ++j)
+                    dw[j] = (double)w[j] - (double)q[j] * (double)qs / (double)sk[j];
+                double e = 0.0;
+                for (int64_t t = 0; t < T; ++t) {
+                    double y = 0.0;
+                    for (int64_t j = 0; j < g; ++j) y += Xd[t * d_in + k * g + j] * dw[j];
+                    e += y * y;
+                }
+                if (i == 0) {
+                    e0 = e;
+                    best = e;
+                } else if (e < best) {
+                    best = e;
+                    b = i;
+                }
+            }
+            clip_idx[r * G + k] = (uint8_t)(bad ? 0 : b);
+            a0 += bad ? NAN : e0;
+            a1 += bad ? NAN : best;
+        }
+        row0[r] = a0;
+        row1[r] = a1;
+    }
+    double t0 = 0.0, t1 = 0.0;
+    for (int64_t r = 0; r < d_out; ++r) {
+        t0 += row0[r];
+        t1 += row1[r];
+    }
+    err[0] = t0;
+    err[1] = t1;
+    free(Xd);
+    free(row0);
+    free(row1);
+}
+
 /* ---------------------------------------------------------- scale search --
  * [P3] "The scale search as code" + [P1] "AWQ scaling": for every grid
  * index i the error of every weight segment that shares the input x is
