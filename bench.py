@@ -64,9 +64,8 @@ FMA_OPS_PER_PAIR = 5.5
 # stand; None where no capture of the current kernel exists.
 # DRAM bytes (read + write) of one launch of the dominant kernel, from an ncu
 # capture of the current kernel: (workload, asymmetric grid) -> bytes.
-NCU_TRAFFIC = {("q_proj_4096x4096", False): 34254848,        # search_kernel<8,0,0>
-               ("q_proj_4096x4096", True): 34256384,         # search_kernel<8,0,1>
-               ("down_proj_output_error", False): 3105129984}  # oe_gemm_kernel, per alpha
+NCU_TRAFFIC = {("q_proj_4096x4096", False): 34258432,        # search_kernel<8,0,0>
+               ("down_proj_output_error", False): 1506610176}  # oe_gemm_kernel, per alpha
 FP32_LANES_PER_SM = 128
 DEFAULT_STEPS = {"single_linear_256x512": 1000, "q_proj_4096x4096": 1000,
                  "qwen3_8b_block": 100, "down_proj_output_error": 10,
@@ -93,6 +92,9 @@ def _args():
     ap.add_argument("--clip", type=int, default=0,
                     help="also run the clip search with this many ratios per member "
                          "(0: off, the method's default path)")
+    ap.add_argument("--clip-space", choices=["weight", "output"], default="weight",
+                    help="score the clip search's ratios on the activation-weighted weight "
+                         "error (weight) or on each group's share of the output error (output)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-graph", action="store_true",
@@ -340,7 +342,7 @@ def run_ours(a):
             jobs.append(pipeline.GroupJob([W.to(dev) for W in Ws], X.to(dev), g, n_grid,
                                           work.output_mode, n_clip=a.clip,
                                           scale_mode=a.scale_mode, duo=a.duo,
-                                          asym=a.asym))
+                                          asym=a.asym, clip_space=a.clip_space))
     if work.layers == 1:
         host_layer = [([W.pin_memory() for W in Ws], X.pin_memory()) for Ws, X in layer_inputs[0]]
     else:
@@ -449,7 +451,7 @@ def run_ours(a):
     template = layer_inputs[0]
     streamer = pipeline.LayerStreamer(template, dev, g, n_grid, work.output_mode,
                                       n_clip=a.clip, scale_mode=a.scale_mode, duo=a.duo,
-                                      asym=a.asym)
+                                      asym=a.asym, clip_space=a.clip_space)
     if work.layers == 1:
         n_e2e = max(20, min(50, a.steps // 20))
         host_layers = [host_layer] * n_e2e
@@ -576,7 +578,15 @@ def run_ours(a):
                 "probe_sm_mhz": probe["sm_mhz"], "probe_clock_samples": probe["samples"],
                 "basis": "FP32 FMA stream (libawq_probe.so, best of scalar / packed / mixed), "
                          "per SM per clock, scaled to the search passes' clock"}
-        if a.clip > 0:
+        if a.clip > 0 and a.clip_space == "output":
+            # Gram matrices (2 T g d_in per group set) + quadratic forms (2 g^2 per row,
+            # group and ratio)
+            gram = sum(2.0 * j.X.shape[0] * g * j.X.shape[1] for j in jobs for _ in j.Ws)
+            forms = sum(2.0 * g * g * (W.numel() // g) * a.clip for j in jobs for W in j.Ws)
+            kernels["clip_search"] = {"ms": ms_clip, "n_clip": a.clip, "space": "output",
+                                      "flop": gram + forms,
+                                      "TFLOP/s": (gram + forms) / (ms_clip * 1e-3) / 1e12}
+        elif a.clip > 0:
             clip_ops = params * a.clip * ALG_OPS_PER_PAIR
             kernels["clip_search"] = {"ms": ms_clip, "n_clip": a.clip,
                                       "Top/s": clip_ops / (ms_clip * 1e-3) / 1e12,
@@ -597,6 +607,7 @@ def run_ours(a):
         "config": {"workload": a.workload, "layers": work.layers, "tokens": work.tokens,
                    "group_size": g, "n_grid": n_grid, "n_clip": a.clip,
                    "scale_mode": a.scale_mode, "duo": a.duo, "asym": a.asym,
+                   "clip_space": a.clip_space,
                    "params_per_step": _total_params(work, world, params),
                    "params_rank0": params,
                    "l2": ("flushed (256 MB write) between timed steps" if flush_l2 else
@@ -612,7 +623,7 @@ def run_ours(a):
     }
     if world == 1 and not a.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(work, g, a.cpu_seconds, a.clip, a.scale_mode,
-                                           a.duo, a.asym)
+                                           a.duo, a.asym, a.clip_space)
     print(json.dumps(out), flush=True)
     if world > 1:
         dist.destroy_process_group()
@@ -663,7 +674,7 @@ def oracle_sample(work, g, row_cap=256, out_rows=16, out_tokens=None):
 
 
 def _oracle_pass(sample, g, n_grid, output_mode, n_clip=0, scale_mode="joint", duo=False,
-                 asym=False):
+                 asym=False, clip_space="weight"):
     import oracle
     fl = (oracle.DUO if duo else 0) | (oracle.ASYM if asym else 0)
     zp = -1 if asym else 8
@@ -678,11 +689,15 @@ def _oracle_pass(sample, g, n_grid, output_mode, n_clip=0, scale_mode="joint", d
         else:
             err, best, s = oracle.scale_search(Ws, x, g, n_grid, fl)
         for W in Ws:
-            idx = oracle.clip_search(W, x, s, g, n_clip)[0] if n_clip > 0 else None
+            if n_clip > 0 and clip_space == "output":
+                idx = oracle.clip_search_output(X, W, s, g, n_clip)[0]
+            else:
+                idx = oracle.clip_search(W, x, s, g, n_clip)[0] if n_clip > 0 else None
             oracle.quantize_pack(W, s, g, zp, idx)
 
 
-def cpu_baseline(work, g, seconds, n_clip=0, scale_mode="joint", duo=False, asym=False):
+def cpu_baseline(work, g, seconds, n_clip=0, scale_mode="joint", duo=False, asym=False,
+                 clip_space="weight"):
     """Passes of the CPU oracle over a bounded sample of the workload until
     `seconds` have elapsed."""
     import oracle
@@ -692,7 +707,8 @@ def cpu_baseline(work, g, seconds, n_clip=0, scale_mode="joint", duo=False, asym
     n = 0
     t0 = time.perf_counter()
     while True:
-        _oracle_pass(sample, g, work.n_grid, work.output_mode, n_clip, scale_mode, duo, asym)
+        _oracle_pass(sample, g, work.n_grid, work.output_mode, n_clip, scale_mode, duo, asym,
+                     clip_space)
         n += 1
         if time.perf_counter() - t0 >= seconds:
             break
@@ -716,11 +732,11 @@ def run_reference(a):
         text += f" + {a.clip}-ratio clip search"
     for _ in range(max(a.warmup, 3)):
         _oracle_pass(sample, g, work.n_grid, work.output_mode, a.clip, a.scale_mode, a.duo,
-                     a.asym)
+                     a.asym, a.clip_space)
     t0 = time.perf_counter()
     for _ in range(a.steps):
         _oracle_pass(sample, g, work.n_grid, work.output_mode, a.clip, a.scale_mode, a.duo,
-                     a.asym)
+                     a.asym, a.clip_space)
     dt = time.perf_counter() - t0
     v = a.steps * params / dt / 1e9
     print(json.dumps({

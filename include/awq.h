@@ -82,6 +82,7 @@ typedef enum awq_status {
 #define AWQ_OP_OUTPUT_ERROR 2
 #define AWQ_OP_CLIP_SEARCH  3
 #define AWQ_OP_SCALE_SEARCH_DUO 4   /* awq_scale_search with AWQ_DUO_SCALING */
+#define AWQ_OP_CLIP_SEARCH_OUTPUT 5 /* awq_clip_search_output */
 
 /* Clip ratios: index i stands for c_i = (AWQ_CLIP_DEN - i) / AWQ_CLIP_DEN
  * rounded to fp32; 0 is no clipping, at most AWQ_CLIP_MAX ratios. */
@@ -351,6 +352,43 @@ awq_status awq_clip_search(const void *W, int64_t d_out, int64_t d_in,
                            int n_clip, int flags, uint8_t *clip_idx,
                            double *err, void *ws, size_t ws_bytes,
                            void *stream);
+
+/*
+ * The clip search scored in output space ("AWQ architecture ...", section
+ * "The pipeline end to end", step 5: the clipping range; section "The scale
+ * search as code": candidates scored on the output).  The pages give no
+ * formula; the reading: ratios and clipped fake quantisation exactly as in
+ * awq_clip_search (codes decided by the IEEE quotient), and each row r,
+ * group k and ratio i scored by the group's share of the output error
+ *
+ *   e[r,k,i] = sum_t ( sum_{j in group k} X[t,j] (W[r,j] - W_hat_i[r,j]) )^2
+ *
+ * (evaluated as v^T H_k v with H_k = X_k^T X_k: the Gram matrix in fp64,
+ * rounded to fp32, the forms in fp32 with fp64 sums across the warp, so e
+ * is within about 1e-6 relative of the fp64 definition and two ratios
+ * closer than that may be ordered differently).  clip_idx[r,k] = the first
+ * i with the smallest e; err[0] = sum of e[.,.,0] (no clipping), err[1] =
+ * sum of the chosen e, fixed-order sums (deterministic).
+ *
+ *   X           fp16 [T, ld] device (the linear's input); 1 <= T <= 2^24,
+ *               ld % 8 == 0, ld >= d_in
+ *   W           fp16 [d_out, d_in] device;  1 <= d_out <= 2^22
+ *   s           fp32 [d_in] device scale (normally s_best), or NULL for 1
+ *   group_size  32, 64 or 128;  d_in a multiple of it, <= 2^20
+ *   n_clip      1..AWQ_CLIP_MAX;  flags AWQ_SCALE_FP16 or AWQ_SCALE_FP32
+ *   clip_idx    uint8 [d_out, d_in / group_size] device output (feeds
+ *               awq_quantize_pack's clip_idx)
+ *   err         fp64 [2] device output (NaN if W holds a non-finite value,
+ *               raising AWQ_FLAG_NONFINITE_SCORE; such a group keeps index 0)
+ *   ws          workspace of awq_workspace_size(AWQ_OP_CLIP_SEARCH_OUTPUT,
+ *               T, d_out, d_in, group_size, 1, ...): the Gram matrices
+ *               (d_in * group_size fp32) and per-CTA partials; 256-byte aligned
+ */
+awq_status awq_clip_search_output(const void *X, int64_t T, int64_t ld, const void *W,
+                                  int64_t d_out, int64_t d_in, const float *s,
+                                  int group_size, int n_clip, int flags,
+                                  uint8_t *clip_idx, double *err, void *ws,
+                                  size_t ws_bytes, void *stream);
 
 /*
  * Optional output-space scoring of every grid point ("AWQ architecture

@@ -23,6 +23,7 @@ OP_SCALE_SEARCH = 1
 OP_OUTPUT_ERROR = 2
 OP_CLIP_SEARCH = 3
 OP_SCALE_SEARCH_DUO = 4
+OP_CLIP_SEARCH_OUTPUT = 5
 DUO_SCALING = 2
 ASYMMETRIC = 4
 ZERO_POINT_ASYM = -1
@@ -81,6 +82,9 @@ def lib() -> ctypes.CDLL:
         L.awq_clip_search.restype = i32
         L.awq_output_error.argtypes = [p, i64, p, i64, i64, p, i32, i32, i32, p, p, p, p, sz, p]
         L.awq_output_error.restype = i32
+        L.awq_clip_search_output.argtypes = [p, i64, i64, p, i64, i64, p, i32, i32, i32, p, p,
+                                             p, sz, p]
+        L.awq_clip_search_output.restype = i32
         L.awq_last_device_flags.argtypes = [ctypes.POINTER(ctypes.c_uint32), i32]
         L.awq_last_device_flags.restype = i32
         _lib = L
@@ -253,6 +257,33 @@ def clip_search(W: torch.Tensor, x: torch.Tensor, s: Optional[torch.Tensor] = No
                                  idx.data_ptr(), err.data_ptr(), ws.data_ptr(), ws.numel(),
                                  _stream(dev)),
            "awq_clip_search")
+    return idx, err
+
+
+def clip_search_output(X: torch.Tensor, W: torch.Tensor, s: Optional[torch.Tensor] = None,
+                       group_size: int = 128, n_clip: int = 10, flags: int = SCALE_FP16,
+                       out: Optional[Tuple[torch.Tensor, torch.Tensor]] = None,
+                       ws: Optional[torch.Tensor] = None):
+    """Clip search scored in output space (each group's share of
+    ||X (W - W_hat)^T||^2): (clip_idx uint8 [d_out, d_in/g], err fp64[2])."""
+    _cuda(X, torch.float16, "X")
+    _cuda(W, torch.float16, "W")
+    if s is not None:
+        _cuda(s, torch.float32, "s")
+    T, d_in = X.shape
+    d_out = W.shape[0]
+    dev = W.device
+    if out is None:
+        out = (torch.empty(d_out, d_in // group_size, dtype=torch.uint8, device=dev),
+               torch.empty(2, dtype=torch.float64, device=dev))
+    idx, err = out
+    if ws is None:
+        ws = workspace(OP_CLIP_SEARCH_OUTPUT, dev, T, d_out, d_in, group_size, 1)
+    _check(lib().awq_clip_search_output(X.data_ptr(), T, d_in, W.data_ptr(), d_out, d_in,
+                                        None if s is None else s.data_ptr(), group_size, n_clip,
+                                        flags, idx.data_ptr(), err.data_ptr(), ws.data_ptr(),
+                                        ws.numel(), _stream(dev)),
+           "awq_clip_search_output")
     return idx, err
 
 

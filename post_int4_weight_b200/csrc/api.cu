@@ -84,7 +84,7 @@ awq_status awq_last_device_flags(uint32_t* flags, int clear) {
     const bool c = clear != 0;
     cudaError_t (*const units[])(unsigned int*, bool) = {
         stats_unit_flags, search_unit_flags, pack_unit_flags, clip_unit_flags,
-        norm_group_unit_flags};
+        norm_group_unit_flags, clip_output_unit_flags};
     for (auto unit : units)
         if (note_cuda(unit(&bits, c), "awq_last_device_flags: flag word") != cudaSuccess)
             return AWQ_ERR_CUDA;
@@ -115,6 +115,12 @@ awq_status awq_workspace_size(int op, int64_t T, int64_t d_out_total, int64_t d_
         case AWQ_OP_CLIP_SEARCH:
             if (!valid_group(group_size)) return AWQ_ERR_INVALID_ARG;
             *bytes = clip_search_workspace();
+            return AWQ_OK;
+        case AWQ_OP_CLIP_SEARCH_OUTPUT:
+            if (!valid_group(group_size) || d_out_total < 1 || d_out_total > (int64_t(1) << 22) ||
+                d_in % group_size || d_in > (int64_t(1) << 20))
+                return AWQ_ERR_INVALID_ARG;
+            *bytes = clip_output_workspace(d_out_total, d_in, group_size);
             return AWQ_OK;
         case AWQ_OP_OUTPUT_ERROR:
             if (!valid_group(group_size) || n_grid < 1 || n_grid > 32 || T < 1 ||
@@ -234,6 +240,32 @@ awq_status awq_clip_search(const void* W, int64_t d_out, int64_t d_in, const flo
     if (note_cuda(launch_clip_search(W, d_out, d_in, x_mean, s, group_size, n_clip, flags,
                                      clip_idx, err, ws, static_cast<cudaStream_t>(stream)),
                   "clip_search launch") != cudaSuccess)
+        return AWQ_ERR_CUDA;
+    return AWQ_OK;
+}
+
+awq_status awq_clip_search_output(const void* X, int64_t T, int64_t ld, const void* W,
+                                  int64_t d_out, int64_t d_in, const float* s, int group_size,
+                                  int n_clip, int flags, uint8_t* clip_idx, double* err,
+                                  void* ws, size_t ws_bytes, void* stream) {
+    const NvtxRange nvtx_range("awq_clip_search_output");
+    if (!X || !W || !clip_idx || !err) return AWQ_ERR_INVALID_ARG;
+    if (!valid_group(group_size)) return AWQ_ERR_UNSUPPORTED;
+    if (n_clip < 1 || n_clip > AWQ_CLIP_MAX) return AWQ_ERR_INVALID_ARG;
+    if (flags != AWQ_SCALE_FP16 && flags != AWQ_SCALE_FP32) return AWQ_ERR_INVALID_ARG;
+    if (T < 1 || T > (int64_t(1) << 24)) return AWQ_ERR_INVALID_ARG;
+    if (d_out < 1 || d_out > (int64_t(1) << 22)) return AWQ_ERR_INVALID_ARG;
+    if (d_in < group_size || d_in % group_size || d_in > (int64_t(1) << 20) || ld < d_in)
+        return AWQ_ERR_INVALID_ARG;
+    if (ld % 8) return AWQ_ERR_ALIGNMENT;
+    if (!aligned16(X) || !aligned16(W) || !aligned16(err) || (s && !aligned16(s)))
+        return AWQ_ERR_ALIGNMENT;
+    if (!ws || ws_bytes < clip_output_workspace(d_out, d_in, group_size)) return AWQ_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(ws) & (kWsAlign - 1)) != 0) return AWQ_ERR_ALIGNMENT;
+    if (note_cuda(launch_clip_search_output(X, T, ld, W, d_out, d_in, s, group_size, n_clip,
+                                            flags, clip_idx, err, ws,
+                                            static_cast<cudaStream_t>(stream)),
+                  "clip_search_output launch") != cudaSuccess)
         return AWQ_ERR_CUDA;
     return AWQ_OK;
 }

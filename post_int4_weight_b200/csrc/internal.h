@@ -51,6 +51,7 @@ cudaError_t search_unit_flags(unsigned int* bits, bool clear);
 cudaError_t pack_unit_flags(unsigned int* bits, bool clear);
 cudaError_t clip_unit_flags(unsigned int* bits, bool clear);
 cudaError_t norm_group_unit_flags(unsigned int* bits, bool clear);
+cudaError_t clip_output_unit_flags(unsigned int* bits, bool clear);
 
 // ---- activation statistics
 size_t act_stats_workspace(int64_t d_in);
@@ -89,6 +90,14 @@ size_t clip_search_workspace();
 cudaError_t launch_clip_search(const void* W, int64_t d_out, int64_t d_in, const float* x_mean,
                                const float* s, int group_size, int n_clip, int flags,
                                uint8_t* clip_idx, double* err, void* ws, cudaStream_t stream);
+
+// ---- output-space clip search (Gram matrices of X's groups, then the
+// per (row, group, ratio) quadratic forms)
+size_t clip_output_workspace(int64_t d_out, int64_t d_in, int group_size);
+cudaError_t launch_clip_search_output(const void* X, int64_t T, int64_t ld, const void* W,
+                                      int64_t d_out, int64_t d_in, const float* s,
+                                      int group_size, int n_clip, int flags, uint8_t* clip_idx,
+                                      double* err, void* ws, cudaStream_t stream);
 
 // ---- output-space scoring
 size_t output_error_workspace(int64_t T, int64_t d_out, int64_t d_in, int group_size,

@@ -27,6 +27,7 @@ from . import awq
 LAUNCHES_STATS = 1
 LAUNCHES_SEARCH = 2            # scale table + fused search with finalize
 LAUNCHES_CLIP = 1              # per member (plus a 4-byte memset of its counter)
+LAUNCHES_CLIP_OUTPUT = 2       # per member: Gram matrices + scoring (plus the memset)
 
 
 def launches_output_error(n_grid: int) -> int:
@@ -68,7 +69,7 @@ class GroupJob:
     def __init__(self, Ws: Sequence[torch.Tensor], X: torch.Tensor, group_size: int = 128,
                  n_grid: int = 20, output_mode: bool = False, zero_point: int = 8,
                  n_clip: int = 0, scale_mode: str = "joint", duo: bool = False,
-                 asym: bool = False):
+                 asym: bool = False, clip_space: str = "weight"):
         if output_mode and len(Ws) != 1:
             raise ValueError("the output-space score takes one linear per call")
         if scale_mode not in ("joint", "geomean"):
@@ -79,6 +80,9 @@ class GroupJob:
         self.n_grid = n_grid
         self.output_mode = output_mode
         self.n_clip = n_clip
+        if clip_space not in ("weight", "output"):
+            raise ValueError("clip_space is 'weight' or 'output'")
+        self.clip_space = clip_space
         self.flags = (awq.DUO_SCALING if duo else 0) | (awq.ASYMMETRIC if asym else 0)
         if (duo or asym) and output_mode:
             raise ValueError("duo scaling and the asymmetric grid are weight-space options")
@@ -130,7 +134,8 @@ class GroupJob:
             search = LAUNCHES_SEARCH * len(self.Ws) + 1
         else:
             search = LAUNCHES_SEARCH
-        clip = LAUNCHES_CLIP * len(self.Ws) if self.n_clip > 0 else 0
+        per_clip = LAUNCHES_CLIP_OUTPUT if self.clip_space == "output" else LAUNCHES_CLIP
+        clip = per_clip * len(self.Ws) if self.n_clip > 0 else 0
         return LAUNCHES_STATS + search + clip + len(self.Ws)
 
     def workspace_bytes(self) -> Tuple[int, int, int]:
@@ -141,8 +146,9 @@ class GroupJob:
         op = awq.OP_OUTPUT_ERROR if self.output_mode else (
             awq.OP_SCALE_SEARCH_DUO if self.flags & awq.DUO_SCALING else awq.OP_SCALE_SEARCH)
         se = awq.workspace_size(op, T, d_out, d_in, self.g, self.n_grid)
-        cl = awq.workspace_size(awq.OP_CLIP_SEARCH, T, d_out, d_in, self.g, 1) \
-            if self.n_clip > 0 else 0
+        cl_op = awq.OP_CLIP_SEARCH_OUTPUT if self.clip_space == "output" else awq.OP_CLIP_SEARCH
+        d_max = max(W.shape[0] for W in self.Ws)
+        cl = awq.workspace_size(cl_op, T, d_max, d_in, self.g, 1) if self.n_clip > 0 else 0
         return st, se, cl
 
     def stats(self, ws: torch.Tensor):
@@ -165,7 +171,11 @@ class GroupJob:
 
     def clip(self, ws: torch.Tensor):
         for W, cl in zip(self.Ws, self.clips):
-            awq.clip_search(W, self.x, self.s_best, self.g, self.n_clip, out=cl, ws=ws)
+            if self.clip_space == "output":
+                awq.clip_search_output(self.X, W, self.s_best, self.g, self.n_clip, out=cl,
+                                       ws=ws)
+            else:
+                awq.clip_search(W, self.x, self.s_best, self.g, self.n_clip, out=cl, ws=ws)
 
     def pack(self):
         for m, (W, pk) in enumerate(zip(self.Ws, self.packs)):
@@ -213,7 +223,7 @@ class LayerStreamer:
     def __init__(self, template, device, group_size: int = 128, n_grid: int = 20,
                  output_mode: bool = False, zero_point: int = 8, depth: int = 2,
                  n_clip: int = 0, scale_mode: str = "joint", duo: bool = False,
-                 asym: bool = False):
+                 asym: bool = False, clip_space: str = "weight"):
         self.device = torch.device(device)
         self.depth = depth
         self.slots = []
@@ -223,7 +233,7 @@ class LayerStreamer:
                 dWs = [torch.empty(W.shape, dtype=torch.float16, device=self.device) for W in Ws]
                 dX = torch.empty(X.shape, dtype=torch.float16, device=self.device)
                 jobs.append(GroupJob(dWs, dX, group_size, n_grid, output_mode, zero_point,
-                                     n_clip, scale_mode, duo, asym))
+                                     n_clip, scale_mode, duo, asym, clip_space))
             self.slots.append(jobs)
         self.ws = Workspaces(self.slots[0], self.device)
         self.h2d = torch.cuda.Stream(self.device)

@@ -148,3 +148,17 @@ def test_output_error_canary():
     res = _twice(lambda: awq.output_error(X, W, x, g, 20, out=out, ws=ws), [X, W, x])
     ar.check()
     assert 0 <= int(res[1].view(np.int32)[0]) < 20
+
+
+@pytest.mark.parametrize("g", [128, 32])
+def test_clip_search_output_canary(g):
+    T, d_out, d_in = 72, 200, 384
+    W = wl.weight(d_out, d_in, 260).cuda()
+    X = wl.activations(T, d_in, 261).cuda()
+    x = awq.act_stats(X)
+    _, _, s = awq.scale_search([W], x, g, 20)
+    ar = Arena()
+    out = (ar.take((d_out, d_in // g), torch.uint8), ar.take((2,), torch.float64))
+    ws = ar.workspace(awq.OP_CLIP_SEARCH_OUTPUT, T, d_out, d_in, g, 1)
+    _twice(lambda: awq.clip_search_output(X, W, s, g, 10, out=out, ws=ws), [X, W, s])
+    ar.check()

@@ -133,3 +133,99 @@ def test_clip_nonfinite_zero_and_deterministic():
     idx_o, err_o = oracle.clip_search(W.numpy(), x, None, 128, 10)
     _check_indices(idx_c, idx_o, W, x, None, 128)
     np.testing.assert_allclose(err_c, err_o, rtol=ERR_RTOL, atol=0)
+
+
+# ------------------------------------------------------------ output space --
+# awq_clip_search_output: each (row, group) and ratio scored by the group's
+# share of the output error, against oracle.clip_search_output.  The GPU
+# evaluates the scores as fp32 quadratic forms of fp64 Gram matrices, so an
+# index may differ only where the oracle's two scores tie within 1e-5.
+
+OUT_TIE_RTOL = 1e-5
+
+
+def _out_score(X, w, s, g_cols, c):
+    q, qs = oracle.fake_quant_group_clip(w[g_cols], s[g_cols], c)
+    dw = w[g_cols].astype(np.float64) - q.astype(np.float64) * qs / s[g_cols].astype(np.float64)
+    y = X[:, g_cols].astype(np.float64) @ dw
+    return float(y @ y)
+
+
+def _check_clip_output(X, W, s, g, n_clip, idx_g, err_g):
+    idx_o, err_o = oracle.clip_search_output(X, W, s, g, n_clip)
+    np.testing.assert_allclose(err_g, err_o, rtol=ERR_RTOL, atol=0)
+    diff = np.argwhere(idx_g != idx_o)
+    assert len(diff) <= max(2, idx_o.size // 1000)
+    for r, k in diff:
+        cols = slice(k * g, (k + 1) * g)
+        w = W[r].astype(np.float32)
+        sv = np.ones(W.shape[1], np.float32) if s is None else s
+        a = _out_score(X, w, sv, cols, oracle.clip_ratio(int(idx_g[r, k])))
+        b = _out_score(X, w, sv, cols, oracle.clip_ratio(int(idx_o[r, k])))
+        assert abs(a - b) <= OUT_TIE_RTOL * b, (r, k, idx_g[r, k], idx_o[r, k], a, b)
+
+
+@pytest.mark.parametrize("d_out,d_in,T,g,n_clip", [(64, 256, 64, 32, 10), (200, 512, 96, 64, 20),
+                                                   (72, 384, 128, 128, 10), (8, 128, 1, 128, 3)])
+def test_clip_output_parity_small(d_out, d_in, T, g, n_clip):
+    seed = d_out + d_in + T + g
+    W = wl.weight(d_out, d_in, seed + 1)
+    W[min(3, d_out - 1), 17] = 0.3           # an outlier whose group wants clipping
+    X = wl.activations(T, d_in, seed)
+    s = np.exp(np.random.default_rng(seed).standard_normal(d_in) * 0.5).astype(np.float32)
+    idx, err = awq.clip_search_output(X.cuda(), W.cuda(), torch.from_numpy(s).cuda(), g, n_clip)
+    torch.cuda.synchronize()
+    _check_clip_output(X.numpy(), W.numpy(), s, g, n_clip, idx.cpu().numpy(), err.cpu().numpy())
+    # without s: the scale is 1
+    idx1, err1 = awq.clip_search_output(X.cuda(), W.cuda(), None, g, n_clip)
+    torch.cuda.synchronize()
+    _check_clip_output(X.numpy(), W.numpy(), None, g, n_clip, idx1.cpu().numpy(),
+                       err1.cpu().numpy())
+
+
+def test_clip_output_q_proj_rows_and_pack():
+    """The full q_proj 4096 x 4096 layer with 4096 tokens at its searched
+    scale: the first 64 rows' indices against the oracle on those rows
+    (a row's indices depend only on its own weights and X), the slice's
+    totals from a run on the slice, and the clipped pack of the full layer
+    against the oracle's pack at the GPU's indices."""
+    work = wl.WORKLOADS["q_proj_4096x4096"]
+    (grp, Ws, X), = wl.group_inputs(work)
+    W = Ws[0]
+    dev = torch.device("cuda")
+    Xd, Wd = X.to(dev), W.to(dev)
+    x = awq.act_stats(Xd)
+    _, best, s = awq.scale_search([Wd], x, 128, 20)
+    idx, err = awq.clip_search_output(Xd, Wd, s, 128, 10)
+    torch.cuda.synchronize()
+    s_np = s.cpu().numpy()
+    idx_np = idx.cpu().numpy()
+    rows = 64
+    idx_s, err_s = awq.clip_search_output(Xd, Wd[:rows].contiguous(), s, 128, 10)
+    torch.cuda.synchronize()
+    assert np.array_equal(idx_s.cpu().numpy(), idx_np[:rows])
+    _check_clip_output(X.numpy(), W[:rows].numpy(), s_np, 128, 10, idx_np[:rows],
+                       err_s.cpu().numpy())
+    assert idx_np.max() > 0 and err.cpu().numpy()[1] <= err.cpu().numpy()[0]
+    qw, sc, qz = awq.quantize_pack(Wd, s, 128, 8, clip_idx=idx)
+    torch.cuda.synchronize()
+    qw_o, sc_o, qz_o = oracle.quantize_pack(W.numpy(), s_np, 128, 8, idx_np)
+    assert np.array_equal(qw.cpu().numpy(), qw_o)
+    assert np.array_equal(sc.cpu().numpy().view(np.uint16), sc_o.view(np.uint16))
+
+
+def test_clip_output_nonfinite_and_deterministic():
+    W = wl.weight(64, 256, 91)
+    X = wl.activations(32, 256, 92)
+    a = awq.clip_search_output(X.cuda(), W.cuda(), None, 64, 10)
+    b = awq.clip_search_output(X.cuda(), W.cuda(), None, 64, 10)
+    torch.cuda.synchronize()
+    assert np.array_equal(a[0].cpu().numpy(), b[0].cpu().numpy())
+    assert np.array_equal(a[1].cpu().numpy(), b[1].cpu().numpy())
+    W[5, 70] = float("nan")
+    awq.last_device_flags(clear=True)
+    idx, err = awq.clip_search_output(X.cuda(), W.cuda(), None, 64, 10)
+    torch.cuda.synchronize()
+    assert np.isnan(err.cpu().numpy()).all()
+    assert int(idx.cpu().numpy()[5, 1]) == 0
+    assert awq.last_device_flags() == (6, awq.FLAG_NONFINITE_SCORE)

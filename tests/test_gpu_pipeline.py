@@ -175,3 +175,50 @@ def test_norm_group_mode_qkv_block_group():
         assert np.array_equal(pk[0].cpu().numpy(), qw_o)
         assert np.array_equal(pk[1].cpu().numpy().view(np.uint16), sc_o.view(np.uint16))
         assert np.array_equal(pk[2].cpu().numpy(), qz_o)
+
+
+def test_checkpointed_layers_resume_bit_identical(tmp_path):
+    """Three small layers quantised through the library with a checkpoint;
+    the first pass stops after layer 0 (a host-side stop, as a preempted job
+    would), the rerun computes only layers 1 and 2, and every layer's packed
+    output equals an uninterrupted run's bit for bit; layer 1 also equals
+    the oracle."""
+    from post_int4_weight_b200 import checkpoint as ck
+    dev = torch.device("cuda")
+    cfg = {"d_out": 256, "d_in": 512, "T": 64, "g": 128, "n_grid": 20}
+
+    def inputs(l):
+        return wl.weight(256, 512, 500 + l), wl.activations(64, 512, 600 + l)
+
+    def compute_fn(stop_at=None, calls=None):
+        def f(l):
+            if calls is not None:
+                calls.append(l)
+            if l == stop_at:
+                raise RuntimeError("stop")
+            W, X = inputs(l)
+            job = pipeline.GroupJob([W.to(dev)], X.to(dev), 128, 20)
+            wss = pipeline.Workspaces([job], dev)
+            job.run(wss)
+            qw, sc, qz = job.packs[0]
+            return {"qweight": qw, "scales": sc, "qzeros": qz, "s_best": job.s_best,
+                    "best": job.best}
+        return f
+
+    c = ck.StackCheckpoint(str(tmp_path / "a"), cfg)
+    with pytest.raises(RuntimeError):
+        ck.run_layers(range(3), compute_fn(stop_at=1), c)
+    calls = []
+    out = ck.run_layers(range(3), compute_fn(calls=calls), ck.StackCheckpoint(str(tmp_path / "a"), cfg))
+    assert calls == [1, 2]
+    ref = ck.run_layers(range(3), compute_fn(), ck.StackCheckpoint(str(tmp_path / "b"), cfg))
+    for l in range(3):
+        for k in out[l]:
+            assert torch.equal(out[l][k], ref[l][k]), (l, k)
+    W, X = inputs(1)
+    x = oracle.act_stats(X.numpy())
+    _, best_o, s_o = oracle.scale_search([W.numpy()], x, 128, 20)
+    qw_o, sc_o, qz_o = oracle.quantize_pack(W.numpy(), s_o, 128, 8)
+    assert int(out[1]["best"][0]) == best_o
+    assert np.array_equal(out[1]["qweight"].numpy(), qw_o)
+    assert np.array_equal(out[1]["scales"].numpy().view(np.uint16), sc_o.view(np.uint16))
