@@ -64,8 +64,11 @@ FMA_OPS_PER_PAIR = 5.5
 # stand; None where no capture of the current kernel exists.
 # DRAM bytes (read + write) of one launch of the dominant kernel, from an ncu
 # capture of the current kernel: (workload, asymmetric grid) -> bytes.
-NCU_TRAFFIC = {("q_proj_4096x4096", False): 34258432,        # search_kernel<8,0,0>
-               ("down_proj_output_error", False): 1506610176}  # oe_gemm_kernel, per alpha
+# (workload, asymmetric grid, group size) -> DRAM bytes of one launch of the
+# dominant kernel, read + written, from one ncu capture of the current kernel
+NCU_TRAFFIC = {("q_proj_4096x4096", False, 128): 34258432,        # search_kernel<8,0,0>
+               ("q_proj_4096x4096", True, 128): 34261248,         # search_kernel<8,0,1>
+               ("down_proj_output_error", False, 128): 1506610176}  # oe_gemm_kernel, per alpha
 FP32_LANES_PER_SM = 128
 DEFAULT_STEPS = {"single_linear_256x512": 1000, "q_proj_4096x4096": 1000,
                  "qwen3_8b_block": 100, "down_proj_output_error": 10,
@@ -539,8 +542,8 @@ def run_ours(a):
                           "GEMM with fused square-sum + finalize)",
                 "achieved": achieved / 1e12, "peak": peak_t / 1e12, "unit": "TFLOP/s",
                 "frac": achieved / peak_t,
-                "traffic": (NCU_TRAFFIC[(a.workload, False)] * n_grid
-                            if (a.workload, False) in NCU_TRAFFIC else None),
+                "traffic": (NCU_TRAFFIC[(a.workload, bool(a.asym), g)] * n_grid
+                            if (a.workload, bool(a.asym), g) in NCU_TRAFFIC else None),
                 "traffic_basis": "DRAM bytes of the n_grid GEMM launches of one call "
                                  "(ncu, per launch x n_grid)",
                 "flops_per_step": flops, "executed_flops_per_step": 2 * flops,
@@ -559,7 +562,7 @@ def run_ours(a):
                 "kernel": "awq_scale_search (table kernel + fused search kernel with finalize)",
                 "achieved": achieved / 1e12, "peak": peak_ops / 1e12, "unit": "Top/s",
                 "frac": achieved / peak_ops,
-                "traffic": NCU_TRAFFIC.get((a.workload, bool(a.asym))),
+                "traffic": NCU_TRAFFIC.get((a.workload, bool(a.asym), g)),
                 "ops_per_weight_alpha": ALG_OPS_PER_PAIR,
                 "executed_fma_pipe_ops_per_weight_alpha": FMA_OPS_PER_PAIR,
                 "executed_frac": executed / peak_ops,
