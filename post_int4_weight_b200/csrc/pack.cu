@@ -9,11 +9,12 @@
 //   scales[k, r]  = fp16 q_scale;   qzeros[k, c] = zero_point in every nibble
 //
 // HBM-bound: each weight is read once (2 B); 0.5 B of codes plus the group
-// scale (2/g B) and zero word (0.5/g B) are written.  One CTA of 8 warps
-// handles a 128-row x 128-column tile (one to four whole groups), several
-// CTAs per SM so that one CTA's tile streams in while others compute:
+// scale (2/g B) and zero word (0.5/g B) are written.  One CTA of 4 warps
+// handles a 64-row x 128-column tile (one to four whole groups), 11 CTAs
+// per SM so that one CTA's tile streams in while others compute (the
+// 64-row tile halves the last wave's work against a 128-row one):
 //   load     one thread issues two TMA copies (cp.async.bulk.tensor, 64
-//            columns x 128 rows each, 128-byte swizzle: 16-byte chunk c of
+//            columns x 64 rows each, 128-byte swizzle: 16-byte chunk c of
 //            row r sits at chunk c ^ (r & 7)); no thread spends an
 //            instruction on loading;
 //   scale    two threads per row (one per 64-column half) take max |w*s|
@@ -40,15 +41,15 @@
 namespace awq {
 namespace {
 
-constexpr int kPackRows = 128;
+constexpr int kPackRows = 64;                   // two threads per row
 constexpr int kPackCols = 128;
 constexpr int kBoxCols = 64;                    // 128 bytes: one swizzle row
-constexpr int kBoxBytes = kPackRows * kBoxCols * 2;   // 16 KB per box
+constexpr int kBoxBytes = kPackRows * kBoxCols * 2;   // 8 KB per box
 constexpr int kTileBytes = 2 * kBoxBytes;
-constexpr int kPackThreads = 256;
+constexpr int kPackThreads = 2 * kPackRows;
 constexpr int kPackWarps = kPackThreads / 32;
 constexpr int kRowsPerWarp = kPackRows / kPackWarps;  // 16
-constexpr int kPackCtasPerSm = 6;
+constexpr int kPackCtasPerSm = 11;              // the shared-memory limit
 constexpr int kClipDen = 20;                    // clip ratio c_i = (20 - i) / 20
 constexpr int kClipMaxIndex = 19;
 // per-(group, row) arrays: rows padded so the groups of one warp's lanes
@@ -56,7 +57,7 @@ constexpr int kClipMaxIndex = 19;
 constexpr int kRowStride = kPackRows + 4;
 
 struct PackParams {
-    CUtensorMap tmap;          // W fp16 [d_out, d_in], box {64, 128}, 128-byte swizzle
+    CUtensorMap tmap;          // W fp16 [d_out, d_in], box {64, 64}, 128-byte swizzle
     int64_t d_out, d_in;
     const float* s;            // [d_in] or NULL (s = 1)
     const uint8_t* clip_idx;   // [d_out, d_in / G] or NULL
@@ -176,11 +177,11 @@ pack_kernel(const __grid_constant__ PackParams p) {
             tma_load_2d(tile + kBoxBytes, &p.tmap, (int32_t)(col0 + kBoxCols), (int32_t)row0,
                         bar);
     }
-    if (tid < kPackCols) {
-        const int64_t gc = col0 + tid;
+    for (int j = tid; j < kPackCols; j += kPackThreads) {
+        const int64_t gc = col0 + j;
         const float sv = gc < p.d_in ? (p.s ? p.s[gc] : 1.0f) : 1.0f;
-        s_tile[s_slot(tid)] = sv;
-        sabs_tile[s_slot(tid)] = fabsf(sv);
+        s_tile[s_slot(j)] = sv;
+        sabs_tile[s_slot(j)] = fabsf(sv);
     }
     // the only wait of the kernel; a copy that has not landed after the
     // drain limit leaves the tile's outputs unwritten and the timeout bit set
