@@ -196,6 +196,8 @@ PACK_CASES = [
     (200, 384, 128, 8, True),     # C = 25 words: scalar stores, ragged rows
     (264, 96, 32, 7, True),       # d_in not a multiple of the 128-column tile
     (8, 192, 64, 8, True),        # a single word row
+    (120, 256, 64, 7, True),      # a 64-row tile, then one with 56 rows (a partial warp)
+    (328, 640, 128, 8, True),     # five whole 64-row tiles and an 8-row one
 ]
 
 
