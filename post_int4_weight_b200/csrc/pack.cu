@@ -21,18 +21,18 @@
 //            (NaN-propagating) of their half from 16-byte shared-memory reads
 //            (conflict-free under the swizzle) -> q_scale, its correctly
 //            rounded reciprocal, the stored fp16 scale;
-//   codes    warp w packs rows 16w..16w+15; lane l takes 4 consecutive
-//            columns of one half (8-byte reads: the 16 lanes of a half read
-//            one whole 128-byte row, conflict-free, and the swizzle term
-//            r & 7 = i & 7 is a constant of the unrolled row loop).  The
-//            quotient comes from the correctly rounded reciprocal with one
-//            residual correction, whose rounding decision is the IEEE
-//            quotient's (quot_rcp1_2, checked against __fdiv_rn around every
-//            half-integer); the 1.5*2^23 addition rounds it; one integer
-//            multiply-add per code places its nibble; two words (rows
-//            16w..16w+7, 16w+8..16w+15) per column are stored together.
-//            Row blocks whose scales are all fp16 normal numbers skip the
-//            clamp (|quotient| < 7.5 there).
+//   codes    warp w packs rows 32(w/2)..32(w/2)+31 of the 64-column half
+//            w % 2; lane l takes 2 consecutive columns of it (4-byte reads:
+//            the warp reads one whole 128-byte row, conflict-free, and the
+//            swizzle term r & 7 = i & 7 is a constant of the unrolled row
+//            loop).  The quotient comes from the correctly rounded
+//            reciprocal with one residual correction, whose rounding
+//            decision is the IEEE quotient's (quot_rcp1_2, checked against
+//            __fdiv_rn around every half-integer); the 1.5*2^23 addition
+//            rounds it; one integer multiply-add per code places its
+//            nibble; the four words of a column (32 rows) leave in one
+//            16-byte store.  Row blocks whose scales are all fp16 normal
+//            numbers skip the clamp (|quotient| < 7.5 there).
 #include <cstring>
 
 #include "common.cuh"
@@ -48,7 +48,7 @@ constexpr int kBoxBytes = kPackRows * kBoxCols * 2;   // 8 KB per box
 constexpr int kTileBytes = 2 * kBoxBytes;
 constexpr int kPackThreads = 2 * kPackRows;
 constexpr int kPackWarps = kPackThreads / 32;
-constexpr int kRowsPerWarp = kPackRows / kPackWarps;  // 16
+constexpr int kRowsPerWarp = 32;                // rows of one warp's codes (one half of the tile)
 constexpr int kPackCtasPerSm = 11;              // the shared-memory limit
 constexpr int kClipDen = 20;                    // clip ratio c_i = (20 - i) / 20
 constexpr int kClipMaxIndex = 19;
@@ -91,27 +91,26 @@ __device__ __forceinline__ int s_slot(int j) { return j + 4 * (j >> 6); }
 // Byte offset of 16-byte chunk c (0..7) of row r in a 128-byte-swizzled box.
 __device__ __forceinline__ int swz(int r, int c) { return r * 128 + ((c ^ (r & 7)) << 4); }
 
-// Codes of one lane's 4 columns over the warp's 16 rows, packed into two
-// words per column.  kSlow: clamp the codes (and store the zero point for a
-// non-finite group); taken per lane outside the row loop, so the loop itself
-// has no branch.
+// Codes of one lane's 2 columns over the warp's 32 rows, packed into four
+// words per column (one 16-byte store).  kSlow: clamp the codes (and store
+// the zero point for a non-finite group); taken per lane outside the row
+// loop, so the loop itself has no branch.
 template <bool kSlow, bool kAsym>
 __device__ __forceinline__ void pack_rows(const unsigned char* box, int chunk, float2 s01,
-                                          float2 s23, const float2* qr_row, const int* bad_row,
-                                          const int* zero_row, uint32_t words[4][2]) {
+                                          const float2* qr_row, const int* bad_row,
+                                          const int* zero_row, uint32_t words[2][4]) {
     const float2 magic2 = make_float2(kRoundMagic, kRoundMagic);
 #pragma unroll
     for (int i = 0; i < kRowsPerWarp; ++i) {
         // row rb + i: (rb + i) & 7 == i & 7, so the swizzle is a constant
-        const uint2 v = *reinterpret_cast<const uint2*>(box + i * 128 + ((chunk ^ (i & 7)) << 4));
+        const uint32_t v = *reinterpret_cast<const uint32_t*>(box + i * 128 +
+                                                              ((chunk ^ (i & 7)) << 4));
         const float2 qr = qr_row[i];           // (q_scale, 1 / q_scale)
         const float2 nb2 = make_float2(-qr.x, -qr.x), y2 = make_float2(qr.y, qr.y);
-        const float2 w01 = __half22float2(*reinterpret_cast<const __half2*>(&v.x));
-        const float2 w23 = __half22float2(*reinterpret_cast<const __half2*>(&v.y));
+        const float2 w01 = __half22float2(*reinterpret_cast<const __half2*>(&v));
         // w s / q_scale with one residual correction of w s * RN(1 / q_scale):
         // its rounding decision is the IEEE quotient's (see quot_rcp1_2)
         float2 t01 = __fadd2_rn(quot_rcp1_2(__fmul2_rn(w01, s01), nb2, y2), magic2);
-        float2 t23 = __fadd2_rn(quot_rcp1_2(__fmul2_rn(w23, s23), nb2, y2), magic2);
         if (kSlow) {
             float lo = kRoundMagic - 7.f, hi = kRoundMagic + 7.f;
             if (kAsym) {
@@ -120,18 +119,12 @@ __device__ __forceinline__ void pack_rows(const unsigned char* box, int chunk, f
                 hi = kRoundMagic + 15.f - z;
             }
             t01 = make_float2(fminf(fmaxf(t01.x, lo), hi), fminf(fmaxf(t01.y, lo), hi));
-            t23 = make_float2(fminf(fmaxf(t23.x, lo), hi), fminf(fmaxf(t23.y, lo), hi));
-            if (bad_row[i]) {   // code = zero point
-                t01 = magic2;
-                t23 = magic2;
-            }
+            if (bad_row[i]) t01 = magic2;   // code = zero point
         }
         const uint32_t shift = 1u << (4 * nibble_of_row(i & 7));
         const int hw = i >> 3;
         words[0][hw] += __float_as_uint(t01.x) * shift;
         words[1][hw] += __float_as_uint(t01.y) * shift;
-        words[2][hw] += __float_as_uint(t23.x) * shift;
-        words[3][hw] += __float_as_uint(t23.y) * shift;
     }
 }
 
@@ -139,7 +132,8 @@ template <int G, bool kAsym>
 __global__ void __launch_bounds__(kPackThreads, kPackCtasPerSm)
 pack_kernel(const __grid_constant__ PackParams p) {
     constexpr int KG = kPackCols / G;                 // groups per tile
-    constexpr int kBlocks = kPackRows / kRowsPerWarp;  // 16-row blocks per tile
+    constexpr int kBlocks = kPackRows / kRowsPerWarp;  // 32-row blocks per tile
+    static_assert(kPackWarps == 2 * kBlocks, "one warp per (32-row block, 64-column half)");
     extern __shared__ unsigned char smem_raw[];
     // the 128-byte swizzle wants 1024-byte aligned boxes
     const uint32_t raw = smem_addr(smem_raw);
@@ -300,49 +294,51 @@ pack_kernel(const __grid_constant__ PackParams p) {
         __syncthreads();
     }
 
-    // ---- codes and packed words: warp = 16 rows, lane = 4 columns of a half
+    // ---- codes and packed words: warp = 32 rows of one 64-column half,
+    // lane = 2 columns of it
     const int64_t C = p.d_out / 8;
     {
-        const int b = lane >> 4;                  // which 64-column half (box)
-        const int q4 = lane & 15;                 // 4-column quad within the half
-        const int jt = 64 * b + 4 * q4;           // first tile column of the lane
+        const int b = warp & 1;                   // which 64-column half (box)
+        const int blk = warp >> 1;                // which 32-row block
+        const int jt = 64 * b + 2 * lane;         // first tile column of the lane
         const int kk = jt / G;
-        const int rb = warp * kRowsPerWarp;       // first row of the warp
-        const unsigned char* box = tile + b * kBoxBytes + rb * 128 + (q4 & 1) * 8;
-        const int chunk = q4 >> 1;
-        const float4 s4 = *reinterpret_cast<const float4*>(&s_tile[s_slot(jt)]);
-        const float2 s01 = make_float2(s4.x, s4.y), s23 = make_float2(s4.z, s4.w);
+        const int rb = blk * kRowsPerWarp;        // first row of the warp
+        const unsigned char* box = tile + b * kBoxBytes + rb * 128 + (lane & 3) * 4;
+        const int chunk = lane >> 2;              // 16-byte chunk (8 columns) of the row
+        const float2 s01 = *reinterpret_cast<const float2*>(&s_tile[s_slot(jt)]);
         const float2* qr_row = qr_tile + kk * kRowStride + rb;
         const int* bad_row = bad_tile + kk * kRowStride + rb;
         const int* zero_row = zero_tile + kk * kRowStride + rb;
         // each nibble starts at (zero point - bits of 1.5*2^23); adding the
         // bits of the rounded quotient + 1.5*2^23 leaves the unsigned code
-        uint32_t words[4][2];
+        uint32_t words[2][4];
 #pragma unroll
-        for (int hw = 0; hw < 2; ++hw) {
+        for (int hw = 0; hw < 4; ++hw) {
             const uint32_t init =
                 kAsym ? zw_tile[kk * (kPackRows / 8) + rb / 8 + hw] - kRoundMagicBits * 0x11111111u
                       : 0u - (kRoundMagicBits - (uint32_t)p.zero_point) * 0x11111111u;
 #pragma unroll
-            for (int e = 0; e < 4; ++e) words[e][hw] = init;
+            for (int e = 0; e < 2; ++e) words[e][hw] = init;
         }
-        if (kAsym || slow_blk[kk * kBlocks + warp] != 0)
-            pack_rows<true, kAsym>(box, chunk, s01, s23, qr_row, bad_row, zero_row, words);
+        if (kAsym || slow_blk[kk * kBlocks + blk] != 0)
+            pack_rows<true, kAsym>(box, chunk, s01, qr_row, bad_row, zero_row, words);
         else
-            pack_rows<false, kAsym>(box, chunk, s01, s23, qr_row, bad_row, zero_row, words);
+            pack_rows<false, kAsym>(box, chunk, s01, qr_row, bad_row, zero_row, words);
         const int64_t cw = row0 / 8 + rb / 8;      // first output word of the warp
         if (cw < C) {   // d_out % 8 == 0: each word is wholly inside or outside
-            const bool two = cw + 1 < C;
+            const bool four = cw + 3 < C;
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
+            for (int e = 0; e < 2; ++e) {
                 const int64_t j = col0 + jt + e;
                 if (j >= p.d_in) continue;
                 int32_t* dst = p.qweight + j * C + cw;
-                if (two && (((uintptr_t)dst & 7u) == 0)) {
-                    *reinterpret_cast<uint2*>(dst) = make_uint2(words[e][0], words[e][1]);
+                if (four && (((uintptr_t)dst & 15u) == 0)) {
+                    *reinterpret_cast<uint4*>(dst) =
+                        make_uint4(words[e][0], words[e][1], words[e][2], words[e][3]);
                 } else {
-                    dst[0] = (int32_t)words[e][0];
-                    if (two) dst[1] = (int32_t)words[e][1];
+#pragma unroll
+                    for (int hw = 0; hw < 4; ++hw)
+                        if (cw + hw < C) dst[hw] = (int32_t)words[e][hw];
                 }
             }
         }
