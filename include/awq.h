@@ -75,6 +75,14 @@ typedef enum awq_status {
 #define AWQ_ASYMMETRIC 4
 /* zero_point argument of awq_quantize_pack selecting the asymmetric grid */
 #define AWQ_ZERO_POINT_ASYM (-1)
+/* awq_scale_search only, a TEST HOOK for the failure path of the bounded
+ * device waits: CTA 0's first weight load is armed for 16 bytes more than
+ * the copy carries, so that load's completion is a phase nothing finishes
+ * (the copy itself lands).  The CTA's waits give up after their 2 s limit
+ * and its drain after 20 s; the call then reports best_idx = -2 (err and
+ * s_best invalid) and raises AWQ_FLAG_WAIT_TIMEOUT, no copy is left in
+ * flight, and later calls run normally.  Never set outside such a test. */
+#define AWQ_TEST_STALL_WAIT 0x40000000
 
 /* Operation ids of awq_workspace_size. */
 #define AWQ_OP_ACT_STATS    0
@@ -196,7 +204,8 @@ awq_status awq_act_stats(const void *X, int64_t T, int64_t d_in, int64_t ld,
  *   x_mean      fp32 [d_in] device (from awq_act_stats)
  *   group_size  32, 64 or 128
  *   n_grid      1..32 grid points (20 in the method)
- *   flags       AWQ_SCALE_FP16 or AWQ_SCALE_FP32
+ *   flags       AWQ_SCALE_FP16 or AWQ_SCALE_FP32, optionally with
+ *               AWQ_DUO_SCALING, AWQ_ASYMMETRIC, AWQ_TEST_STALL_WAIT
  *   err         fp64 [n_grid] device output
  *   best_idx    int32 [1] device output; -1 if any err is not finite (NaN or
  *               infinite input; raises AWQ_FLAG_NONFINITE_SCORE), -2 if a

@@ -27,6 +27,9 @@ OP_CLIP_SEARCH_OUTPUT = 5
 DUO_SCALING = 2
 ASYMMETRIC = 4
 ZERO_POINT_ASYM = -1
+# test hook of scale_search: one weight load that never completes (see
+# AWQ_TEST_STALL_WAIT in include/awq.h); only for the failure-path test
+TEST_STALL_WAIT = 0x40000000
 CLIP_DEN = 20
 MAX_SEGMENTS = 8
 # sticky device-side condition bits (awq_last_device_flags)

@@ -159,7 +159,8 @@ awq_status awq_scale_search(int n_seg, const void* const* W, const int64_t* d_ou
     if (!x_mean || !err || !best_idx || !s_best) return AWQ_ERR_INVALID_ARG;
     if (!valid_group(group_size)) return AWQ_ERR_UNSUPPORTED;
     if (n_grid < 1 || n_grid > 32) return AWQ_ERR_INVALID_ARG;
-    if (flags & ~(AWQ_SCALE_FP32 | AWQ_DUO_SCALING | AWQ_ASYMMETRIC)) return AWQ_ERR_INVALID_ARG;
+    if (flags & ~(AWQ_SCALE_FP32 | AWQ_DUO_SCALING | AWQ_ASYMMETRIC | AWQ_TEST_STALL_WAIT))
+        return AWQ_ERR_INVALID_ARG;
     const bool duo = (flags & AWQ_DUO_SCALING) != 0;
     if (duo && d_in > kDuoMaxDin) return AWQ_ERR_UNSUPPORTED;
     if (d_in < group_size || d_in % group_size || d_in > (int64_t(1) << 24))

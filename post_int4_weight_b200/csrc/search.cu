@@ -447,7 +447,10 @@ search_kernel(const __grid_constant__ SearchParams p) {
     auto issue = [&](int64_t u, int stage) {
         int seg, grp, rb;
         decode(u, &seg, &grp, &rb);
-        mbar_arrive_expect_tx(&full[stage], kUnitBytes);
+        // the test hook: CTA 0's first load is armed for 16 bytes that never
+        // come, so its phase never completes (the copy itself lands)
+        const bool stall = (p.flags & AWQ_TEST_STALL_WAIT) && blockIdx.x == 0 && u == u0;
+        mbar_arrive_expect_tx(&full[stage], kUnitBytes + (stall ? 16u : 0u));
         // R rows in boxes of at most kMaxBoxRows (R = 512 for g = 32)
 #pragma unroll
         for (int b = 0; b * kMaxBoxRows < R; ++b)

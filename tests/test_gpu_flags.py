@@ -4,19 +4,25 @@ Non-finite data is made on the host (a NaN or an infinity written into an
 input before it is copied to the device), never by a fault.  Each call that
 meets it must raise its AWQ_FLAG_* bit besides what its outputs show; clean
 inputs raise nothing; a clearing read zeroes the bits and a non-clearing
-read keeps them.  The bounded-wait bit (AWQ_FLAG_WAIT_TIMEOUT) is not made
-to fire here: that would need a wait that never ends.
+read keeps them.  The bounded-wait bit (AWQ_FLAG_WAIT_TIMEOUT) fires through
+the search's test hook AWQ_TEST_STALL_WAIT: one weight load is armed for 16
+bytes that never come, a phase that nothing completes (the copy itself
+lands), so the waits run to their limits and give up; no fault, trap or
+endless loop is involved.
 """
+import time
+
 import numpy as np
 import pytest
 import torch
 
+import oracle
 from post_int4_weight_b200 import awq
 from post_int4_weight_b200 import workloads as wl
 
 pytestmark = pytest.mark.gpu
 
-OK, NONFINITE = 0, 6
+OK, NONFINITE, TIMEOUT = 0, 6, 7
 
 
 @pytest.fixture(autouse=True)
@@ -112,3 +118,37 @@ def test_bits_accumulate_until_read():
     st, bits = awq.last_device_flags()
     assert st == NONFINITE
     assert bits == awq.FLAG_NONFINITE_X | awq.FLAG_NONFINITE_GROUP
+
+
+def test_stalled_wait_gives_up_and_the_next_call_runs():
+    """The give-up path of the bounded waits, on the search kernel: with
+    AWQ_TEST_STALL_WAIT, CTA 0's first weight load never completes its
+    phase.  Its consumer warps give up after the 2 s limit, the CTA stops
+    computing but takes every barrier, its drain gives up after 20 s (the
+    copy has landed; only the phase is missing), and the call reports
+    best_idx = -2, NaN s_best and AWQ_FLAG_WAIT_TIMEOUT.  The context stays
+    usable: the same search without the hook then matches the oracle."""
+    W, X = _clean_inputs(d_out=512, d_in=1024, T=128, seed=11)
+    x = awq.act_stats(X)
+    torch.cuda.synchronize()
+    t0 = time.monotonic()
+    err, best, s = awq.scale_search([W], x, 128, 20, awq.TEST_STALL_WAIT)
+    b = int(best.cpu()[0])
+    waited = time.monotonic() - t0
+    assert b == -2
+    assert np.isnan(s.cpu().numpy()).all()
+    assert waited >= 2.0                     # the waits ran to their limit
+    st, bits = awq.last_device_flags()
+    assert st == TIMEOUT and (bits & awq.FLAG_WAIT_TIMEOUT)
+    assert awq.last_device_flags() == (OK, 0)
+    # the next call on the same context runs normally
+    err2, best2, s2 = awq.scale_search([W], x, 128, 20)
+    torch.cuda.synchronize()
+    e_o, b_o, s_o = oracle.scale_search([W.cpu().numpy()], x.cpu().numpy(), 128, 20)
+    np.testing.assert_allclose(err2.cpu().numpy(), e_o, rtol=1e-5, atol=0)
+    b2 = int(best2.cpu()[0])
+    if b2 != b_o:   # a tie within the method's 1e-6 (the first minimum may differ)
+        assert abs(e_o[b2] - e_o[b_o]) <= 1e-6 * e_o[b_o]
+    else:
+        assert np.array_equal(s2.cpu().numpy(), s_o)
+    assert awq.last_device_flags() == (OK, 0)
