@@ -146,8 +146,8 @@ const char *awq_last_error(void);
  * Bytes of workspace that `op` needs for the given sizes.  For
  * AWQ_OP_ACT_STATS only d_in matters; for AWQ_OP_SCALE_SEARCH d_in, the
  * group size and n_grid; for AWQ_OP_OUTPUT_ERROR all of them (T is the token
- * count, d_out_total the rows of W); for AWQ_OP_CLIP_SEARCH only the group
- * size is checked (the workspace is a fixed 16.6 KB).  Writes *bytes; returns
+ * count, d_out_total the rows of W); for AWQ_OP_CLIP_SEARCH the group size
+ * and d_in (16.6 KB plus 4 bytes per input channel).  Writes *bytes; returns
  * AWQ_ERR_INVALID_ARG for an unknown op or out-of-range size.
  */
 awq_status awq_workspace_size(int op, int64_t T, int64_t d_out_total,

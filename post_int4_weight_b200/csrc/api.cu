@@ -113,8 +113,9 @@ awq_status awq_workspace_size(int op, int64_t T, int64_t d_out_total, int64_t d_
                      duo_workspace_bound(d_in, n_grid);
             return AWQ_OK;
         case AWQ_OP_CLIP_SEARCH:
-            if (!valid_group(group_size)) return AWQ_ERR_INVALID_ARG;
-            *bytes = clip_search_workspace();
+            if (!valid_group(group_size) || d_in < 1 || d_in > (int64_t(1) << 24))
+                return AWQ_ERR_INVALID_ARG;
+            *bytes = clip_search_workspace(d_in);
             return AWQ_OK;
         case AWQ_OP_CLIP_SEARCH_OUTPUT:
             if (!valid_group(group_size) || d_out_total < 1 || d_out_total > (int64_t(1) << 22) ||
@@ -236,7 +237,7 @@ awq_status awq_clip_search(const void* W, int64_t d_out, int64_t d_in, const flo
         return AWQ_ERR_INVALID_ARG;
     if (!aligned16(W) || !aligned16(x_mean) || !aligned16(err) || (s && !aligned16(s)))
         return AWQ_ERR_ALIGNMENT;
-    if (!ws || ws_bytes < clip_search_workspace()) return AWQ_ERR_WORKSPACE;
+    if (!ws || ws_bytes < clip_search_workspace(d_in)) return AWQ_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(ws) & (kWsAlign - 1)) != 0) return AWQ_ERR_ALIGNMENT;
     if (note_cuda(launch_clip_search(W, d_out, d_in, x_mean, s, group_size, n_clip, flags,
                                      clip_idx, err, ws, static_cast<cudaStream_t>(stream)),

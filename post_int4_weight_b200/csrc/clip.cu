@@ -19,6 +19,8 @@
 // lanes per row, 16 weights of two rows per lane, the search's layout);
 // tasks are dealt to warps in a fixed order by a persistent grid, so every
 // CTA's partial, and the final sums, are the same on every run.
+#include <algorithm>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -35,7 +37,7 @@ struct ClipParams {
     const uint4* W;        // fp16 [d_out, d_in], rows of d_in / 8 chunks
     int64_t d_out;
     int64_t d_in;
-    const float* x;        // [d_in]
+    const float* tau2;     // [d_in] (x / s)^2, from clip_tau_kernel
     const float* s;        // [d_in] or NULL (s = 1)
     int64_t groups;        // d_in / g
     int64_t n_tasks;       // row blocks x groups
@@ -67,15 +69,15 @@ __device__ __forceinline__ void unpack8(const uint4 v, float2* w) {
 // rq; 0 for a zero group): codes by the rounding addition, clamped to +-7.
 __device__ __forceinline__ float lane_error(const float2* ws, const float2* t2, float qs,
                                             float rq) {
-    const float2 nqs = f2(-qs, -qs);
+    const float2 nqs = f2(-qs, -qs), rq2 = f2(rq, rq);
+    const float2 magic2 = f2(kRoundMagic, kRoundMagic), nmagic2 = f2(-kRoundMagic, -kRoundMagic);
     float2 acc = f2(0.f, 0.f);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-        float tx = __fmaf_rn(ws[i].x, rq, kRoundMagic);
-        float ty = __fmaf_rn(ws[i].y, rq, kRoundMagic);
-        tx = fminf(fmaxf(tx, kRoundMagic - 7.f), kRoundMagic + 7.f);
-        ty = fminf(fmaxf(ty, kRoundMagic - 7.f), kRoundMagic + 7.f);
-        const float2 q = f2(__fadd_rn(tx, -kRoundMagic), __fadd_rn(ty, -kRoundMagic));
+        float2 t = __ffma2_rn(ws[i], rq2, magic2);
+        t = f2(fminf(fmaxf(t.x, kRoundMagic - 7.f), kRoundMagic + 7.f),
+               fminf(fmaxf(t.y, kRoundMagic - 7.f), kRoundMagic + 7.f));
+        const float2 q = __fadd2_rn(t, nmagic2);
         const float2 d = __ffma2_rn(q, nqs, ws[i]);
         acc = __ffma2_rn(__fmul2_rn(d, d), t2[i], acc);
     }
@@ -97,7 +99,11 @@ clip_kernel(const ClipParams p) {
     constexpr int RPT = 2 * kSlots;         // rows per task
     __shared__ double red[kClipWarps][2];
     __shared__ int last;
+    __shared__ float ratio[AWQ_CLIP_MAX];   // c_i = RN((20 - i) / 20), once per CTA
 
+    if (threadIdx.x < AWQ_CLIP_MAX)
+        ratio[threadIdx.x] = __fdiv_rn((float)(kClipDen - (int)threadIdx.x), (float)kClipDen);
+    __syncthreads();
     pdl_wait();   // W, x and s may come from the kernel before
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int l = lane % L, slot = lane / L;
@@ -114,7 +120,7 @@ clip_kernel(const ClipParams p) {
 
         float2 ws0[8], ws1[8], t2[8];
         {
-            float sv[16], xv[16];
+            float sv[16], tv[16];
             if (p.s) {
                 load_chunk_f32(p.s + ch0, sv);
                 load_chunk_f32(p.s + ch1, sv + 8);
@@ -122,8 +128,8 @@ clip_kernel(const ClipParams p) {
 #pragma unroll
                 for (int i = 0; i < 16; ++i) sv[i] = 1.f;
             }
-            load_chunk_f32(p.x + ch0, xv);
-            load_chunk_f32(p.x + ch1, xv + 8);
+            load_chunk_f32(p.tau2 + ch0, tv);
+            load_chunk_f32(p.tau2 + ch1, tv + 8);
             const uint4 z = make_uint4(0, 0, 0, 0);
             const uint4 a0 = v0 ? __ldg(p.W + r0 * ld + ch0 / 8) : z;
             const uint4 b0 = v0 ? __ldg(p.W + r0 * ld + ch1 / 8) : z;
@@ -139,9 +145,7 @@ clip_kernel(const ClipParams p) {
                 const float2 s2 = f2(sv[2 * i], sv[2 * i + 1]);
                 ws0[i] = __fmul2_rn(w0[i], s2);
                 ws1[i] = __fmul2_rn(w1[i], s2);
-                const float tx = __fdiv_rn(xv[2 * i], sv[2 * i]);
-                const float ty = __fdiv_rn(xv[2 * i + 1], sv[2 * i + 1]);
-                t2[i] = f2(tx * tx, ty * ty);
+                t2[i] = f2(tv[2 * i], tv[2 * i + 1]);
             }
         }
         // group maxima; fmaxf drops NaN, so a NaN product is tracked apart and
@@ -174,7 +178,7 @@ clip_kernel(const ClipParams p) {
         float e_first = 0.f, best = 0.f;
         int b_own = 0;
         for (int i = 0; i < p.n_clip; ++i) {
-            const float c = __fdiv_rn((float)(kClipDen - i), (float)kClipDen);
+            const float c = ratio[i];
             bool unused;
             const float qs = group_scale(__fmul_rn(m_own, c), p.fp32_scale != 0, &unused);
             const float rq = qs > 0.f ? rcp_approx(qs) : (qs == 0.f ? 0.f : qs);
@@ -261,6 +265,20 @@ clip_kernel(const ClipParams p) {
     }
 }
 
+// tau2[j] = (RN(x_j / s_j))^2 in fp32, once per call (every task of a
+// column's group reads it)
+__global__ void __launch_bounds__(256)
+clip_tau_kernel(const float* __restrict__ x, const float* __restrict__ s, int64_t d_in,
+                float* __restrict__ tau2) {
+    pdl_wait();   // x and s may come from the kernel before
+    pdl_launch_dependents();
+    for (int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; j < d_in;
+         j += (int64_t)gridDim.x * blockDim.x) {
+        const float t = s ? __fdiv_rn(x[j], s[j]) : x[j];
+        tau2[j] = __fmul_rn(t, t);
+    }
+}
+
 template <int L>
 cudaError_t launch_clip_L(const ClipParams& p, int grid, cudaStream_t st) {
     return launch_pdl(clip_kernel<L>, dim3(grid), dim3(kClipThreads), 0, st, p);
@@ -272,8 +290,9 @@ cudaError_t clip_unit_flags(unsigned int* bits, bool clear) {
     return unit_device_flags(bits, clear);
 }
 
-size_t clip_search_workspace() {
-    return align_up((size_t)kMaxClipCtas * 2 * sizeof(double), kWsAlign) + kWsAlign;
+size_t clip_search_workspace(int64_t d_in) {
+    return align_up((size_t)kMaxClipCtas * 2 * sizeof(double), kWsAlign) + kWsAlign +
+           align_up((size_t)d_in * sizeof(float), kWsAlign);
 }
 
 cudaError_t launch_clip_search(const void* W, int64_t d_out, int64_t d_in, const float* x_mean,
@@ -288,7 +307,6 @@ cudaError_t launch_clip_search(const void* W, int64_t d_out, int64_t d_in, const
     p.W = static_cast<const uint4*>(W);
     p.d_out = d_out;
     p.d_in = d_in;
-    p.x = x_mean;
     p.s = s;
     p.groups = d_in / group_size;
     p.n_tasks = (d_out + rows_per_task - 1) / rows_per_task * p.groups;
@@ -299,6 +317,9 @@ cudaError_t launch_clip_search(const void* W, int64_t d_out, int64_t d_in, const
     p.partial = reinterpret_cast<double*>(base);
     p.counter = reinterpret_cast<int*>(
         base + align_up((size_t)kMaxClipCtas * 2 * sizeof(double), kWsAlign));
+    float* tau2 = reinterpret_cast<float*>(
+        base + align_up((size_t)kMaxClipCtas * 2 * sizeof(double), kWsAlign) + kWsAlign);
+    p.tau2 = tau2;
     p.err = err;
     int64_t grid = (int64_t)dev.num_sms * kClipCtasPerSm;
     const int64_t need = (p.n_tasks + kClipWarps - 1) / kClipWarps;
@@ -306,6 +327,9 @@ cudaError_t launch_clip_search(const void* W, int64_t d_out, int64_t d_in, const
     if (grid > kMaxClipCtas) grid = kMaxClipCtas;
     if (grid < 1) grid = 1;
     e = cudaMemsetAsync(p.counter, 0, sizeof(int), stream);
+    if (e != cudaSuccess) return e;
+    const int tau_blocks = (int)std::min<int64_t>((d_in + 255) / 256, 4 * (int64_t)dev.num_sms);
+    e = launch_pdl(clip_tau_kernel, dim3(tau_blocks), dim3(256), 0, stream, x_mean, s, d_in, tau2);
     if (e != cudaSuccess) return e;
     switch (L) {
         case 2: return launch_clip_L<2>(p, (int)grid, stream);

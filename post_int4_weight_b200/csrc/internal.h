@@ -86,7 +86,7 @@ cudaError_t launch_norm_group_scale(int n, const float* const* s, int64_t d_in, 
                                     int num_sms, cudaStream_t stream);
 
 // ---- clip search
-size_t clip_search_workspace();
+size_t clip_search_workspace(int64_t d_in);
 cudaError_t launch_clip_search(const void* W, int64_t d_out, int64_t d_in, const float* x_mean,
                                const float* s, int group_size, int n_clip, int flags,
                                uint8_t* clip_idx, double* err, void* ws, cudaStream_t stream);

@@ -26,7 +26,7 @@ from . import awq
 # kernels each call launches (the library's own count, used for reporting)
 LAUNCHES_STATS = 1
 LAUNCHES_SEARCH = 2            # scale table + fused search with finalize
-LAUNCHES_CLIP = 1              # per member (plus a 4-byte memset of its counter)
+LAUNCHES_CLIP = 2              # per member: (x / s)^2 + clip search (plus the memset)
 LAUNCHES_CLIP_OUTPUT = 2       # per member: Gram matrices + scoring (plus the memset)
 
 
