@@ -361,6 +361,7 @@ __device__ __forceinline__ float2 rows_errors_asym_next(float2* ws0, float2* ws1
                                                         float2* mm0, float2* mm1) {
     const float2 nqs0 = f2(-qs0, -qs0), nqs1 = f2(-qs1, -qs1);
     const float2 rq02 = f2(rq0, rq0), mz02 = f2(mz0, mz0), nmz02 = f2(-mz0, -mz0);
+    const float2 rq12 = f2(rq1, rq1), mz12 = f2(mz1, mz1), nmz12 = f2(-mz1, -mz1);
     constexpr float lo = kRoundMagic, hi = kRoundMagic + 15.f;
     float2 acc2[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
     float mx0 = __int_as_float(0xff800000), mn0 = __int_as_float(0x7f800000);
@@ -374,15 +375,13 @@ __device__ __forceinline__ float2 rows_errors_asym_next(float2* ws0, float2* ws1
         for (int j = 0; j < 2; ++j) {
             const int i = 2 * k + j;
             float2 t0 = __ffma2_rn(ws0[i], rq02, mz02);
-            float t1x = __fmaf_rn(ws1[i].x, rq1, mz1);
-            float t1y = __fmaf_rn(ws1[i].y, rq1, mz1);
+            float2 t1 = __ffma2_rn(ws1[i], rq12, mz12);
             if (kClamp) {
                 t0 = f2(fminf(fmaxf(t0.x, lo), hi), fminf(fmaxf(t0.y, lo), hi));
-                t1x = fminf(fmaxf(t1x, lo), hi);
-                t1y = fminf(fmaxf(t1y, lo), hi);
+                t1 = f2(fminf(fmaxf(t1.x, lo), hi), fminf(fmaxf(t1.y, lo), hi));
             }
             const float2 q0 = __fadd2_rn(t0, nmz02);
-            const float2 q1 = f2(__fadd_rn(t1x, -mz1), __fadd_rn(t1y, -mz1));
+            const float2 q1 = __fadd2_rn(t1, nmz12);
             const float2 d0 = __ffma2_rn(q0, nqs0, ws0[i]);
             const float2 d1 = __ffma2_rn(q1, nqs1, ws1[i]);
             float2 sq = __fmul2_rn(d0, d0);
