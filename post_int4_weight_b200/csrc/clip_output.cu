@@ -13,10 +13,12 @@
 // the smallest e, err[0] / err[1] the totals without clipping / with the
 // chosen ratios.
 //
-//   gram_kernel         H_k for every group, in fp64 (fp16 products are exact
-//                       in fp64; T terms per entry), rounded once to fp32.
-//                       One CTA per (group, tile of H); HBM: X read once per
-//                       tile row of H.  2 T g d_in flop.
+//   gram_kernel         partial H_k for every group over up to 4 token slices,
+//                       in fp64 (fp16 products are exact in fp64), 16-byte
+//                       loads of X; one CTA per (group, tile of H, slice), so
+//                       the grid covers the SMs even for 32 groups.  HBM: X
+//                       read once per tile row of H.  2 T g d_in flop.
+//   gram_reduce_kernel  H_k = fp32(sum of the slices in order): deterministic.
 //   clip_output_kernel  one CTA per (group, 64 rows): H_k staged in shared
 //                       memory; warp w takes 8 rows; per ratio each lane forms
 //                       its g/32 entries of every row's v exactly (the IEEE
@@ -26,6 +28,7 @@
 //                       2 g^2 flop per (row, group, ratio).  Fixed task order
 //                       and a last-CTA sum of the per-CTA partials in a fixed
 //                       order: deterministic.
+#include <algorithm>
 #include <cstring>
 
 #include "common.cuh"
@@ -42,13 +45,18 @@ constexpr int kClipDen = 20;
 constexpr int kMaxCoCtas = 1 << 20;
 
 // ---------------------------------------------------------------- Gram
-// H_k[a][b] = sum_t X[t, k g + a] X[t, k g + b] for a 64 x 64 (g >= 64) or
-// 32 x 32 tile of H_k; each thread accumulates a 4 x 4 block in fp64.
+// Partial H_k[a][b] = sum_t X[t, k g + a] X[t, k g + b] over one slice of the
+// tokens (blockIdx.y; slices of t_per tokens) for a 64 x 64 (g >= 64) or
+// 32 x 32 tile of H_k; each thread accumulates a 4 x 4 block in fp64, tokens
+// in order, and writes it unrounded.  X arrives in 16-byte loads (8 halves).
+constexpr int kMaxGramSlices = 4;
 template <int TILE>
 __global__ void __launch_bounds__((TILE / 4) * (TILE / 4))
-gram_kernel(const __half* __restrict__ X, int64_t T, int64_t ld, int g, float* __restrict__ H) {
+gram_kernel(const __half* __restrict__ X, int64_t T, int64_t ld, int g, int64_t t_per,
+            double* __restrict__ Hpart) {
     constexpr int kT = 32;                      // tokens per staged chunk
     constexpr int kN = (TILE / 4) * (TILE / 4);
+    constexpr int kV = TILE / 8;                // 16-byte vectors per token row of a tile
     __shared__ double sa[kT][TILE];
     __shared__ double sb[kT][TILE];
     pdl_wait();
@@ -57,13 +65,27 @@ gram_kernel(const __half* __restrict__ X, int64_t T, int64_t ld, int g, float* _
     const int ti = (blockIdx.x / tiles) % tiles, tj = blockIdx.x % tiles;
     const int64_t ca = (int64_t)k * g + ti * TILE, cb = (int64_t)k * g + tj * TILE;
     const int tx = threadIdx.x % (TILE / 4), ty = threadIdx.x / (TILE / 4);
+    const int64_t t_begin = (int64_t)blockIdx.y * t_per;
+    const int64_t t_end = min(T, t_begin + t_per);
     double acc[4][4] = {};
-    for (int64_t t0 = 0; t0 < T; t0 += kT) {
-        for (int e = threadIdx.x; e < kT * TILE; e += kN) {
-            const int tt = e / TILE, c = e % TILE;
-            const bool in = t0 + tt < T;
-            sa[tt][c] = in ? (double)__half2float(X[(t0 + tt) * ld + ca + c]) : 0.0;
-            sb[tt][c] = in ? (double)__half2float(X[(t0 + tt) * ld + cb + c]) : 0.0;
+    for (int64_t t0 = t_begin; t0 < t_end; t0 += kT) {
+        for (int e = threadIdx.x; e < kT * kV; e += kN) {
+            const int tt = e / kV, c8 = e % kV;
+            const bool in = t0 + tt < t_end;
+            const uint4 va = in ? __ldg(reinterpret_cast<const uint4*>(X + (t0 + tt) * ld + ca) + c8)
+                                : make_uint4(0, 0, 0, 0);
+            const uint4 vb = in ? __ldg(reinterpret_cast<const uint4*>(X + (t0 + tt) * ld + cb) + c8)
+                                : make_uint4(0, 0, 0, 0);
+            const uint32_t wa[4] = {va.x, va.y, va.z, va.w}, wb[4] = {vb.x, vb.y, vb.z, vb.w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float2 fa = __half22float2(*reinterpret_cast<const __half2*>(&wa[q]));
+                const float2 fb = __half22float2(*reinterpret_cast<const __half2*>(&wb[q]));
+                sa[tt][8 * c8 + 2 * q] = (double)fa.x;
+                sa[tt][8 * c8 + 2 * q + 1] = (double)fa.y;
+                sb[tt][8 * c8 + 2 * q] = (double)fb.x;
+                sb[tt][8 * c8 + 2 * q + 1] = (double)fb.y;
+            }
         }
         __syncthreads();
 #pragma unroll 4
@@ -82,13 +104,27 @@ gram_kernel(const __half* __restrict__ X, int64_t T, int64_t ld, int g, float* _
         __syncthreads();
     }
     pdl_launch_dependents();
-    float* Hk = H + (int64_t)k * g * g;
+    // slice blockIdx.y of [slices][G][g][g]; gridDim.x / (tiles * tiles) = G
+    double* Hk = Hpart + ((int64_t)blockIdx.y * (gridDim.x / (tiles * tiles)) + k) * g * g;
 #pragma unroll
     for (int q = 0; q < 4; ++q)
 #pragma unroll
         for (int r = 0; r < 4; ++r)
-            Hk[(int64_t)(ti * TILE + 4 * ty + q) * g + tj * TILE + 4 * tx + r] =
-                __double2float_rn(acc[q][r]);
+            Hk[(int64_t)(ti * TILE + 4 * ty + q) * g + tj * TILE + 4 * tx + r] = acc[q][r];
+}
+
+// H = fp32(sum of the slices' partials, slices in order): deterministic.
+__global__ void __launch_bounds__(256)
+gram_reduce_kernel(const double* __restrict__ Hpart, int slices, int64_t n,
+                   float* __restrict__ H) {
+    pdl_wait();
+    pdl_launch_dependents();
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        double v = Hpart[i];
+        for (int s = 1; s < slices; ++s) v += Hpart[(int64_t)s * n + i];
+        H[i] = __double2float_rn(v);
+    }
 }
 
 // ---------------------------------------------------------- clip scoring
@@ -305,7 +341,8 @@ cudaError_t launch_co(const CoParams& p, int64_t row_blocks, cudaStream_t st) {
 size_t clip_output_workspace(int64_t d_out, int64_t d_in, int group_size) {
     const int64_t ctas = (d_in / group_size) * ((d_out + kCoRows - 1) / kCoRows);
     return align_up((size_t)d_in * (size_t)group_size * sizeof(float), kWsAlign) +
-           align_up((size_t)ctas * 2 * sizeof(double), kWsAlign) + kWsAlign;
+           align_up((size_t)ctas * 2 * sizeof(double), kWsAlign) + kWsAlign +
+           align_up((size_t)kMaxGramSlices * d_in * group_size * sizeof(double), kWsAlign);
 }
 
 cudaError_t clip_output_unit_flags(unsigned int* bits, bool clear) {
@@ -325,18 +362,35 @@ cudaError_t launch_clip_search_output(const void* X, int64_t T, int64_t ld, cons
     double* partial = reinterpret_cast<double*>(base);
     base += align_up((size_t)G * row_blocks * 2 * sizeof(double), kWsAlign);
     int* counter = reinterpret_cast<int*>(base);
+    base += kWsAlign;
+    double* Hpart = reinterpret_cast<double*>(base);
 
-    cudaError_t e = cudaMemsetAsync(counter, 0, sizeof(int), stream);
+    DeviceInfo dev;
+    cudaError_t e = query_device(&dev);
+    if (e != cudaSuccess) return e;
+    e = cudaMemsetAsync(counter, 0, sizeof(int), stream);
     if (e != cudaSuccess) return e;
     const __half* Xh = static_cast<const __half*>(X);
+    // token slices: about two CTAs per SM in all, at least 64 tokens a slice
+    const int tiles = group_size == 32 ? 1 : group_size / 64;
+    const int64_t gram_ctas = G * tiles * tiles;
+    int64_t slices = (2 * (int64_t)dev.num_sms + gram_ctas - 1) / gram_ctas;
+    slices = std::max<int64_t>(1, std::min<int64_t>({slices, (int64_t)kMaxGramSlices, T / 64}));
+    const int64_t t_per = ((T + slices - 1) / slices + 31) / 32 * 32;
+    slices = (T + t_per - 1) / t_per;
+    if (slices < 1) slices = 1;
     if (group_size == 32) {
-        e = launch_pdl(gram_kernel<32>, dim3((unsigned)G), dim3(64), 0, stream, Xh, T, ld,
-                       group_size, H);
+        e = launch_pdl(gram_kernel<32>, dim3((unsigned)G, (unsigned)slices), dim3(64), 0, stream,
+                       Xh, T, ld, group_size, t_per, Hpart);
     } else {
-        const int tiles = group_size / 64;
-        e = launch_pdl(gram_kernel<64>, dim3((unsigned)(G * tiles * tiles)), dim3(256), 0, stream,
-                       Xh, T, ld, group_size, H);
+        e = launch_pdl(gram_kernel<64>, dim3((unsigned)gram_ctas, (unsigned)slices), dim3(256), 0,
+                       stream, Xh, T, ld, group_size, t_per, Hpart);
     }
+    if (e != cudaSuccess) return e;
+    const int64_t n_h = d_in * (int64_t)group_size;
+    e = launch_pdl(gram_reduce_kernel, dim3((unsigned)std::min<int64_t>((n_h + 255) / 256,
+                                                                          4 * (int64_t)dev.num_sms)),
+                   dim3(256), 0, stream, static_cast<const double*>(Hpart), (int)slices, n_h, H);
     if (e != cudaSuccess) return e;
     CoParams p;
     std::memset(&p, 0, sizeof(p));

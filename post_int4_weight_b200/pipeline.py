@@ -27,7 +27,7 @@ from . import awq
 LAUNCHES_STATS = 1
 LAUNCHES_SEARCH = 2            # scale table + fused search with finalize
 LAUNCHES_CLIP = 2              # per member: (x / s)^2 + clip search (plus the memset)
-LAUNCHES_CLIP_OUTPUT = 2       # per member: Gram matrices + scoring (plus the memset)
+LAUNCHES_CLIP_OUTPUT = 3       # per member: Gram slices + their sum + scoring (plus the memset)
 
 
 def launches_output_error(n_grid: int) -> int:

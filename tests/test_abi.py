@@ -165,10 +165,13 @@ def test_pipeline_workspace_sizes_from_host_query():
     assert se_o >= 2 * 256 * 512 * 2            # the hi/lo dW buffer at least
     jc = pipeline.GroupJob(Ws, X, 128, 20, n_clip=10)
     assert jc.workspace_bytes()[2] > 0
-    # stats 1; search 2 (table, search); output mode 1 + 2 * 20 + 1; clip 1 per member;
-    # pack 1 per member
+    # stats 1; search 2 (table, search); output mode 1 + 2 * 20 + 1; clip 2 per
+    # member ((x / s)^2, search), 3 in output space (Gram slices, their sum,
+    # scoring); pack 1 per member
     assert j.launches == 1 + 2 + 2 and jo.launches == 1 + 42 + 1
-    assert jc.launches == 1 + 2 + 2 + 2
+    assert jc.launches == 1 + 2 + 2 * 2 + 2
+    jco = pipeline.GroupJob(Ws, X, 128, 20, n_clip=10, clip_space="output")
+    assert jco.launches == 1 + 2 + 2 * 3 + 2
     ws = pipeline.Workspaces([j, jo, jc], "cpu")
     assert ws.search.numel() == max(se, se_o)
 
