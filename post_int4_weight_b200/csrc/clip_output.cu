@@ -142,8 +142,11 @@ struct CoParams {
 };
 
 // kE = g / 32 entries of a group per lane (lane l holds entries kE*l ..).
+// Two CTAs per SM (128 registers; for g = 128 a few values spill): 1.86 ->
+// 1.76 ms on q_proj against one CTA of 207 registers, which left 8 warps per
+// SM to hide the shared-memory and FMA latencies.
 template <int kE>
-__global__ void __launch_bounds__(kCoThreads)
+__global__ void __launch_bounds__(kCoThreads, 2)
 clip_output_kernel(const CoParams p) {
     constexpr int G = 32 * kE;
     extern __shared__ __align__(16) float co_smem[];
