@@ -226,22 +226,41 @@ clip_output_kernel(const CoParams p) {
             }
         }
         __syncwarp();
-        // (H v)[a] for this lane's entries a = kE*lane + e, all rows at once
+        // (H v)[a] for this lane's entries a = kE*lane + e, all rows at once:
+        // v read four j at a time (one 16-byte broadcast per row), the lane's
+        // entries in pairs (packed fp32x2 FMAs); every entry still adds its
+        // terms in j order, one rounding each, as the scalar loop would
         float hv[kCoRowsPerWarp][kE];
 #pragma unroll
         for (int rr = 0; rr < kCoRowsPerWarp; ++rr)
 #pragma unroll
             for (int e = 0; e < kE; ++e) hv[rr][e] = 0.f;
-#pragma unroll 4
-        for (int j = 0; j < G; ++j) {
-            float h[kE];
+#pragma unroll 2
+        for (int j0 = 0; j0 < G; j0 += 4) {
+            float h[4][kE];
 #pragma unroll
-            for (int e = 0; e < kE; ++e) h[e] = Hs[j * G + kE * lane + e];
+            for (int q = 0; q < 4; ++q)
+#pragma unroll
+                for (int e = 0; e < kE; ++e) h[q][e] = Hs[(j0 + q) * G + kE * lane + e];
 #pragma unroll
             for (int rr = 0; rr < kCoRowsPerWarp; ++rr) {
-                const float vj = vb[rr * G + j];
+                const float4 v4 = *reinterpret_cast<const float4*>(&vb[rr * G + j0]);
+                const float vq[4] = {v4.x, v4.y, v4.z, v4.w};
 #pragma unroll
-                for (int e = 0; e < kE; ++e) hv[rr][e] = __fmaf_rn(h[e], vj, hv[rr][e]);
+                for (int q = 0; q < 4; ++q) {
+                    if constexpr (kE >= 2) {
+#pragma unroll
+                        for (int e = 0; e < kE; e += 2) {
+                            const float2 r2 = __ffma2_rn(make_float2(h[q][e], h[q][e + 1]),
+                                                         make_float2(vq[q], vq[q]),
+                                                         make_float2(hv[rr][e], hv[rr][e + 1]));
+                            hv[rr][e] = r2.x;
+                            hv[rr][e + 1] = r2.y;
+                        }
+                    } else {
+                        hv[rr][0] = __fmaf_rn(h[q][0], vq[q], hv[rr][0]);
+                    }
+                }
             }
         }
 #pragma unroll
