@@ -15,9 +15,10 @@
 //
 //   gram_kernel         partial H_k for every group over up to 4 token slices,
 //                       in fp64 (fp16 products are exact in fp64), 16-byte
-//                       loads of X; one CTA per (group, tile of H, slice), so
-//                       the grid covers the SMs even for 32 groups.  HBM: X
-//                       read once per tile row of H.  2 T g d_in flop.
+//                       loads of X; one CTA per (group, tile of H on or above
+//                       the diagonal, slice), so the grid covers the SMs even
+//                       for 32 groups.  HBM: X read once per tile row of H.
+//                       2 T g d_in flop (3/4 of it at g = 128: H_k is symmetric).
 //   gram_reduce_kernel  H_k = fp32(sum of the slices in order): deterministic.
 //   clip_output_kernel  one CTA per (group, 64 rows): H_k staged in shared
 //                       memory; warp w takes 8 rows; per ratio each lane forms
@@ -60,9 +61,17 @@ gram_kernel(const __half* __restrict__ X, int64_t T, int64_t ld, int g, int64_t 
     __shared__ double sa[kT][TILE];
     __shared__ double sb[kT][TILE];
     pdl_wait();
+    // H_k is symmetric: only tiles ti <= tj are computed (tiles (tiles + 1) / 2
+    // per group), an off-diagonal one also written transposed
     const int tiles = g / TILE;
-    const int k = blockIdx.x / (tiles * tiles);
-    const int ti = (blockIdx.x / tiles) % tiles, tj = blockIdx.x % tiles;
+    const int pairs = tiles * (tiles + 1) / 2;
+    const int k = blockIdx.x / pairs;
+    int ti = 0, tj = blockIdx.x % pairs;
+    while (tj >= tiles - ti) {
+        tj -= tiles - ti;
+        ++ti;
+    }
+    tj += ti;
     const int64_t ca = (int64_t)k * g + ti * TILE, cb = (int64_t)k * g + tj * TILE;
     const int tx = threadIdx.x % (TILE / 4), ty = threadIdx.x / (TILE / 4);
     const int64_t t_begin = (int64_t)blockIdx.y * t_per;
@@ -104,13 +113,16 @@ gram_kernel(const __half* __restrict__ X, int64_t T, int64_t ld, int g, int64_t 
         __syncthreads();
     }
     pdl_launch_dependents();
-    // slice blockIdx.y of [slices][G][g][g]; gridDim.x / (tiles * tiles) = G
-    double* Hk = Hpart + ((int64_t)blockIdx.y * (gridDim.x / (tiles * tiles)) + k) * g * g;
+    // slice blockIdx.y of [slices][G][g][g]; gridDim.x / pairs = G
+    double* Hk = Hpart + ((int64_t)blockIdx.y * (gridDim.x / pairs) + k) * g * g;
 #pragma unroll
     for (int q = 0; q < 4; ++q)
 #pragma unroll
-        for (int r = 0; r < 4; ++r)
-            Hk[(int64_t)(ti * TILE + 4 * ty + q) * g + tj * TILE + 4 * tx + r] = acc[q][r];
+        for (int r = 0; r < 4; ++r) {
+            const int a_ = ti * TILE + 4 * ty + q, b_ = tj * TILE + 4 * tx + r;
+            Hk[(int64_t)a_ * g + b_] = acc[q][r];
+            if (ti != tj) Hk[(int64_t)b_ * g + a_] = acc[q][r];
+        }
 }
 
 // H = fp32(sum of the slices' partials, slices in order): deterministic.
@@ -395,7 +407,7 @@ cudaError_t launch_clip_search_output(const void* X, int64_t T, int64_t ld, cons
     const __half* Xh = static_cast<const __half*>(X);
     // token slices: about two CTAs per SM in all, at least 64 tokens a slice
     const int tiles = group_size == 32 ? 1 : group_size / 64;
-    const int64_t gram_ctas = G * tiles * tiles;
+    const int64_t gram_ctas = G * (tiles * (tiles + 1) / 2);
     int64_t slices = (2 * (int64_t)dev.num_sms + gram_ctas - 1) / gram_ctas;
     slices = std::max<int64_t>(1, std::min<int64_t>({slices, (int64_t)kMaxGramSlices, T / 64}));
     const int64_t t_per = ((T + slices - 1) / slices + 31) / 32 * 32;
