@@ -14,11 +14,15 @@
 // chosen ratios.
 //
 //   gram_kernel         partial H_k for every group over up to 4 token slices,
-//                       in fp64 (fp16 products are exact in fp64), 16-byte
-//                       loads of X; one CTA per (group, tile of H on or above
-//                       the diagonal, slice), so the grid covers the SMs even
-//                       for 32 groups.  HBM: X read once per tile row of H.
-//                       2 T g d_in flop (3/4 of it at g = 128: H_k is symmetric).
+//                       in fp64 (fp16 products are exact in fp64); X staged
+//                       two halves per thread and step, so a warp's shared-
+//                       memory stores are one contiguous run, and each lane
+//                       reads tile columns tx + (tile width / 4) r
+//                       (consecutive lanes, consecutive doubles); one
+//                       CTA per (group, tile of H on or above the diagonal,
+//                       slice), so the grid covers the SMs even for 32
+//                       groups.  HBM: X read once per tile row of H.  2 T g
+//                       d_in flop (3/4 of it at g = 128: H_k is symmetric).
 //   gram_reduce_kernel  H_k = fp32(sum of the slices in order): deterministic.
 //   clip_output_kernel  one CTA per (group, 64 rows): H_k staged in shared
 //                       memory; warp w takes 8 rows; per ratio each lane forms
@@ -57,9 +61,8 @@ gram_kernel(const __half* __restrict__ X, int64_t T, int64_t ld, int g, int64_t 
             double* __restrict__ Hpart) {
     constexpr int kT = 32;                      // tokens per staged chunk
     constexpr int kN = (TILE / 4) * (TILE / 4);
-    constexpr int kV = TILE / 8;                // 16-byte vectors per token row of a tile
-    __shared__ double sa[kT][TILE];
-    __shared__ double sb[kT][TILE];
+    __shared__ __align__(16) double sa[kT][TILE];   // 16-byte pairs are stored into it
+    __shared__ __align__(16) double sb[kT][TILE];
     pdl_wait();
     // H_k is symmetric: only tiles ti <= tj are computed (tiles (tiles + 1) / 2
     // per group), an off-diagonal one also written transposed
@@ -78,32 +81,32 @@ gram_kernel(const __half* __restrict__ X, int64_t T, int64_t ld, int g, int64_t 
     const int64_t t_end = min(T, t_begin + t_per);
     double acc[4][4] = {};
     for (int64_t t0 = t_begin; t0 < t_end; t0 += kT) {
-        for (int e = threadIdx.x; e < kT * kV; e += kN) {
-            const int tt = e / kV, c8 = e % kV;
+        // one half2 per thread and step: a warp stores one contiguous run of
+        // 16-byte pairs (no bank conflicts)
+        for (int e = threadIdx.x; e < kT * (TILE / 2); e += kN) {
+            const int tt = e / (TILE / 2), c2 = e % (TILE / 2);
             const bool in = t0 + tt < t_end;
-            const uint4 va = in ? __ldg(reinterpret_cast<const uint4*>(X + (t0 + tt) * ld + ca) + c8)
-                                : make_uint4(0, 0, 0, 0);
-            const uint4 vb = in ? __ldg(reinterpret_cast<const uint4*>(X + (t0 + tt) * ld + cb) + c8)
-                                : make_uint4(0, 0, 0, 0);
-            const uint32_t wa[4] = {va.x, va.y, va.z, va.w}, wb[4] = {vb.x, vb.y, vb.z, vb.w};
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const float2 fa = __half22float2(*reinterpret_cast<const __half2*>(&wa[q]));
-                const float2 fb = __half22float2(*reinterpret_cast<const __half2*>(&wb[q]));
-                sa[tt][8 * c8 + 2 * q] = (double)fa.x;
-                sa[tt][8 * c8 + 2 * q + 1] = (double)fa.y;
-                sb[tt][8 * c8 + 2 * q] = (double)fb.x;
-                sb[tt][8 * c8 + 2 * q + 1] = (double)fb.y;
-            }
+            const uint32_t ha = in ? __ldg(reinterpret_cast<const unsigned int*>(
+                                             X + (t0 + tt) * ld + ca) + c2)
+                                   : 0u;
+            const uint32_t hb = in ? __ldg(reinterpret_cast<const unsigned int*>(
+                                             X + (t0 + tt) * ld + cb) + c2)
+                                   : 0u;
+            const float2 fa = __half22float2(*reinterpret_cast<const __half2*>(&ha));
+            const float2 fb = __half22float2(*reinterpret_cast<const __half2*>(&hb));
+            *reinterpret_cast<double2*>(&sa[tt][2 * c2]) = make_double2(fa.x, fa.y);
+            *reinterpret_cast<double2*>(&sb[tt][2 * c2]) = make_double2(fb.x, fb.y);
         }
         __syncthreads();
 #pragma unroll 4
         for (int tt = 0; tt < kT; ++tt) {
+            // rows 4 ty + q (two per warp: broadcasts) against columns
+            // tx + (TILE / 4) r (consecutive lanes, consecutive doubles)
             double a[4], b[4];
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 a[q] = sa[tt][4 * ty + q];
-                b[q] = sb[tt][4 * tx + q];
+                b[q] = sb[tt][tx + (TILE / 4) * q];
             }
 #pragma unroll
             for (int q = 0; q < 4; ++q)
@@ -119,7 +122,7 @@ gram_kernel(const __half* __restrict__ X, int64_t T, int64_t ld, int g, int64_t 
     for (int q = 0; q < 4; ++q)
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
-            const int a_ = ti * TILE + 4 * ty + q, b_ = tj * TILE + 4 * tx + r;
+            const int a_ = ti * TILE + 4 * ty + q, b_ = tj * TILE + tx + (TILE / 4) * r;
             Hk[(int64_t)a_ * g + b_] = acc[q][r];
             if (ti != tj) Hk[(int64_t)b_ * g + a_] = acc[q][r];
         }
