@@ -166,7 +166,11 @@ def _check_clip_output(X, W, s, g, n_clip, idx_g, err_g):
 
 
 @pytest.mark.parametrize("d_out,d_in,T,g,n_clip", [(64, 256, 64, 32, 10), (200, 512, 96, 64, 20),
-                                                   (72, 384, 128, 128, 10), (8, 128, 1, 128, 3)])
+                                                   (72, 384, 128, 128, 10), (8, 128, 1, 128, 3),
+                                                   # Gram over 4 token slices, the last one
+                                                   # ragged (232 and 124 tokens)
+                                                   (96, 512, 1000, 64, 10),
+                                                   (136, 256, 700, 128, 10)])
 def test_clip_output_parity_small(d_out, d_in, T, g, n_clip):
     seed = d_out + d_in + T + g
     W = wl.weight(d_out, d_in, seed + 1)
