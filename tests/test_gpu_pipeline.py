@@ -135,6 +135,53 @@ def test_layer_streamer_with_clip_search():
                 assert np.array_equal(qz, qz_o)
 
 
+def test_layer_streamer_with_output_clip():
+    """Two layers streamed with the clip search scored on the output: for
+    every member the indices agree with the oracle's output-space clip at the
+    chosen scale (a differing index only where the two ratios' output scores
+    tie within 1e-5) and the packed output equals the oracle's pack of the
+    GPU's indices."""
+    g, n_grid, n_clip = 128, 20, 10
+    layers = [_small_layer(3000 + 10 * l) for l in range(2)]
+    host = [[([W.pin_memory() for W in Ws], X.pin_memory()) for Ws, X in lay]
+            for lay in layers]
+    st = pipeline.LayerStreamer(layers[0], "cuda", g, n_grid, False, n_clip=n_clip,
+                                clip_space="output")
+    out = [st.host_outputs() for _ in range(2)]
+    st.run(host, out)
+    torch.cuda.synchronize()
+    for lay, res in zip(layers, out):
+        for (Ws, X), (err, best, s, packs) in zip(lay, res):
+            Xn = X.numpy()
+            x = oracle.act_stats(Xn)
+            err_o, best_o, s_o = oracle.scale_search([W.numpy() for W in Ws], x, g, n_grid)
+            assert int(best[0]) == best_o
+            assert np.array_equal(s.numpy(), s_o)
+            Xd = Xn.astype(np.float64)
+            for W, pk in zip(Ws, packs):
+                qw, sc, qz, idx = (t.numpy() for t in pk)
+                idx_o, _ = oracle.clip_search_output(Xn, W.numpy(), s_o, g, n_clip)
+                diff = np.argwhere(idx != idx_o)
+                assert len(diff) <= max(2, idx_o.size // 1000)
+                for r, k in diff:
+                    cols = slice(k * g, (k + 1) * g)
+                    w = W.numpy()[r].astype(np.float32)
+
+                    def score(i):
+                        q, qs = oracle.fake_quant_group_clip(w[cols], s_o[cols],
+                                                             oracle.clip_ratio(int(i)))
+                        dw = (w[cols].astype(np.float64)
+                              - q.astype(np.float64) * qs / s_o[cols].astype(np.float64))
+                        y = Xd[:, cols] @ dw
+                        return float(y @ y)
+                    a, b = score(idx[r, k]), score(idx_o[r, k])
+                    assert abs(a - b) <= 1e-5 * b
+                qw_o, sc_o, qz_o = oracle.quantize_pack(W.numpy(), s_o, g, 8, idx)
+                assert np.array_equal(qw, qw_o)
+                assert np.array_equal(sc.view(np.uint16), sc_o.view(np.uint16))
+                assert np.array_equal(qz, qz_o)
+
+
 def test_norm_group_geomean_kernel_bit_exact():
     from post_int4_weight_b200 import awq
     rng = np.random.default_rng(61)
